@@ -1,0 +1,431 @@
+"""Benchmark: one layer of Prism dynamic sparse video self-attention at the 2K grid.
+
+A step is the whole hot path on one batch: plan (zone statistics, volumes and
+shapes, block-contiguous permutation, pooled scoring, Top-k U Top-p CSR),
+sparse attention forward, and sparse attention backward (dQ, dK, dV).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  `value` is effective TFLOP/s over the
+selected blocks (forward 4*D and backward 10*D FLOP per selected
+query-key token pair), summed over ranks; `ms_per_step` is ms per layer.
+Multi-GPU runs are independent replicas (the path has no exchange step).
+The reference arm times the fp64 CPU oracle on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn ms/layer fwd+bwd & effective TFLOP/s (selected blocks) at 2K grid"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"prism_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sms, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sms.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+# --------------------------------------------------------------------------
+def selected_pairs(view, D):
+    """sum over rows of |B_i| * sum_{j in S_i} |B_j| (token pairs), per sample."""
+    import torch
+    blk = view["blk_off"].long()
+    nbmax = view["nbmax"]
+    rp = view["row_ptr"].long()
+    col = view["col_idx"].long()
+    B = blk.shape[0]
+    rows = rp.numel() - 1
+    counts = rp[1:] - rp[:-1]
+    row_ids = torch.repeat_interleave(torch.arange(rows, device=rp.device), counts)
+    sample = row_ids // (rows // B)
+    i = row_ids % nbmax
+    sizes = blk[:, 1:] - blk[:, :-1]                     # [B, nbmax]
+    si = sizes[sample, i]
+    sj = sizes[sample, col]
+    return int((si * sj).sum().item())
+
+
+def kernel_bytes(name, w, nb, pairs_unused):
+    """Algorithmic HBM bytes of one launch of the plan kernels (one sample)."""
+    N, C, D, h = w.N, w.heads * w.head_dim, w.head_dim, w.heads
+    if name == "zone_stats_v":
+        return N * C * 2
+    if name == "permute_pool":
+        return 6 * N * C * 2 + 2 * h * nb * D * 8 + N * 4
+    if name == "select":
+        return 2 * h * nb * D * 8
+    if name == "attn_bwd_pre":
+        return 2 * N * C * 2 + N * C * 2 + h * N * 4
+    if name == "dq_finalize":
+        return h * N * D * 4 + N * C * 2
+    return None
+
+
+def run_ours(args, rank, world, dev):
+    import torch
+    import torch.distributed as dist
+    import dynamic_block_sparse_zone_b200 as P
+    from dynamic_block_sparse_zone_b200.synth import WORKLOADS, make_inputs
+
+    w = WORKLOADS[args.workload]
+    P.load_library()
+    inp = make_inputs(w, seed=0, device=dev, with_grad_output=True)
+    plan = P.PrismPlan(P.params_for(w))
+    shp = inp.Q.shape
+    O = torch.empty(shp, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.batch, w.heads, w.N), dtype=torch.float32, device=dev)
+    dQ, dK, dV = (torch.empty(shp, dtype=torch.bfloat16, device=dev) for _ in range(3))
+
+    def step(Q, K, V, a, dO):
+        plan.build(Q, K, V, a)
+        plan.fwd(O, lse)
+        plan.bwd(O, dO, dQ, dK, dV)
+
+    for _ in range(args.warmup):
+        step(inp.Q, inp.K, inp.V, inp.a, inp.dO)
+    torch.cuda.synchronize()
+    plan.check()
+    view = plan.view()
+    pairs = selected_pairs(view, w.head_dim)
+    nb = view["n_blocks"][0]
+    flops_fwd = 4.0 * w.head_dim * pairs
+    flops_bwd = 10.0 * w.head_dim * pairs
+    flops_step = flops_fwd + flops_bwd
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- device-resident timed region ----
+    plan.set_timing(True)
+    plan.read_timing()
+    clocks = ClockSampler(torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(inp.Q, inp.K, inp.V, inp.a, inp.dO)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    timing = plan.read_timing()
+    plan.set_timing(False)
+    plan.check()
+
+    # ---- end to end through the public API with pinned host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        host_in = [x.cpu().pin_memory() for x in (inp.Q, inp.K, inp.V, inp.a, inp.dO)]
+        host_out = [torch.empty(shp, dtype=torch.bfloat16).pin_memory() for _ in range(4)]
+        dev_in = [torch.empty_like(x, device=dev) for x in host_in]
+        h2d = sum(x.numel() * x.element_size() for x in host_in)
+        d2h = sum(x.numel() * x.element_size() for x in host_out)
+
+        def e2e_step():
+            for d, h in zip(dev_in, host_in):
+                d.copy_(h, non_blocking=True)
+            step(*dev_in)
+            for h, d in zip(host_out, (O, dQ, dK, dV)):
+                h.copy_(d, non_blocking=True)
+
+        for _ in range(max(1, args.warmup // 2)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1))
+        e2e = {"value": round(flops_step * args.steps * world / (ms_e2e * 1e-3) / 1e12, 3),
+               "unit": "TFLOP/s", "ms_per_step": round(ms_e2e / args.steps, 3),
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del host_in, host_out, dev_in
+
+    peaks, peak_src = load_peaks()
+    kernels = {}
+    total_k = sum(v[0] for v in timing.values()) or 1.0
+    for name, (tms, n) in timing.items():
+        if n == 0:
+            continue
+        avg = tms / n
+        rec = {"launches": n, "avg_ms": round(avg, 4), "share": round(tms / total_k, 4)}
+        if name == "attn_fwd":
+            rec["tflops"] = round(flops_fwd / (avg * 1e-3) / 1e12, 2)
+        elif name == "attn_bwd":
+            rec["tflops"] = round(flops_bwd / (avg * 1e-3) / 1e12, 2)
+        else:
+            by = kernel_bytes(name, w, nb, pairs)
+            if by:
+                rec["gbs"] = round(by / (avg * 1e-3) / 1e9, 1)
+        kernels[name] = rec
+    dom = max(kernels, key=lambda k: kernels[k]["share"])
+    if "tflops" in kernels[dom]:
+        peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        ach = kernels[dom]["tflops"]
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": round(ach / peak, 4), "peak_kind": f"bf16 dense sustained ({peak_src})",
+                "traffic": traffic_for(dom)}
+    else:
+        peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        ach = kernels[dom].get("gbs", 0.0)
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
+                "frac": round(ach / peak, 4), "peak_kind": f"HBM copy ({peak_src})", "traffic": traffic_for(dom)}
+    launches_per_step = sum(n * (9 if k == "csr_csc" else 1) for k, (t, n) in timing.items()) // max(args.steps, 1)
+    result = {
+        "metric": METRIC,
+        "value": round(flops_step * args.steps * world / (ms * 1e-3) / 1e12, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 3),
+        "ms_per_layer": round(ms / args.steps, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "grid": [w.T, w.H, w.W], "tokens": w.N, "heads": w.heads,
+                   "head_dim": w.head_dim, "top_k": w.top_k, "top_p": w.top_p, "max_frac": w.max_frac,
+                   "n_blocks": nb, "selected_token_pairs": pairs, "flops_per_step": flops_step,
+                   "l2": "inputs larger than L2 (Q,K,V,dO 2.26 GB each)", "parallelism": f"replicas x{world}"},
+        "kernels": kernels,
+        "roofline": roof,
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": e2e,
+        "clocks": clk,
+    }
+    plan.close()
+    return result
+
+
+def traffic_for(kernel):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
+    the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        rec = d.get(kernel)
+        if not rec:
+            return None
+        import hashlib
+        src = os.path.join(ROOT, "dynamic_block_sparse_zone_b200", "csrc", rec["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        return rec["bytes_per_launch"] if h == rec["source_sha"] else None
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+# --------------------------------------------------------------------------
+def oracle_setup(w, dev):
+    import numpy as np
+    import oracle
+    from dynamic_block_sparse_zone_b200.synth import bf16_bits, make_inputs
+    inp = make_inputs(w, seed=0, device=dev, with_grad_output=True)
+    bits = [bf16_bits(x[0]) for x in (inp.Q, inp.K, inp.V, inp.dO)]
+    a = inp.a[0].cpu().numpy()
+    del inp
+    t0 = time.time()
+    pl = oracle.plan(bits[0], bits[1], bits[2], a, w.T, w.H, w.W, w.heads, w.head_dim, w.top_k,
+                     float(np.float32(w.top_p)), float(np.float32(w.max_frac)), with_select=False)
+    head = [0]
+    cnt, cols, diag = oracle.select(pl.Qbar[head], pl.Kbar[head], w.top_k, float(np.float32(w.top_p)),
+                                    float(np.float32(w.max_frac)))
+    pl.cnt, pl.cols, pl.diag = cnt, cols, diag
+    pl.heads = 1
+    hb = [np.ascontiguousarray(x[:, head, :]) for x in bits]
+    plan_s = time.time() - t0
+    return pl, hb, plan_s
+
+
+def oracle_sample(pl, hb, w, rows, seed):
+    """fwd + dQ of `rows` query tokens of one head; returns (seconds, flops)."""
+    import numpy as np
+    import oracle
+    rs = np.random.default_rng(seed)
+    req_t = rs.integers(0, w.N, size=rows).astype(np.int32)
+    req_h = np.zeros(rows, np.int32)
+    sizes = pl.box[:, 3] * pl.box[:, 4] * pl.box[:, 5]
+    tok2blk = np.empty(w.N, np.int64)
+    off = pl.blk_off()
+    for j in range(pl.nb):
+        tok2blk[pl.perm[off[j]:off[j + 1]]] = j
+    keys = 0
+    for t in req_t:
+        i = tok2blk[t]
+        keys += int(sizes[pl.cols[0, i, :pl.cnt[0, i]]].sum())
+    t0 = time.time()
+    oracle.attn_fwd_rows(pl, hb[0], hb[1], hb[2], req_h, req_t)
+    oracle.attn_bwd_dq_rows(pl, hb[0], hb[1], hb[2], hb[3], req_h, req_t)
+    dt = time.time() - t0
+    # forward 4*D per pair; dQ needs S, dP and dQ: 6*D per pair
+    return dt, 10.0 * w.head_dim * keys
+
+
+def cpu_baseline(w, dev, rows):
+    import oracle
+    pl, hb, plan_s = oracle_setup(w, dev)
+    dt, fl = oracle_sample(pl, hb, w, rows, 123)
+    return {"value": round(fl / dt / 1e12, 8), "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle forward + dQ of {rows} random query tokens of head 0 on the same "
+                      f"workload ({dt:.1f} s); oracle plan with 1-head selection took {plan_s:.1f} s, not counted"}
+
+
+def run_reference(args, dev):
+    import oracle
+    from dynamic_block_sparse_zone_b200.synth import WORKLOADS
+    w = WORKLOADS[args.workload]
+    pl, hb, plan_s = oracle_setup(w, dev)
+    rows = args.ref_rows
+    for s in range(args.warmup):
+        oracle_sample(pl, hb, w, rows, 1000 + s)
+    tot_t, tot_f = 0.0, 0.0
+    for s in range(args.steps):
+        dt, fl = oracle_sample(pl, hb, w, rows, s)
+        tot_t += dt
+        tot_f += fl
+    val = tot_f / tot_t / 1e12
+    sample = (f"fp64 oracle forward + dQ of {rows} random query tokens of head 0 per step; "
+              f"oracle plan (1-head selection) {plan_s:.1f} s outside the timed steps")
+    return {"impl": "reference", "metric": METRIC, "value": round(val, 8), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name},
+            "cpu_baseline": {"value": round(val, 8), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(val, 8), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="latent2k_train_24x96x160")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=48)
+    ap.add_argument("--ref-rows", type=int, default=16)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    import torch
+    if args.impl == "reference":
+        if rank == 0:
+            dev = "cuda" if torch.cuda.is_available() else "cpu"
+            print(json.dumps(run_reference(args, dev)), flush=True)
+        return
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    res = run_ours(args, rank, world, dev)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            torch.cuda.empty_cache()
+            from dynamic_block_sparse_zone_b200.synth import WORKLOADS
+            res["cpu_baseline"] = cpu_baseline(WORKLOADS[args.workload], dev, args.cpu_rows)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,263 @@
+"""Thin Python binding of libprism.so (the C ABI in include/prism.h).
+
+Argument marshalling only: torch tensors provide device memory and the
+current CUDA stream; every step of the computation runs in the library's
+kernels.  There is no fallback: if the library is missing or a call fails, an
+exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libprism.so")
+
+PRISM_OK = 0
+_STATUS = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_UNSUPPORTED", 3: "PRISM_ERR_CUDA",
+           4: "PRISM_ERR_TIMEOUT", 5: "PRISM_ERR_NOMEM", 6: "PRISM_ERR_STATE"}
+
+EXPORTED = ("prism_plan_create", "prism_plan_bytes", "prism_plan_build", "prism_attn_fwd", "prism_attn_bwd",
+            "prism_plan_view_get", "prism_plan_check", "prism_plan_destroy", "prism_last_error",
+            "prism_plan_set_timing", "prism_plan_read_timing", "prism_timer_name")
+NUM_TIMERS = 10
+
+
+class PrismError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class prism_params(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+                ("heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("top_k", ctypes.c_int),
+                ("top_p", ctypes.c_float), ("max_frac", ctypes.c_float), ("fixed_shape", ctypes.c_int * 3),
+                ("eps", ctypes.c_double)]
+
+
+class prism_plan_view(ctypes.Structure):
+    _fields_ = [("zone_B", ctypes.c_void_p), ("zone_shape", ctypes.c_void_p), ("perm", ctypes.c_void_p),
+                ("blk_off", ctypes.c_void_p), ("row_ptr", ctypes.c_void_p), ("col_idx", ctypes.c_void_p),
+                ("nbmax", ctypes.c_int), ("nnz", ctypes.c_longlong), ("n_blocks", ctypes.c_int * 64)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libprism.so; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libprism.so not built ({path}); run python -m dynamic_block_sparse_zone_b200.build")
+    lib = ctypes.CDLL(path)
+    P, V = ctypes.c_void_p, ctypes.c_void_p
+    lib.prism_plan_create.argtypes = [ctypes.POINTER(prism_params), ctypes.POINTER(V)]
+    lib.prism_plan_bytes.argtypes = [ctypes.POINTER(prism_params)]
+    lib.prism_plan_bytes.restype = ctypes.c_size_t
+    lib.prism_plan_build.argtypes = [V, P, P, P, P, P]
+    lib.prism_attn_fwd.argtypes = [V, P, P, P]
+    lib.prism_attn_bwd.argtypes = [V, P, P, P, P, P, P]
+    lib.prism_plan_view_get.argtypes = [V, ctypes.POINTER(prism_plan_view), P]
+    lib.prism_plan_check.argtypes = [V, P]
+    lib.prism_plan_destroy.argtypes = [V]
+    lib.prism_plan_destroy.restype = None
+    lib.prism_last_error.restype = ctypes.c_char_p
+    lib.prism_plan_set_timing.argtypes = [V, ctypes.c_int]
+    lib.prism_plan_read_timing.argtypes = [V, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
+    lib.prism_timer_name.argtypes = [ctypes.c_int]
+    lib.prism_timer_name.restype = ctypes.c_char_p
+    for name in ("prism_plan_create", "prism_plan_build", "prism_attn_fwd", "prism_attn_bwd",
+                 "prism_plan_view_get", "prism_plan_check", "prism_plan_set_timing", "prism_plan_read_timing"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != PRISM_OK:
+        raise PrismError(status, load_library().prism_last_error().decode())
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape):
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor of shape {tuple(shape)}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+class _DevArray:
+    """Zero-copy view of device memory via __cuda_array_interface__."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr, "data": (ptr, True),
+                                         "version": 3, "strides": None}
+
+
+def _dev_tensor(ptr: int, shape, dtype=torch.int32) -> torch.Tensor:
+    ts = {torch.int32: "<i4"}[dtype]
+    return torch.as_tensor(_DevArray(ptr, shape, ts), device="cuda").clone()
+
+
+@dataclass
+class Params:
+    batch: int
+    T: int
+    H: int
+    W: int
+    heads: int
+    head_dim: int
+    top_k: int
+    top_p: float
+    max_frac: float = 0.0
+    fixed_shape: Tuple[int, int, int] = (0, 0, 0)
+    eps: float = 1e-6
+
+    def to_c(self) -> prism_params:
+        return prism_params(self.batch, self.T, self.H, self.W, self.heads, self.head_dim, self.top_k,
+                            float(self.top_p), float(self.max_frac), (ctypes.c_int * 3)(*self.fixed_shape),
+                            float(self.eps))
+
+    @property
+    def N(self) -> int:
+        return self.T * self.H * self.W
+
+
+def prism_plan_bytes(params: Params) -> int:
+    c = params.to_c()
+    return int(load_library().prism_plan_bytes(ctypes.byref(c)))
+
+
+class PrismPlan:
+    """Owns one prism_plan (C handle) and its device buffers."""
+
+    def __init__(self, params: Params):
+        self.params = params
+        self._c = params.to_c()
+        h = ctypes.c_void_p()
+        _check(load_library().prism_plan_create(ctypes.byref(self._c), ctypes.byref(h)))
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            load_library().prism_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- shapes -------------------------------------------------------------
+    def _qkv_shape(self):
+        p = self.params
+        return (p.batch, p.N, p.heads, p.head_dim)
+
+    # -- the three hot-path calls ---------------------------------------------
+    def build(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, a_norm: torch.Tensor):
+        p = self.params
+        for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+            _need(t, n, torch.bfloat16, self._qkv_shape())
+        _need(a_norm, "a_norm", torch.float32, (p.batch, p.T, p.H, p.W))
+        _check(load_library().prism_plan_build(self._h, _ptr(Q), _ptr(K), _ptr(V), _ptr(a_norm), _stream()))
+        return self
+
+    def fwd(self, O: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, want_lse: bool = True):
+        p = self.params
+        if O is None:
+            O = torch.empty(self._qkv_shape(), dtype=torch.bfloat16, device="cuda")
+        _need(O, "O", torch.bfloat16, self._qkv_shape())
+        if lse is None and want_lse:
+            lse = torch.empty((p.batch, p.heads, p.N), dtype=torch.float32, device="cuda")
+        if lse is not None:
+            _need(lse, "lse", torch.float32, (p.batch, p.heads, p.N))
+        _check(load_library().prism_attn_fwd(self._h, _ptr(O), _ptr(lse), _stream()))
+        return O, lse
+
+    def bwd(self, O: torch.Tensor, dO: torch.Tensor, dQ=None, dK=None, dV=None):
+        shp = self._qkv_shape()
+        _need(O, "O", torch.bfloat16, shp)
+        _need(dO, "dO", torch.bfloat16, shp)
+        dQ = torch.empty(shp, dtype=torch.bfloat16, device="cuda") if dQ is None else dQ
+        dK = torch.empty(shp, dtype=torch.bfloat16, device="cuda") if dK is None else dK
+        dV = torch.empty(shp, dtype=torch.bfloat16, device="cuda") if dV is None else dV
+        for t, n in ((dQ, "dQ"), (dK, "dK"), (dV, "dV")):
+            _need(t, n, torch.bfloat16, shp)
+        _check(load_library().prism_attn_bwd(self._h, _ptr(O), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _stream()))
+        return dQ, dK, dV
+
+    # -- per-kernel event timing ---------------------------------------------
+    def set_timing(self, enable: bool = True):
+        _check(load_library().prism_plan_set_timing(self._h, int(bool(enable))))
+
+    def read_timing(self) -> dict:
+        """{kernel name: (total ms, launches)} since the previous read (waits for the events)."""
+        lib = load_library()
+        ms = (ctypes.c_float * NUM_TIMERS)()
+        n = (ctypes.c_int * NUM_TIMERS)()
+        _check(lib.prism_plan_read_timing(self._h, ms, n))
+        return {lib.prism_timer_name(k).decode(): (float(ms[k]), int(n[k])) for k in range(NUM_TIMERS)}
+
+    # -- inspection ----------------------------------------------------------
+    def check(self):
+        _check(load_library().prism_plan_check(self._h, _stream()))
+
+    def view(self) -> dict:
+        """Copies of the plan's arrays (syncs the current stream)."""
+        v = prism_plan_view()
+        _check(load_library().prism_plan_view_get(self._h, ctypes.byref(v), _stream()))
+        p = self.params
+        M = p.N // 512
+        nbmax = v.nbmax
+        rows = p.batch * p.heads * nbmax
+        return dict(
+            zone_B=_dev_tensor(v.zone_B, (p.batch, M)),
+            zone_shape=_dev_tensor(v.zone_shape, (p.batch, M)),
+            perm=_dev_tensor(v.perm, (p.batch, p.N)),
+            blk_off=_dev_tensor(v.blk_off, (p.batch, nbmax + 1)),
+            row_ptr=_dev_tensor(v.row_ptr, (rows + 1,)),
+            col_idx=_dev_tensor(v.col_idx, (max(int(v.nnz), 1),))[: int(v.nnz)],
+            n_blocks=[int(v.n_blocks[b]) for b in range(p.batch)],
+            nbmax=nbmax,
+        )
+
+
+# Module-level names that mirror the C ABI.
+def prism_plan_create(params: Params) -> PrismPlan:
+    return PrismPlan(params)
+
+
+def prism_plan_build(plan: PrismPlan, Q, K, V, a_norm) -> PrismPlan:
+    return plan.build(Q, K, V, a_norm)
+
+
+def prism_attn_fwd(plan: PrismPlan, O=None, lse=None):
+    return plan.fwd(O, lse)
+
+
+def prism_attn_bwd(plan: PrismPlan, O, dO, dQ=None, dK=None, dV=None):
+    return plan.bwd(O, dO, dQ, dK, dV)
+
+
+def prism_plan_destroy(plan: PrismPlan):
+    plan.close()
+
+
+def params_for(w, batch: Optional[int] = None) -> Params:
+    """Params of a synth.Workload."""
+    return Params(batch=batch or w.batch, T=w.T, H=w.H, W=w.W, heads=w.heads, head_dim=w.head_dim,
+                  top_k=w.top_k, top_p=w.top_p, max_frac=w.max_frac, fixed_shape=tuple(w.fixed_shape))

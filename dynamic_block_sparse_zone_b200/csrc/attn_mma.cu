@@ -1,0 +1,631 @@
+// attn_mma.cu -- block-sparse attention forward / backward over the selected
+// key blocks, warp-level bf16 MMA (m16n8k16) with an online softmax.
+//
+// [Prism guide, Method section 3, last sentence]: each query block attends,
+// under one softmax, only to the key blocks of S_i.  Blocks are 64, 128 or 256
+// tokens and start at multiples of 64 in the block-contiguous order, so the
+// kernels work in 64-row tiles with no masking and no ragged tails.
+//
+// Forward : CTA = 4 warps = one 64-query tile; loops over the 64-key chunks of
+//           every selected key block (cp.async double buffer), S = QK^T,
+//           online softmax in registers (exp2 domain), O += P V.
+// Backward: key-stationary.  CTA = one 64-key tile; loops over the query
+//           tiles of every query block that selected this key block (block
+//           CSC), recomputes P from the forward's log-sum-exp, accumulates
+//           dK, dV in registers and adds dQ into an fp32 buffer.
+#include "prism_internal.cuh"
+
+namespace prism {
+
+namespace mma {
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int n>
+__device__ __forceinline__ void cp_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(n));
+}
+__device__ __forceinline__ void ldsm4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm4t(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Tile of 64 rows x D bf16 in shared memory; 16-byte chunks of a row are
+// XOR-swizzled with (row & 7) so that ldmatrix reads are conflict-free.
+template <int D>
+struct Tile {
+    static constexpr int kChunks = D / 8;
+    static constexpr int kBytes = 64 * D * 2;
+    __device__ static __forceinline__ uint32_t off(int row, int chunk) {
+        return (uint32_t)(row * D * 2 + ((chunk ^ (row & 7)) << 4));
+    }
+    // 64 rows starting at src (row stride D elements), 128 threads
+    __device__ static __forceinline__ void load(uint32_t base, const __nv_bfloat16 *src, int tid) {
+#pragma unroll
+        for (int it = 0; it < 64 * kChunks / 128; ++it) {
+            const int idx = it * 128 + tid;
+            const int row = idx / kChunks, ch = idx % kChunks;
+            cp_async16(base + off(row, ch), src + (size_t)row * D + ch * 8);
+        }
+    }
+};
+
+// Chunk walker over the selected key blocks of one row (or the selected query
+// blocks of one column): yields the first block-contiguous row of every 64-row
+// chunk in order.
+struct ChunkWalk {
+    const int *list;
+    const int *blk_off;
+    int u, u_end, r, r_end;
+    __device__ __forceinline__ void init(const int *l, int u0, int u1, const int *bo) {
+        list = l;
+        blk_off = bo;
+        u = u0;
+        u_end = u1;
+        r = r_end = 0;
+        if (u < u_end) {
+            const int j = list[u];
+            r = blk_off[j];
+            r_end = blk_off[j + 1];
+        }
+    }
+    __device__ __forceinline__ bool valid() const { return u < u_end; }
+    __device__ __forceinline__ int row() const { return r; }
+    __device__ __forceinline__ int block() const { return list[u]; }
+    __device__ __forceinline__ void next() {
+        r += kTile;
+        if (r >= r_end) {
+            ++u;
+            if (u < u_end) {
+                const int j = list[u];
+                r = blk_off[j];
+                r_end = blk_off[j + 1];
+            }
+        }
+    }
+};
+
+}  // namespace mma
+
+using namespace mma;
+
+// ---------------------------------------------------------------------------
+// forward
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128, 2)
+    k_attn_fwd_mma(Geo g, const __nv_bfloat16 *__restrict__ Qp, const __nv_bfloat16 *__restrict__ Kp,
+                   const __nv_bfloat16 *__restrict__ Vp, const int *__restrict__ blk_off,
+                   const int *__restrict__ tile_blk, const int *__restrict__ row_ptr, const int *__restrict__ col,
+                   const int *__restrict__ perm, __nv_bfloat16 *__restrict__ O, float *__restrict__ lse_user,
+                   float *__restrict__ lse_p, float scale_log2) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    using TL = Tile<D>;
+    const uint32_t sQ = smem_u32(smem);
+    // stage s: K at sQ + (1 + s) * kBytes, V at sQ + (3 + s) * kBytes
+    const uint32_t sK0 = sQ + TL::kBytes, sV0 = sQ + 3 * TL::kBytes;
+    const int tile = blockIdx.x, bh = blockIdx.y, b = bh / g.heads, h = bh % g.heads;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gr = lane >> 2, t4 = lane & 3, mi = lane >> 3, rr = lane & 7;
+    const int *bo = blk_off + (size_t)b * (g.nbmax + 1);
+    const int i = tile_blk[(size_t)b * g.nbmax + tile];
+    const size_t row = (size_t)bh * g.nbmax + i;
+    const __nv_bfloat16 *Qh = Qp + (size_t)bh * g.N * D;
+    const __nv_bfloat16 *Kh = Kp + (size_t)bh * g.N * D;
+    const __nv_bfloat16 *Vh = Vp + (size_t)bh * g.N * D;
+
+    ChunkWalk cw;
+    cw.init(col, row_ptr[row], row_ptr[row + 1], bo);
+    TL::load(sQ, Qh + (size_t)tile * 64 * D, tid);
+    TL::load(sK0, Kh + (size_t)cw.row() * D, tid);
+    TL::load(sV0, Vh + (size_t)cw.row() * D, tid);
+    cp_commit();
+
+    uint32_t qf[D / 16][4];
+    float o[D / 8][4];
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+
+    int stage = 0;
+    bool first = true;
+    while (cw.valid()) {
+        cp_wait<0>();
+        __syncthreads();
+        if (first) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                ldsm4(qf[kk], sQ + TL::off(warp * 16 + (mi & 1) * 8 + rr, kk * 2 + (mi >> 1)));
+            first = false;
+        }
+        ChunkWalk nx = cw;
+        nx.next();
+        if (nx.valid()) {
+            TL::load(sK0 + (stage ^ 1) * TL::kBytes, Kh + (size_t)nx.row() * D, tid);
+            TL::load(sV0 + (stage ^ 1) * TL::kBytes, Vh + (size_t)nx.row() * D, tid);
+        }
+        cp_commit();
+
+        // S = Q K^T for this warp's 16 rows x 64 keys
+        float s[8][4];
+#pragma unroll
+        for (int n = 0; n < 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t bfr[4];
+                ldsm4(bfr, sK0 + stage * TL::kBytes + TL::off(np * 16 + (mi >> 1) * 8 + rr, kk * 2 + (mi & 1)));
+                mma16816(s[2 * np], qf[kk], bfr[0], bfr[1]);
+                mma16816(s[2 * np + 1], qf[kk], bfr[2], bfr[3]);
+            }
+        }
+        // online softmax (rows gr and gr+8)
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int n = 0; n < 8; ++n) mx = fmaxf(mx, fmaxf(s[n][2 * rh], s[n][2 * rh + 1]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float mnew = fmaxf(mrow[rh], mx * scale_log2);
+            const float corr = exp2f(mrow[rh] - mnew);
+            mrow[rh] = mnew;
+            float sum = 0.f;
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                const float p0 = exp2f(s[n][2 * rh] * scale_log2 - mnew);
+                const float p1 = exp2f(s[n][2 * rh + 1] * scale_log2 - mnew);
+                s[n][2 * rh] = p0;
+                s[n][2 * rh + 1] = p1;
+                sum += p0 + p1;
+            }
+            lrow[rh] = lrow[rh] * corr + sum;
+#pragma unroll
+            for (int n = 0; n < D / 8; ++n) {
+                o[n][2 * rh] *= corr;
+                o[n][2 * rh + 1] *= corr;
+            }
+        }
+        // O += P V
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            uint32_t a[4];
+            a[0] = pack_bf16(s[2 * ks][0], s[2 * ks][1]);
+            a[1] = pack_bf16(s[2 * ks][2], s[2 * ks][3]);
+            a[2] = pack_bf16(s[2 * ks + 1][0], s[2 * ks + 1][1]);
+            a[3] = pack_bf16(s[2 * ks + 1][2], s[2 * ks + 1][3]);
+#pragma unroll
+            for (int dp = 0; dp < D / 16; ++dp) {
+                uint32_t bfr[4];
+                ldsm4t(bfr, sV0 + stage * TL::kBytes + TL::off(ks * 16 + (mi & 1) * 8 + rr, dp * 2 + (mi >> 1)));
+                mma16816(o[2 * dp], a, bfr[0], bfr[1]);
+                mma16816(o[2 * dp + 1], a, bfr[2], bfr[3]);
+            }
+        }
+        stage ^= 1;
+        cw = nx;
+    }
+    cp_wait<0>();
+
+    // normalise, stage through shared memory, store rows through perm
+#pragma unroll
+    for (int rh = 0; rh < 2; ++rh) {
+        float l = lrow[rh];
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        lrow[rh] = l;
+        const float inv = 1.f / l;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+            o[n][2 * rh] *= inv;
+            o[n][2 * rh + 1] *= inv;
+        }
+    }
+    __syncthreads();  // every warp is done with sQ's Q tile (fragments are in registers)
+    unsigned char *sOut = smem;
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+        const int r0 = warp * 16 + gr;
+        *reinterpret_cast<uint32_t *>(sOut + TL::off(r0, n) + t4 * 4) = pack_bf16(o[n][0], o[n][1]);
+        *reinterpret_cast<uint32_t *>(sOut + TL::off(r0 + 8, n) + t4 * 4) = pack_bf16(o[n][2], o[n][3]);
+    }
+    if (t4 == 0) {
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh) {
+            const int n = tile * 64 + warp * 16 + gr + rh * 8;
+            const float lse = (mrow[rh] + log2f(lrow[rh])) * 0.69314718055994531f;
+            lse_p[(size_t)bh * g.N + n] = lse;
+            if (lse_user) lse_user[(size_t)bh * g.N + perm[(size_t)b * g.N + n]] = lse;
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int it = 0; it < 16 * TL::kChunks / 32; ++it) {
+        const int idx = it * 32 + lane;
+        const int r = warp * 16 + idx / TL::kChunks, ch = idx % TL::kChunks;
+        const int n = tile * 64 + r;
+        const int tok = perm[(size_t)b * g.N + n];
+        const uint4 v = *reinterpret_cast<const uint4 *>(sOut + TL::off(r, ch));
+        *reinterpret_cast<uint4 *>(O + (((size_t)b * g.N + tok) * g.heads + h) * D + ch * 8) = v;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// backward, part 1: Delta = rowsum(dO * O) and the permuted copy of dO
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) k_attn_bwd_pre(Geo g, const __nv_bfloat16 *__restrict__ O,
+                                                      const __nv_bfloat16 *__restrict__ dO,
+                                                      const int *__restrict__ perm, __nv_bfloat16 *__restrict__ dOp,
+                                                      float *__restrict__ delta) {
+    constexpr int L = D / 8;  // lanes per (token, head)
+    const int b = blockIdx.y;
+    const int G = g.C / 8;
+    const size_t items = (size_t)kTile * G;
+    for (size_t it = threadIdx.x; it < items; it += blockDim.x) {
+        const int nl = (int)(it / G), grp = (int)(it % G);
+        const int n = blockIdx.x * kTile + nl;
+        const int tok = perm[(size_t)b * g.N + n];
+        const size_t src = ((size_t)b * g.N + tok) * g.C + grp * 8;
+        const uint4 ov = *reinterpret_cast<const uint4 *>(O + src);
+        const uint4 dv = *reinterpret_cast<const uint4 *>(dO + src);
+        const int hd = grp * 8 / D, d0 = grp * 8 % D;
+        const size_t bh = (size_t)b * g.heads + hd;
+        *reinterpret_cast<uint4 *>(dOp + (bh * g.N + n) * D + d0) = dv;
+        const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            acc += __uint_as_float(ow[k] << 16) * __uint_as_float(dw[k] << 16);
+            acc += __uint_as_float(ow[k] & 0xffff0000u) * __uint_as_float(dw[k] & 0xffff0000u);
+        }
+#pragma unroll
+        for (int o2 = L / 2; o2 > 0; o2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o2, L);
+        if ((threadIdx.x & (L - 1)) == 0) delta[bh * g.N + n] = acc;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// backward, part 2: key-stationary dK, dV; dQ accumulated in fp32
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128, 2)
+    k_attn_bwd_mma(Geo g, const __nv_bfloat16 *__restrict__ Qp, const __nv_bfloat16 *__restrict__ Kp,
+                   const __nv_bfloat16 *__restrict__ Vp, const __nv_bfloat16 *__restrict__ dOp,
+                   const float *__restrict__ lse_p, const float *__restrict__ delta,
+                   const int *__restrict__ blk_off, const int *__restrict__ tile_blk,
+                   const int *__restrict__ colT_ptr, const int *__restrict__ rowT, const int *__restrict__ perm,
+                   float *__restrict__ dQacc, __nv_bfloat16 *__restrict__ dK, __nv_bfloat16 *__restrict__ dV,
+                   float scale, float scale_log2) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    using TL = Tile<D>;
+    const uint32_t sK = smem_u32(smem), sV = sK + TL::kBytes;
+    // stage s: Q at sK + (2 + s) * kBytes, dO at sK + (4 + s) * kBytes
+    const uint32_t sQ0 = sK + 2 * TL::kBytes, sO0 = sK + 4 * TL::kBytes;
+    unsigned char *dS_bytes = smem + 6 * TL::kBytes;  // 64 keys x 64 queries bf16, swizzled rows of 128 B
+    const uint32_t sdS = sK + 6 * TL::kBytes;
+    float *sL = reinterpret_cast<float *>(smem + 6 * TL::kBytes + 64 * 64 * 2);  // [2][64]
+    float *sDl = sL + 128;                                                        // [2][64]
+
+    const int ktile = blockIdx.x, bh = blockIdx.y, b = bh / g.heads, h = bh % g.heads;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gr = lane >> 2, t4 = lane & 3, mi = lane >> 3, rr = lane & 7;
+    const int *bo = blk_off + (size_t)b * (g.nbmax + 1);
+    const int j = tile_blk[(size_t)b * g.nbmax + ktile];
+    const size_t colid = (size_t)bh * g.nbmax + j;
+    const __nv_bfloat16 *Qh = Qp + (size_t)bh * g.N * D;
+    const __nv_bfloat16 *dOh = dOp + (size_t)bh * g.N * D;
+    const float *Lh = lse_p + (size_t)bh * g.N;
+    const float *Dh = delta + (size_t)bh * g.N;
+    const float log2e = 1.4426950408889634f;
+
+    ChunkWalk cw;
+    cw.init(rowT, colT_ptr[colid], colT_ptr[colid + 1], bo);
+    TL::load(sK, Kp + ((size_t)bh * g.N + (size_t)ktile * 64) * D, tid);
+    TL::load(sV, Vp + ((size_t)bh * g.N + (size_t)ktile * 64) * D, tid);
+    if (cw.valid()) {
+        TL::load(sQ0, Qh + (size_t)cw.row() * D, tid);
+        TL::load(sO0, dOh + (size_t)cw.row() * D, tid);
+        if (tid < 64) {
+            sL[tid] = Lh[cw.row() + tid] * log2e;
+            sDl[tid] = Dh[cw.row() + tid];
+        }
+    }
+    cp_commit();
+
+    float dv[D / 8][4], dk[D / 8][4];
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dv[n][e] = dk[n][e] = 0.f;
+
+    int stage = 0;
+    while (cw.valid()) {
+        cp_wait<0>();
+        __syncthreads();
+        const int qrow0 = cw.row();
+        ChunkWalk nx = cw;
+        nx.next();
+        if (nx.valid()) {
+            TL::load(sQ0 + (stage ^ 1) * TL::kBytes, Qh + (size_t)nx.row() * D, tid);
+            TL::load(sO0 + (stage ^ 1) * TL::kBytes, dOh + (size_t)nx.row() * D, tid);
+            if (tid < 64) {
+                sL[(stage ^ 1) * 64 + tid] = Lh[nx.row() + tid] * log2e;
+                sDl[(stage ^ 1) * 64 + tid] = Dh[nx.row() + tid];
+            }
+        }
+        cp_commit();
+        const float *Ls = sL + stage * 64;
+        const float *Ds = sDl + stage * 64;
+
+        // S^T = K_w Q^T : 16 keys x 64 queries
+        float st[8][4];
+#pragma unroll
+        for (int n = 0; n < 8; ++n) st[n][0] = st[n][1] = st[n][2] = st[n][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            uint32_t a[4];
+            ldsm4(a, sK + TL::off(warp * 16 + (mi & 1) * 8 + rr, kk * 2 + (mi >> 1)));
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t bfr[4];
+                ldsm4(bfr, sQ0 + stage * TL::kBytes + TL::off(np * 16 + (mi >> 1) * 8 + rr, kk * 2 + (mi & 1)));
+                mma16816(st[2 * np], a, bfr[0], bfr[1]);
+                mma16816(st[2 * np + 1], a, bfr[2], bfr[3]);
+            }
+        }
+        // P^T = exp2(s * scale*log2e - LSE_q*log2e); the column index is the query
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            const int q = n * 8 + 2 * t4;
+            st[n][0] = exp2f(st[n][0] * scale_log2 - Ls[q]);
+            st[n][1] = exp2f(st[n][1] * scale_log2 - Ls[q + 1]);
+            st[n][2] = exp2f(st[n][2] * scale_log2 - Ls[q]);
+            st[n][3] = exp2f(st[n][3] * scale_log2 - Ls[q + 1]);
+        }
+        // dV += P^T dO
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            uint32_t a[4];
+            a[0] = pack_bf16(st[2 * ks][0], st[2 * ks][1]);
+            a[1] = pack_bf16(st[2 * ks][2], st[2 * ks][3]);
+            a[2] = pack_bf16(st[2 * ks + 1][0], st[2 * ks + 1][1]);
+            a[3] = pack_bf16(st[2 * ks + 1][2], st[2 * ks + 1][3]);
+#pragma unroll
+            for (int dp = 0; dp < D / 16; ++dp) {
+                uint32_t bfr[4];
+                ldsm4t(bfr, sO0 + stage * TL::kBytes + TL::off(ks * 16 + (mi & 1) * 8 + rr, dp * 2 + (mi >> 1)));
+                mma16816(dv[2 * dp], a, bfr[0], bfr[1]);
+                mma16816(dv[2 * dp + 1], a, bfr[2], bfr[3]);
+            }
+        }
+        // dP^T = V_w dO^T
+        float dpt[8][4];
+#pragma unroll
+        for (int n = 0; n < 8; ++n) dpt[n][0] = dpt[n][1] = dpt[n][2] = dpt[n][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            uint32_t a[4];
+            ldsm4(a, sV + TL::off(warp * 16 + (mi & 1) * 8 + rr, kk * 2 + (mi >> 1)));
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t bfr[4];
+                ldsm4(bfr, sO0 + stage * TL::kBytes + TL::off(np * 16 + (mi >> 1) * 8 + rr, kk * 2 + (mi & 1)));
+                mma16816(dpt[2 * np], a, bfr[0], bfr[1]);
+                mma16816(dpt[2 * np + 1], a, bfr[2], bfr[3]);
+            }
+        }
+        // dS^T = P^T (dP^T - Delta_q)
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            const int q = n * 8 + 2 * t4;
+            dpt[n][0] = st[n][0] * (dpt[n][0] - Ds[q]);
+            dpt[n][1] = st[n][1] * (dpt[n][1] - Ds[q + 1]);
+            dpt[n][2] = st[n][2] * (dpt[n][2] - Ds[q]);
+            dpt[n][3] = st[n][3] * (dpt[n][3] - Ds[q + 1]);
+        }
+        // dK += dS^T Q ; dS^T -> shared for dQ
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            uint32_t a[4];
+            a[0] = pack_bf16(dpt[2 * ks][0], dpt[2 * ks][1]);
+            a[1] = pack_bf16(dpt[2 * ks][2], dpt[2 * ks][3]);
+            a[2] = pack_bf16(dpt[2 * ks + 1][0], dpt[2 * ks + 1][1]);
+            a[3] = pack_bf16(dpt[2 * ks + 1][2], dpt[2 * ks + 1][3]);
+            // rows warp*16+gr (+8), query columns ks*16 + 2t4 (+8): chunk = 2ks (+1)
+            const int r0 = warp * 16 + gr;
+            *reinterpret_cast<uint32_t *>(dS_bytes + r0 * 128 + (((2 * ks) ^ (r0 & 7)) << 4) + t4 * 4) = a[0];
+            *reinterpret_cast<uint32_t *>(dS_bytes + (r0 + 8) * 128 + (((2 * ks) ^ ((r0 + 8) & 7)) << 4) + t4 * 4) =
+                a[1];
+            *reinterpret_cast<uint32_t *>(dS_bytes + r0 * 128 + (((2 * ks + 1) ^ (r0 & 7)) << 4) + t4 * 4) = a[2];
+            *reinterpret_cast<uint32_t *>(dS_bytes + (r0 + 8) * 128 + (((2 * ks + 1) ^ ((r0 + 8) & 7)) << 4) +
+                                          t4 * 4) = a[3];
+#pragma unroll
+            for (int dp = 0; dp < D / 16; ++dp) {
+                uint32_t bfr[4];
+                ldsm4t(bfr, sQ0 + stage * TL::kBytes + TL::off(ks * 16 + (mi & 1) * 8 + rr, dp * 2 + (mi >> 1)));
+                mma16816(dk[2 * dp], a, bfr[0], bfr[1]);
+                mma16816(dk[2 * dp + 1], a, bfr[2], bfr[3]);
+            }
+        }
+        __syncthreads();
+        // dQ rows warp*16.. (+16) = dS (16 queries x 64 keys) K, in two halves of D
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float dq[D / 16][4];
+#pragma unroll
+            for (int n = 0; n < D / 16; ++n) dq[n][0] = dq[n][1] = dq[n][2] = dq[n][3] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                uint32_t a[4];
+                {
+                    const int key = ks * 16 + (mi >> 1) * 8 + rr;
+                    const int qc = warp * 2 + (mi & 1);
+                    ldsm4t(a, sdS + key * 128 + ((qc ^ (key & 7)) << 4));
+                }
+#pragma unroll
+                for (int dp = 0; dp < D / 32; ++dp) {
+                    uint32_t bfr[4];
+                    const int dpg = half * (D / 32) + dp;
+                    ldsm4t(bfr, sK + TL::off(ks * 16 + (mi & 1) * 8 + rr, dpg * 2 + (mi >> 1)));
+                    mma16816(dq[2 * dp], a, bfr[0], bfr[1]);
+                    mma16816(dq[2 * dp + 1], a, bfr[2], bfr[3]);
+                }
+            }
+            float *dst = dQacc + ((size_t)bh * g.N + qrow0 + warp * 16 + gr) * D + half * (D / 2);
+#pragma unroll
+            for (int n = 0; n < D / 16; ++n) {
+                atomicAdd(dst + n * 8 + 2 * t4, dq[n][0] * scale);
+                atomicAdd(dst + n * 8 + 2 * t4 + 1, dq[n][1] * scale);
+                atomicAdd(dst + 8 * D + n * 8 + 2 * t4, dq[n][2] * scale);
+                atomicAdd(dst + 8 * D + n * 8 + 2 * t4 + 1, dq[n][3] * scale);
+            }
+        }
+        stage ^= 1;
+        cw = nx;
+    }
+    cp_wait<0>();
+    __syncthreads();
+    // dK (scaled), dV -> shared (reuse the Q stages) -> user layout through perm
+    unsigned char *sOutK = smem + 2 * TL::kBytes;
+    unsigned char *sOutV = smem + 3 * TL::kBytes;
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+        const int r0 = warp * 16 + gr;
+        *reinterpret_cast<uint32_t *>(sOutK + TL::off(r0, n) + t4 * 4) = pack_bf16(dk[n][0] * scale, dk[n][1] * scale);
+        *reinterpret_cast<uint32_t *>(sOutK + TL::off(r0 + 8, n) + t4 * 4) =
+            pack_bf16(dk[n][2] * scale, dk[n][3] * scale);
+        *reinterpret_cast<uint32_t *>(sOutV + TL::off(r0, n) + t4 * 4) = pack_bf16(dv[n][0], dv[n][1]);
+        *reinterpret_cast<uint32_t *>(sOutV + TL::off(r0 + 8, n) + t4 * 4) = pack_bf16(dv[n][2], dv[n][3]);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int it = 0; it < 16 * TL::kChunks / 32; ++it) {
+        const int idx = it * 32 + lane;
+        const int r = warp * 16 + idx / TL::kChunks, ch = idx % TL::kChunks;
+        const int tok = perm[(size_t)b * g.N + (size_t)ktile * 64 + r];
+        const size_t dst = (((size_t)b * g.N + tok) * g.heads + h) * D + ch * 8;
+        *reinterpret_cast<uint4 *>(dK + dst) = *reinterpret_cast<const uint4 *>(sOutK + TL::off(r, ch));
+        *reinterpret_cast<uint4 *>(dV + dst) = *reinterpret_cast<const uint4 *>(sOutV + TL::off(r, ch));
+    }
+}
+
+// dQ (fp32, permuted, head-major) -> bf16 user layout
+template <int D>
+__global__ void __launch_bounds__(256) k_dq_finalize(Geo g, const float *__restrict__ dQacc,
+                                                     const int *__restrict__ perm, __nv_bfloat16 *__restrict__ dQ) {
+    const int b = blockIdx.y;
+    const int G = g.C / 8;
+    const size_t items = (size_t)kTile * G;
+    for (size_t it = threadIdx.x; it < items; it += blockDim.x) {
+        const int nl = (int)(it / G), grp = (int)(it % G);
+        const int n = blockIdx.x * kTile + nl;
+        const int hd = grp * 8 / D, d0 = grp * 8 % D;
+        const size_t bh = (size_t)b * g.heads + hd;
+        const float4 *src = reinterpret_cast<const float4 *>(dQacc + (bh * g.N + n) * D + d0);
+        const float4 x = src[0], y = src[1];
+        uint4 v;
+        v.x = pack_bf16(x.x, x.y);
+        v.y = pack_bf16(x.z, x.w);
+        v.z = pack_bf16(y.x, y.y);
+        v.w = pack_bf16(y.z, y.w);
+        const int tok = perm[(size_t)b * g.N + n];
+        *reinterpret_cast<uint4 *>(dQ + ((size_t)b * g.N + tok) * g.C + grp * 8) = v;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+template <int D>
+static constexpr size_t fwd_smem() {
+    return 5 * Tile<D>::kBytes;
+}
+template <int D>
+static constexpr size_t bwd_smem() {
+    return 6 * Tile<D>::kBytes + 64 * 64 * 2 + 4 * 64 * sizeof(float);
+}
+
+template <int D>
+static prism_status fwd_impl(Plan &pl, void *O, float *lse, cudaStream_t st) {
+    const Geo &g = pl.g;
+    const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+    TimerScope ts(pl, kTAttnFwd, st);
+    k_attn_fwd_mma<D><<<dim3(g.nbmax, g.batch * g.heads), 128, fwd_smem<D>(), st>>>(
+        g, pl.Qp, pl.Kp, pl.Vp, pl.blk_off, pl.tile_blk, pl.row_ptr, pl.col, pl.perm,
+        static_cast<__nv_bfloat16 *>(O), lse, pl.lse_p, scale_log2);
+    PRISM_CUDA_OK(cudaGetLastError());
+    return PRISM_OK;
+}
+
+template <int D>
+static prism_status bwd_impl(Plan &pl, const void *O, const void *dO, void *dQ, void *dK, void *dV,
+                             cudaStream_t st) {
+    const Geo &g = pl.g;
+    const double scale = 1.0 / sqrt((double)D);
+    PRISM_CUDA_OK(cudaMemsetAsync(pl.dQacc, 0, (size_t)g.batch * g.heads * g.N * D * sizeof(float), st));
+    {
+    TimerScope ts(pl, kTBwdPre, st);
+    k_attn_bwd_pre<D><<<dim3(g.nbmax, g.batch), 256, 0, st>>>(g, static_cast<const __nv_bfloat16 *>(O),
+                                                             static_cast<const __nv_bfloat16 *>(dO), pl.perm,
+                                                             pl.dOp, pl.delta);
+    }
+    {
+    TimerScope ts(pl, kTAttnBwd, st);
+    k_attn_bwd_mma<D><<<dim3(g.nbmax, g.batch * g.heads), 128, bwd_smem<D>(), st>>>(
+        g, pl.Qp, pl.Kp, pl.Vp, pl.dOp, pl.lse_p, pl.delta, pl.blk_off, pl.tile_blk, pl.colT_ptr, pl.rowT,
+        pl.perm, pl.dQacc, static_cast<__nv_bfloat16 *>(dK), static_cast<__nv_bfloat16 *>(dV), (float)scale,
+        (float)(scale * 1.4426950408889634));
+    }
+    TimerScope ts(pl, kTDqFinal, st);
+    k_dq_finalize<D><<<dim3(g.nbmax, g.batch), 256, 0, st>>>(g, pl.dQacc, pl.perm,
+                                                            static_cast<__nv_bfloat16 *>(dQ));
+    PRISM_CUDA_OK(cudaGetLastError());
+    return PRISM_OK;
+}
+
+prism_status configure_attn_kernels() {
+    PRISM_CUDA_OK(cudaFuncSetAttribute(k_attn_fwd_mma<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)fwd_smem<64>()));
+    PRISM_CUDA_OK(cudaFuncSetAttribute(k_attn_fwd_mma<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)fwd_smem<128>()));
+    PRISM_CUDA_OK(cudaFuncSetAttribute(k_attn_bwd_mma<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)bwd_smem<64>()));
+    PRISM_CUDA_OK(cudaFuncSetAttribute(k_attn_bwd_mma<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)bwd_smem<128>()));
+    return PRISM_OK;
+}
+
+prism_status launch_attn_fwd(Plan &pl, void *O, float *lse, cudaStream_t st) {
+    return pl.g.D == 64 ? fwd_impl<64>(pl, O, lse, st) : fwd_impl<128>(pl, O, lse, st);
+}
+
+prism_status launch_attn_bwd(Plan &pl, const void *O, const void *dO, void *dQ, void *dK, void *dV,
+                             cudaStream_t st) {
+    return pl.g.D == 64 ? bwd_impl<64>(pl, O, dO, dQ, dK, dV, st) : bwd_impl<128>(pl, O, dO, dQ, dK, dV, st);
+}
+
+}  // namespace prism

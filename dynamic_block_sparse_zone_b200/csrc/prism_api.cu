@@ -1,0 +1,405 @@
+// prism_api.cu -- the C ABI declared in include/prism.h: parameter checks,
+// plan allocation and the three hot-path calls.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <new>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "prism_internal.cuh"
+
+namespace prism {
+
+static thread_local std::string g_last_error;
+
+prism_status fail(prism_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+prism_status fail_cuda(cudaError_t e, const char *what, const char *file, int line) {
+    const prism_status s = (e == cudaErrorMemoryAllocation) ? PRISM_ERR_NOMEM : PRISM_ERR_CUDA;
+    return fail(s, "%s failed: %s (%s:%d)", what, cudaGetErrorString(e), file, line);
+}
+
+int host_shape_table(int (*e)[3]);
+prism_status configure_plan_kernels(const Plan &pl);
+prism_status configure_attn_kernels();
+size_t select_smem_bytes(const Plan &pl);
+
+static int log2_exact(int x) {
+    for (int k = 0; k < 31; ++k)
+        if ((1 << k) == x) return k;
+    return -1;
+}
+
+// Validates params and fills geometry; returns PRISM_OK or an error with a message.
+static prism_status check_params(const prism_params *p, Geo *g, int *fixed_idx, int *cap_stride) {
+    if (!p) return fail(PRISM_ERR_INVALID_ARG, "params is NULL");
+    if (p->batch < 1 || p->batch > 64) return fail(PRISM_ERR_INVALID_ARG, "batch must be in [1, 64]");
+    if (p->T <= 0 || p->H <= 0 || p->W <= 0) return fail(PRISM_ERR_INVALID_ARG, "grid sizes must be positive");
+    if (p->T % 8 || p->H % 8 || p->W % 8)
+        return fail(PRISM_ERR_UNSUPPORTED, "grid T x H x W = %d x %d x %d is not a multiple of the 8x8x8 macro-zone",
+                    p->T, p->H, p->W);
+    if (p->heads < 1) return fail(PRISM_ERR_INVALID_ARG, "heads must be >= 1");
+    if (p->head_dim != 64 && p->head_dim != 128)
+        return fail(PRISM_ERR_UNSUPPORTED, "head_dim %d unsupported (64 or 128)", p->head_dim);
+    if (p->top_k < 1) return fail(PRISM_ERR_INVALID_ARG, "top_k must be >= 1");
+    if (!(p->top_p > 0.0f && p->top_p <= 1.0f)) return fail(PRISM_ERR_INVALID_ARG, "top_p must be in (0, 1]");
+    if (!(p->max_frac >= 0.0f && p->max_frac <= 1.0f)) return fail(PRISM_ERR_INVALID_ARG, "max_frac must be in [0, 1]");
+    const long long N = (long long)p->T * p->H * p->W;
+    if (N > (1ll << 26)) return fail(PRISM_ERR_UNSUPPORTED, "grid too large (N = %lld tokens)", N);
+    *fixed_idx = -1;
+    const int *fs = p->fixed_shape;
+    if (fs[0] || fs[1] || fs[2]) {
+        const int e0 = log2_exact(fs[0]), e1 = log2_exact(fs[1]), e2 = log2_exact(fs[2]);
+        int table[kNumShapes][3];
+        host_shape_table(table);
+        for (int c = 0; c < kNumShapes; ++c)
+            if (table[c][0] == e0 && table[c][1] == e1 && table[c][2] == e2) *fixed_idx = c;
+        if (*fixed_idx < 0)
+            return fail(PRISM_ERR_INVALID_ARG, "fixed_shape %dx%dx%d is not one of the 16 candidates", fs[0], fs[1],
+                        fs[2]);
+    }
+    g->batch = p->batch;
+    g->T = p->T;
+    g->H = p->H;
+    g->W = p->W;
+    g->heads = p->heads;
+    g->D = p->head_dim;
+    g->N = (int)N;
+    g->MT = p->T / 8;
+    g->MH = p->H / 8;
+    g->MW = p->W / 8;
+    g->M = g->MT * g->MH * g->MW;
+    g->nbmax = g->N / 64;
+    g->C = p->heads * p->head_dim;
+    *cap_stride = cap_for(g->nbmax, p->top_k, p->max_frac);
+    const long long rows = (long long)g->batch * g->heads * g->nbmax;
+    if (rows * (long long)*cap_stride >= (1ll << 31))
+        return fail(PRISM_ERR_UNSUPPORTED, "selection too large for 32-bit CSR offsets (%lld x %d)", rows, *cap_stride);
+    if ((long long)g->batch * g->heads * g->N * g->D >= (1ll << 40))
+        return fail(PRISM_ERR_UNSUPPORTED, "tensors too large");
+    return PRISM_OK;
+}
+
+struct Alloc {
+    void **ptr;
+    size_t bytes;
+};
+
+static size_t plan_allocs(Plan &pl, Alloc *out) {
+    const Geo &g = pl.g;
+    const size_t BH = (size_t)g.batch * g.heads, rows = BH * g.nbmax;
+    const int nchunk = (g.C + kStatChunk - 1) / kStatChunk;
+    const size_t nnz = rows * (size_t)pl.cap_stride;
+    size_t n = 0;
+    auto add = [&](void **p, size_t b) { out[n++] = Alloc{p, b}; };
+    add((void **)&pl.zone_part, (size_t)g.batch * g.M * nchunk * 3 * sizeof(double));
+    add((void **)&pl.zone_a, (size_t)g.batch * g.M * 5 * sizeof(double));
+    add((void **)&pl.zone_B, (size_t)g.batch * g.M * sizeof(int));
+    add((void **)&pl.zone_shape, (size_t)g.batch * g.M * sizeof(int));
+    add((void **)&pl.zone_blk0, (size_t)g.batch * (g.M + 1) * sizeof(int));
+    add((void **)&pl.nb, (size_t)g.batch * sizeof(int));
+    add((void **)&pl.blk_off, (size_t)g.batch * (g.nbmax + 1) * sizeof(int));
+    add((void **)&pl.tile_blk, (size_t)g.batch * g.nbmax * sizeof(int));
+    add((void **)&pl.perm, (size_t)g.batch * g.N * sizeof(int));
+    add((void **)&pl.Qp, BH * g.N * g.D * 2);
+    add((void **)&pl.Kp, BH * g.N * g.D * 2);
+    add((void **)&pl.Vp, BH * g.N * g.D * 2);
+    add((void **)&pl.Qbar, rows * g.D * sizeof(double));
+    add((void **)&pl.Kbar, rows * g.D * sizeof(double));
+    add((void **)&pl.cnt, rows * sizeof(int));
+    add((void **)&pl.cols_pad, nnz * sizeof(int));
+    add((void **)&pl.row_ptr, (rows + 1) * sizeof(int));
+    add((void **)&pl.col, nnz * sizeof(int));
+    add((void **)&pl.colT_ptr, (rows + 1) * sizeof(int));
+    add((void **)&pl.rowT, nnz * sizeof(int));
+    add((void **)&pl.colT_cursor, rows * sizeof(int));
+    add((void **)&pl.scan_tmp, ((rows + 1023) / 1024 + 1) * sizeof(int));
+    add((void **)&pl.lse_p, BH * g.N * sizeof(float));
+    add((void **)&pl.dOp, BH * g.N * g.D * 2);
+    add((void **)&pl.delta, BH * g.N * sizeof(float));
+    add((void **)&pl.dQacc, BH * g.N * g.D * sizeof(float));
+    add((void **)&pl.status, 16 * sizeof(int));
+    return n;
+}
+
+// ---------------------------------------------------------------------------
+// per-kernel event timing
+// ---------------------------------------------------------------------------
+struct TimerState {
+    std::vector<cudaEvent_t> pool;                              // free events
+    std::vector<std::pair<cudaEvent_t, cudaEvent_t>> rec[kTCount];
+    cudaEvent_t take() {
+        if (pool.empty()) {
+            cudaEvent_t e;
+            if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+            return e;
+        }
+        cudaEvent_t e = pool.back();
+        pool.pop_back();
+        return e;
+    }
+    ~TimerState() {
+        for (auto e : pool) cudaEventDestroy(e);
+        for (auto &v : rec)
+            for (auto &pr : v) {
+                cudaEventDestroy(pr.first);
+                cudaEventDestroy(pr.second);
+            }
+    }
+};
+
+TimerScope::TimerScope(Plan &p, int i, cudaStream_t s) : pl(p), id(i), st(s) {
+    if (!pl.timers) return;
+    cudaEvent_t a = pl.timers->take(), b = pl.timers->take();
+    if (!a || !b) return;
+    cudaEventRecord(a, st);
+    pl.timers->rec[id].push_back({a, b});
+}
+
+TimerScope::~TimerScope() {
+    if (!pl.timers || pl.timers->rec[id].empty()) return;
+    cudaEventRecord(pl.timers->rec[id].back().second, st);
+}
+
+static void release_buffers(Plan &pl) {
+    Alloc a[64];
+    const size_t n = plan_allocs(pl, a);
+    for (size_t k = 0; k < n; ++k)
+        if (*a[k].ptr) {
+            cudaFree(*a[k].ptr);
+            *a[k].ptr = nullptr;
+        }
+    if (pl.host_nb) {
+        cudaFreeHost(pl.host_nb);
+        pl.host_nb = nullptr;
+    }
+    delete pl.timers;
+    pl.timers = nullptr;
+}
+
+}  // namespace prism
+
+using namespace prism;
+
+struct prism_plan {
+    Plan pl;
+};
+
+extern "C" {
+
+const char *prism_last_error(void) { return g_last_error.c_str(); }
+
+size_t prism_plan_bytes(const prism_params *params) {
+    Plan pl;
+    memset(&pl, 0, sizeof pl);
+    if (check_params(params, &pl.g, &pl.fixed_idx, &pl.cap_stride) != PRISM_OK) return 0;
+    Alloc a[64];
+    const size_t n = plan_allocs(pl, a);
+    size_t tot = 0;
+    for (size_t k = 0; k < n; ++k) tot += (a[k].bytes + 255) & ~(size_t)255;
+    return tot;
+}
+
+prism_status prism_plan_create(const prism_params *params, prism_plan **out) {
+    g_last_error.clear();
+    if (!out) return fail(PRISM_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    prism_plan *h = new (std::nothrow) prism_plan;
+    if (!h) return fail(PRISM_ERR_NOMEM, "host allocation failed");
+    memset(&h->pl, 0, sizeof h->pl);
+    Plan &pl = h->pl;
+    prism_status s = check_params(params, &pl.g, &pl.fixed_idx, &pl.cap_stride);
+    if (s != PRISM_OK) {
+        delete h;
+        return s;
+    }
+    pl.p = *params;
+    if (!(pl.p.eps > 0.0)) pl.p.eps = 1e-6;
+    if (select_smem_bytes(pl) > 220 * 1024) {
+        delete h;
+        return fail(PRISM_ERR_UNSUPPORTED, "selection working set (%zu bytes of shared memory) too large",
+                    select_smem_bytes(pl));
+    }
+    cudaError_t e = cudaGetDevice(&pl.device);
+    if (e != cudaSuccess) {
+        delete h;
+        return fail_cuda(e, "cudaGetDevice", __FILE__, __LINE__);
+    }
+    Alloc a[64];
+    const size_t n = plan_allocs(pl, a);
+    for (size_t k = 0; k < n; ++k) *a[k].ptr = nullptr;
+    for (size_t k = 0; k < n; ++k) {
+        e = cudaMalloc(a[k].ptr, a[k].bytes);
+        if (e != cudaSuccess) {
+            *a[k].ptr = nullptr;
+            release_buffers(pl);
+            delete h;
+            return fail_cuda(e, "cudaMalloc", __FILE__, __LINE__);
+        }
+    }
+    e = cudaMallocHost((void **)&pl.host_nb, 64 * sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(pl.status, 0, 16 * sizeof(int));
+    if (e != cudaSuccess) {
+        release_buffers(pl);
+        delete h;
+        return fail_cuda(e, "plan setup", __FILE__, __LINE__);
+    }
+    s = configure_plan_kernels(pl);
+    if (s == PRISM_OK) s = configure_attn_kernels();
+    if (s != PRISM_OK) {
+        release_buffers(pl);
+        delete h;
+        return s;
+    }
+    *out = h;
+    return PRISM_OK;
+}
+
+void prism_plan_destroy(prism_plan *plan) {
+    if (!plan) return;
+    release_buffers(plan->pl);
+    delete plan;
+}
+
+static prism_status device_guard(const Plan &pl) {
+    int cur = -1;
+    PRISM_CUDA_OK(cudaGetDevice(&cur));
+    if (cur != pl.device)
+        return fail(PRISM_ERR_INVALID_ARG, "current device %d is not the plan's device %d", cur, pl.device);
+    return PRISM_OK;
+}
+
+prism_status prism_plan_build(prism_plan *plan, const void *Q, const void *K, const void *V, const float *a_norm,
+                              void *stream) {
+    g_last_error.clear();
+    if (!plan || !Q || !K || !V || !a_norm) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_plan_build");
+    prism_status s = device_guard(plan->pl);
+    if (s != PRISM_OK) return s;
+    const uintptr_t al = (uintptr_t)Q | (uintptr_t)K | (uintptr_t)V;
+    if (al & 15) return fail(PRISM_ERR_INVALID_ARG, "Q, K, V must be 16-byte aligned");
+    plan->pl.have_fwd = false;
+    return launch_plan(plan->pl, Q, K, V, a_norm, static_cast<cudaStream_t>(stream));
+}
+
+prism_status prism_attn_fwd(prism_plan *plan, void *O, float *lse, void *stream) {
+    g_last_error.clear();
+    if (!plan || !O) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_attn_fwd");
+    prism_status s = device_guard(plan->pl);
+    if (s != PRISM_OK) return s;
+    if ((uintptr_t)O & 15) return fail(PRISM_ERR_INVALID_ARG, "O must be 16-byte aligned");
+    s = launch_attn_fwd(plan->pl, O, lse, static_cast<cudaStream_t>(stream));
+    if (s == PRISM_OK) plan->pl.have_fwd = true;
+    return s;
+}
+
+prism_status prism_attn_bwd(prism_plan *plan, const void *O, const void *dO, void *dQ, void *dK, void *dV,
+                            void *stream) {
+    g_last_error.clear();
+    if (!plan || !O || !dO || !dQ || !dK || !dV) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_attn_bwd");
+    prism_status s = device_guard(plan->pl);
+    if (s != PRISM_OK) return s;
+    if (!plan->pl.have_fwd) return fail(PRISM_ERR_STATE, "prism_attn_bwd needs a prism_attn_fwd after the build");
+    const uintptr_t al = (uintptr_t)O | (uintptr_t)dO | (uintptr_t)dQ | (uintptr_t)dK | (uintptr_t)dV;
+    if (al & 15) return fail(PRISM_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+    return launch_attn_bwd(plan->pl, O, dO, dQ, dK, dV, static_cast<cudaStream_t>(stream));
+}
+
+prism_status prism_plan_view_get(prism_plan *plan, prism_plan_view *view, void *stream) {
+    g_last_error.clear();
+    if (!plan || !view) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_plan_view_get");
+    Plan &pl = plan->pl;
+    prism_status s = device_guard(pl);
+    if (s != PRISM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t rows = (size_t)pl.g.batch * pl.g.heads * pl.g.nbmax;
+    int nnz = 0;
+    PRISM_CUDA_OK(cudaMemcpyAsync(pl.host_nb, pl.nb, pl.g.batch * sizeof(int), cudaMemcpyDeviceToHost, st));
+    PRISM_CUDA_OK(cudaMemcpyAsync(&nnz, pl.row_ptr + rows, sizeof(int), cudaMemcpyDeviceToHost, st));
+    PRISM_CUDA_OK(cudaStreamSynchronize(st));
+    memset(view, 0, sizeof *view);
+    view->zone_B = pl.zone_B;
+    view->zone_shape = pl.zone_shape;
+    view->perm = pl.perm;
+    view->blk_off = pl.blk_off;
+    view->row_ptr = pl.row_ptr;
+    view->col_idx = pl.col;
+    view->nbmax = pl.g.nbmax;
+    view->nnz = nnz;
+    for (int b = 0; b < pl.g.batch; ++b) view->n_blocks[b] = pl.host_nb[b];
+    return PRISM_OK;
+}
+
+static const char *const kTimerNames[kTCount] = {"zone_stats_v", "zone_stats_a", "zone_decide", "permute_pool",
+                                                  "select", "csr_csc", "attn_fwd", "attn_bwd_pre", "attn_bwd",
+                                                  "dq_finalize"};
+
+const char *prism_timer_name(int id) { return (id >= 0 && id < kTCount) ? kTimerNames[id] : ""; }
+
+prism_status prism_plan_set_timing(prism_plan *plan, int enable) {
+    g_last_error.clear();
+    if (!plan) return fail(PRISM_ERR_INVALID_ARG, "plan is NULL");
+    if (enable && !plan->pl.timers) {
+        plan->pl.timers = new (std::nothrow) TimerState;
+        if (!plan->pl.timers) return fail(PRISM_ERR_NOMEM, "timer allocation failed");
+    } else if (!enable && plan->pl.timers) {
+        cudaDeviceSynchronize();
+        delete plan->pl.timers;
+        plan->pl.timers = nullptr;
+    }
+    return PRISM_OK;
+}
+
+prism_status prism_plan_read_timing(prism_plan *plan, float *total_ms, int *launches) {
+    g_last_error.clear();
+    if (!plan || !total_ms || !launches) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_plan_read_timing");
+    TimerState *ts = plan->pl.timers;
+    for (int k = 0; k < kTCount; ++k) {
+        total_ms[k] = 0.f;
+        launches[k] = 0;
+        if (!ts) continue;
+        for (auto &pr : ts->rec[k]) {
+            PRISM_CUDA_OK(cudaEventSynchronize(pr.second));
+            float ms = 0.f;
+            PRISM_CUDA_OK(cudaEventElapsedTime(&ms, pr.first, pr.second));
+            total_ms[k] += ms;
+            launches[k] += 1;
+            ts->pool.push_back(pr.first);
+            ts->pool.push_back(pr.second);
+        }
+        ts->rec[k].clear();
+    }
+    return PRISM_OK;
+}
+
+prism_status prism_plan_check(prism_plan *plan, void *stream) {
+    g_last_error.clear();
+    if (!plan) return fail(PRISM_ERR_INVALID_ARG, "plan is NULL");
+    Plan &pl = plan->pl;
+    prism_status s = device_guard(pl);
+    if (s != PRISM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int word[2] = {0, 0};
+    PRISM_CUDA_OK(cudaMemcpyAsync(word, pl.status, sizeof word, cudaMemcpyDeviceToHost, st));
+    PRISM_CUDA_OK(cudaStreamSynchronize(st));
+    PRISM_CUDA_OK(cudaGetLastError());
+    if (word[0] != 0) {
+        PRISM_CUDA_OK(cudaMemsetAsync(pl.status, 0, 16 * sizeof(int), st));
+        PRISM_CUDA_OK(cudaStreamSynchronize(st));
+        return fail(PRISM_ERR_TIMEOUT, "device-side wait gave up (code %d, site %d)", word[0], word[1]);
+    }
+    return PRISM_OK;
+}
+
+}  // extern "C"

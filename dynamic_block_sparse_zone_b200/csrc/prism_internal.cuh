@@ -1,0 +1,107 @@
+// prism_internal.cuh -- shared declarations of the CUDA library (not part of
+// the C ABI).  Layout of every internal buffer is documented in the plan
+// struct below.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/prism.h"
+
+namespace prism {
+
+constexpr int kZone = 8;           // macro-zone edge [Prism guide, core ideas, bullet 1]
+constexpr int kZoneVol = 512;
+constexpr int kTile = 64;          // every block is a multiple of 64 tokens
+constexpr int kStatChunk = 128;    // channels per zone-statistics CTA
+constexpr int kNumShapes = 16;
+
+enum TimerId {
+    kTZoneV = 0, kTZoneA, kTDecide, kTPermutePool, kTSelect, kTCsr, kTAttnFwd, kTBwdPre, kTAttnBwd, kTDqFinal,
+    kTCount
+};
+static_assert(kTCount == PRISM_NUM_TIMERS, "timer count");
+
+struct TimerState;  // event pools, defined in prism_api.cu
+
+// Per-launch problem geometry, passed by value to kernels.
+struct Geo {
+    int batch, T, H, W, heads, D;
+    int N, M, MT, MH, MW, nbmax, C;
+};
+
+// Everything a plan owns (device pointers unless noted).
+struct Plan {
+    prism_params p;
+    Geo g;
+    int fixed_idx;          // table index of the fixed shape, -1 = dynamic
+    int cap_stride;         // worst-case selected blocks per row
+    int device;
+    bool have_fwd;
+    // zone statistics and decisions
+    double *zone_part;      // [batch][M][nchunk][3]  sum_c of directional variances
+    double *zone_a;         // [batch][M][5]  sigma2_a T,H,W, mean a, max a
+    int *zone_B;            // [batch][M]
+    int *zone_shape;        // [batch][M]
+    int *zone_blk0;         // [batch][M+1]  first block of each zone
+    int *nb;                // [batch]
+    int *blk_off;           // [batch][nbmax+1]
+    int *tile_blk;          // [batch][nbmax]  64-row tile -> block
+    int *perm;              // [batch][N]  block-contiguous position -> raster token
+    // permuted head-major inputs and pooled blocks
+    __nv_bfloat16 *Qp, *Kp, *Vp;   // [batch*heads][N][D]
+    double *Qbar, *Kbar;           // [batch*heads][nbmax][D]
+    // selection
+    int *cnt;               // [batch*heads*nbmax]
+    int *cols_pad;          // [batch*heads*nbmax][cap_stride]
+    int *row_ptr;           // [rows+1]
+    int *col;               // [rows*cap_stride]
+    int *colT_ptr;          // [rows+1]   CSC over (b*heads+h)*nbmax + j
+    int *rowT;              // [rows*cap_stride]
+    int *colT_cursor;       // [rows]
+    int *scan_tmp;          // block partial sums for scans
+    // attention statistics / backward scratch
+    float *lse_p;           // [batch*heads][N] natural-log LSE, permuted order
+    __nv_bfloat16 *dOp;     // [batch*heads][N][D]
+    float *delta;           // [batch*heads][N]
+    float *dQacc;           // [batch*heads][N][D]
+    int *status;            // device error word (0 = ok)
+    int *host_nb;           // pinned host copy of nb
+    TimerState *timers;     // NULL unless timing is on
+};
+
+// Records CUDA events around the launches in its scope when timing is on.
+struct TimerScope {
+    Plan &pl;
+    int id;
+    cudaStream_t st;
+    TimerScope(Plan &p, int i, cudaStream_t s);
+    ~TimerScope();
+};
+
+#define PRISM_CUDA_OK(call)                                                       \
+    do {                                                                          \
+        cudaError_t e_ = (call);                                                  \
+        if (e_ != cudaSuccess) return prism::fail_cuda(e_, #call, __FILE__, __LINE__); \
+    } while (0)
+
+prism_status fail(prism_status s, const char *fmt, ...);
+prism_status fail_cuda(cudaError_t e, const char *what, const char *file, int line);
+
+// Launchers (each returns PRISM_OK or an error after checking the launch).
+prism_status launch_plan(Plan &pl, const void *Q, const void *K, const void *V, const float *a,
+                         cudaStream_t st);
+prism_status launch_attn_fwd(Plan &pl, void *O, float *lse, cudaStream_t st);
+prism_status launch_attn_bwd(Plan &pl, const void *O, const void *dO, void *dQ, void *dK, void *dV,
+                             cudaStream_t st);
+
+__host__ __device__ inline int cap_for(int nb, int k, float max_frac) {
+    if (!(max_frac > 0.0f)) return nb;
+    int c = (int)floor((double)max_frac * (double)nb);
+    if (c < k) c = k;
+    if (c > nb) c = nb;
+    return c;
+}
+
+}  // namespace prism

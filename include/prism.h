@@ -1,0 +1,167 @@
+/*
+ * prism.h -- C ABI of the B200 (sm_100a) implementation of Prism's dynamic
+ * sparse video self-attention hot path.
+ *
+ * Source of the method: paper guide "Prism: Dynamic Sparse Attention cho Huan
+ * luyen Mo hinh Tao Video-Am thanh Dong thoi Do phan giai Goc 2K" (xyznot.com,
+ * paper 2610.05416), cited as [Prism guide, <section>].
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Plain C types only.  "device" pointers are CUDA global-memory addresses of
+ *   the device that was current when the plan was created; "host" pointers are
+ *   ordinary CPU memory.  `stream` is a cudaStream_t passed as void* (NULL =
+ *   the legacy default stream).
+ * - Tensor layouts (row-major, no padding):
+ *     Q, K, V, O, dO, dQ, dK, dV : bf16 [batch][N][heads][head_dim]
+ *     a_norm                     : fp32 [batch][T][H][W]
+ *     lse                        : fp32 [batch][heads][N]
+ *   with N = T*H*W and tokens in raster order n = (t*H + h)*W + w.
+ * - Ownership: the caller owns every tensor argument and the stream.  The plan
+ *   owns its internal device buffers (permuted copies, pooled tensors, block
+ *   CSR and CSC, softmax statistics) and frees them in prism_plan_destroy.
+ * - Errors: every call returns a prism_status; no exception crosses the ABI.
+ *   Argument errors are detected on the host before any launch.  Launch
+ *   failures return PRISM_ERR_CUDA.  prism_last_error() gives a message for
+ *   the calling thread's last failure.
+ * - Synchronisation: prism_plan_build, prism_attn_fwd and prism_attn_bwd only
+ *   enqueue work on `stream`; they never wait for the device.  Calls on one
+ *   plan must be ordered on one stream (or by the caller's events).
+ *   prism_plan_view and prism_plan_check synchronise the stream they are given.
+ */
+#ifndef PRISM_H
+#define PRISM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PRISM_API __attribute__((visibility("default")))
+#else
+#define PRISM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum prism_status {
+    PRISM_OK = 0,
+    PRISM_ERR_INVALID_ARG = 1,  /* a NULL pointer, a size out of range        */
+    PRISM_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. odd grid)   */
+    PRISM_ERR_CUDA = 3,         /* a CUDA call or kernel launch failed         */
+    PRISM_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up          */
+    PRISM_ERR_NOMEM = 5,        /* device allocation failed                    */
+    PRISM_ERR_STATE = 6         /* call out of order (e.g. bwd before fwd)     */
+} prism_status;
+
+/* Problem description.
+ * T, H, W: latent grid, each a positive multiple of 8 (the 8x8x8 macro-zone,
+ *   [Prism guide, core ideas, bullet 1]).
+ * heads, head_dim: head_dim is 64 or 128.
+ * top_k >= 1, 0 < top_p <= 1: hybrid selection S_i = Top-k U Top-p
+ *   [Prism guide, Method section 3].
+ * max_frac: 0 means no per-row cap; otherwise a query block keeps at most
+ *   max(top_k, floor(max_frac * N_b)) key blocks (N_b = number of blocks).
+ * fixed_shape: {0,0,0} selects the dynamic shape of every zone
+ *   [Prism guide, Method sections 1-2]; otherwise every zone uses this edge
+ *   triple, which must be one of the 16 candidates (edges in {2,4,8}).
+ * eps: the epsilon of the indicator g_d (1e-6 when <= 0 is given).        */
+typedef struct prism_params {
+    int batch, T, H, W, heads, head_dim;
+    int top_k;
+    float top_p;
+    float max_frac;
+    int fixed_shape[3];
+    double eps;
+} prism_params;
+
+typedef struct prism_plan prism_plan;
+
+/* Read-only device views of a built plan (all arrays are device memory of
+ * the plan; valid until the next prism_plan_build or prism_plan_destroy).
+ * NBMAX = N/64 is the most blocks a sample can have; every per-block array is
+ * sized for it, entries past a sample's n_blocks are unspecified.
+ *   zone_B      int [batch][N/512]      block volume B(m) in {64,128,256}
+ *   zone_shape  int [batch][N/512]      index into the 16-entry candidate
+ *                                       table (volume 64: 0-6, 128: 7-12,
+ *                                       256: 13-15; lexicographic (bT,bH,bW))
+ *   perm        int [batch][N]          perm[n_new] = raster index of the
+ *                                       token stored at block-contiguous
+ *                                       position n_new
+ *   blk_off     int [batch][NBMAX+1]    first block-contiguous position of
+ *                                       each block; blk_off[n_blocks] = N
+ *   row_ptr     int [batch*heads*NBMAX+1]  block CSR over rows
+ *                                       r = (b*heads + h)*NBMAX + i
+ *   col_idx     int [nnz]               selected key blocks, ascending per row
+ *   n_blocks    host copy, one per sample (first `batch` entries)          */
+typedef struct prism_plan_view {
+    const int *zone_B, *zone_shape, *perm, *blk_off, *row_ptr, *col_idx;
+    int nbmax;
+    long long nnz;
+    int n_blocks[64];
+} prism_plan_view;
+
+/* Allocates a plan and all of its device buffers for the worst case
+ * (N/64 blocks per sample).  Validates params.  *out receives the plan.    */
+PRISM_API prism_status prism_plan_create(const prism_params *params, prism_plan **out);
+
+/* Device bytes a plan with these params holds (0 on invalid params).      */
+PRISM_API size_t prism_plan_bytes(const prism_params *params);
+
+/* Builds the plan from one batch of inputs [Prism guide, Method sections
+ * 1-3]: per-zone statistics and the indicator g_d from V and a_norm, block
+ * volume and shape, the block-contiguous permutation (Q, K, V are gathered
+ * into the plan's head-major permuted copies), mean-pooled Q and K per block,
+ * pooled block scores and the hybrid Top-k U Top-p key-block CSR and its
+ * transpose.  Q, K, V, a_norm: device, layouts above; read only.            */
+PRISM_API prism_status prism_plan_build(prism_plan *plan, const void *Q, const void *K, const void *V,
+                              const float *a_norm, void *stream);
+
+/* Sparse attention forward over the selected blocks of the last build
+ * [Prism guide, Method section 3, last sentence]: each query token of block
+ * i attends under one online softmax to every token of the key blocks in
+ * S_i.  Reads the permuted Q, K, V of the last build.  Writes O (device,
+ * bf16, user layout) and, if lse != NULL, the natural-log log-sum-exp of the
+ * scaled scores (device, fp32 [batch][heads][N], raster token order).  The
+ * plan keeps its own copy of the statistics for prism_attn_bwd.           */
+PRISM_API prism_status prism_attn_fwd(prism_plan *plan, void *O, float *lse, void *stream);
+
+/* Gradient of sum(O * dO) with respect to Q, K, V through the same sparse
+ * attention (the plan and the forward's statistics are reused).  O is the
+ * forward's output and dO the incoming gradient (device, bf16, user layout);
+ * dQ, dK, dV are written (device, bf16, user layout).  Returns
+ * PRISM_ERR_STATE if no forward ran since the last build.                  */
+PRISM_API prism_status prism_attn_bwd(prism_plan *plan, const void *O, const void *dO, void *dQ, void *dK,
+                            void *dV, void *stream);
+
+/* Synchronises `stream`, then fills *view (device pointers + host n_blocks).*/
+PRISM_API prism_status prism_plan_view_get(prism_plan *plan, prism_plan_view *view, void *stream);
+
+/* Synchronises `stream` and reports a device-side error recorded by a
+ * kernel of this plan (PRISM_ERR_TIMEOUT for a bounded wait that gave up),
+ * then clears it.                                                          */
+PRISM_API prism_status prism_plan_check(prism_plan *plan, void *stream);
+
+/* Optional per-kernel timing with CUDA events recorded on the launch stream
+ * around every kernel of the plan (off by default; adds two event records
+ * per launch).  prism_plan_read_timing waits for the recorded events, writes
+ * for each timer id the summed milliseconds and the number of launches since
+ * the previous read (arrays of PRISM_NUM_TIMERS host entries), and resets.
+ * Timer ids and names: prism_timer_name(id).                               */
+#define PRISM_NUM_TIMERS 10
+PRISM_API prism_status prism_plan_set_timing(prism_plan *plan, int enable);
+PRISM_API prism_status prism_plan_read_timing(prism_plan *plan, float *total_ms, int *launches);
+PRISM_API const char *prism_timer_name(int id);
+
+/* Frees the plan and its device buffers (NULL is ignored).                 */
+PRISM_API void prism_plan_destroy(prism_plan *plan);
+
+/* Message of the calling thread's last failed call ("" if none).          */
+PRISM_API const char *prism_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PRISM_H */
