@@ -103,7 +103,7 @@ class _DevArray:
     """Zero-copy view of device memory via __cuda_array_interface__."""
 
     def __init__(self, ptr: int, shape, typestr: str):
-        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr, "data": (ptr, True),
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr, "data": (ptr, False),
                                          "version": 3, "strides": None}
 
 

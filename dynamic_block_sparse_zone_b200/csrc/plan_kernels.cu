@@ -276,7 +276,9 @@ __global__ void __launch_bounds__(1024) k_zone_decide(Geo g, int nchunk, const d
                                                       int fixed_idx, int *__restrict__ zone_B,
                                                       int *__restrict__ zone_shape, int *__restrict__ zone_blk0,
                                                       int *__restrict__ nb_out, int *__restrict__ blk_off,
-                                                      int *__restrict__ tile_blk) {
+                                                      int *__restrict__ tile_blk, int *__restrict__ zone_qt0,
+                                                      int *__restrict__ nqt, int *__restrict__ qt_row,
+                                                      int *__restrict__ qt_blk) {
     __shared__ double red_s[32], red_a[32];
     __shared__ int sbuf[64];
     __shared__ double s_max_sh, a_max_sh;
@@ -314,10 +316,10 @@ __global__ void __launch_bounds__(1024) k_zone_decide(Geo g, int nchunk, const d
     const double s_max = s_max_sh, a_max = a_max_sh;
 
     // pass 2: decisions, then a running exclusive scan of blocks per zone
-    int carry = 0;
+    int carry = 0, carry_t = 0;
     for (int base = 0; base < M; base += blockDim.x) {
         const int m = base + tid;
-        int nblk = 0;
+        int nblk = 0, ntile = 0;
         if (m < M) {
             size_t zm = (size_t)b * M + m;
             double sg[3], sa[3];
@@ -368,15 +370,23 @@ __global__ void __launch_bounds__(1024) k_zone_decide(Geo g, int nchunk, const d
             zone_B[zm] = B;
             zone_shape[zm] = idx;
             nblk = kZoneVol / B;
+            ntile = nblk * ((B + 127) / 128);  // 128-row query tiles of the zone
         }
-        int total;
-        int excl = block_scan_excl_1024(nblk, sbuf, &total);
-        if (m < M) zone_blk0[(size_t)b * (M + 1) + m] = carry + excl;
+        int total, total_t;
+        const int excl = block_scan_excl_1024(nblk, sbuf, &total);
+        const int excl_t = block_scan_excl_1024(ntile, sbuf, &total_t);
+        if (m < M) {
+            zone_blk0[(size_t)b * (M + 1) + m] = carry + excl;
+            zone_qt0[(size_t)b * (M + 1) + m] = carry_t + excl_t;
+        }
         carry += total;
+        carry_t += total_t;
     }
     if (tid == 0) {
         zone_blk0[(size_t)b * (M + 1) + M] = carry;
+        zone_qt0[(size_t)b * (M + 1) + M] = carry_t;
         nb_out[b] = carry;
+        nqt[b] = carry_t;
         blk_off[(size_t)b * (g.nbmax + 1) + carry] = g.N;
     }
     __syncthreads();
@@ -385,10 +395,15 @@ __global__ void __launch_bounds__(1024) k_zone_decide(Geo g, int nchunk, const d
         size_t zm = (size_t)b * M + m;
         const int B = zone_B[zm];
         const int j0 = zone_blk0[(size_t)b * (M + 1) + m];
+        int t = zone_qt0[(size_t)b * (M + 1) + m];
         for (int l = 0; l < kZoneVol / B; ++l) {
             const int off = m * kZoneVol + l * B;
             blk_off[(size_t)b * (g.nbmax + 1) + j0 + l] = off;
             for (int u = 0; u < B / kTile; ++u) tile_blk[(size_t)b * g.nbmax + off / kTile + u] = j0 + l;
+            for (int r = 0; r < B; r += 128, ++t) {
+                qt_row[(size_t)b * g.nbmax + t] = off + r;
+                qt_blk[(size_t)b * g.nbmax + t] = j0 + l;
+            }
         }
     }
 }
@@ -911,7 +926,7 @@ prism_status launch_plan(Plan &pl, const void *Qv, const void *Kv, const void *V
     { TimerScope ts(pl, kTDecide, st);
     k_zone_decide<<<g.batch, 1024, 0, st>>>(g, nchunk, pl.zone_part, pl.zone_a, pl.p.eps, pl.fixed_idx,
                                             pl.zone_B, pl.zone_shape, pl.zone_blk0, pl.nb, pl.blk_off,
-                                            pl.tile_blk); }
+                                            pl.tile_blk, pl.zone_qt0, pl.nqt, pl.qt_row, pl.qt_blk); }
     const int pp_threads = g.C / 8 >= 384 ? 384 : ((g.C / 8 + 31) / 32) * 32;
     { TimerScope ts(pl, kTPermutePool, st);
     k_permute_pool<<<dim3(g.nbmax, g.batch), pp_threads, 0, st>>>(Q, K, V, g, pl.nb, pl.blk_off, pl.zone_shape,

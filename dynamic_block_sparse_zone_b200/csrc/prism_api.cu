@@ -3,6 +3,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <new>
@@ -34,6 +35,7 @@ prism_status fail_cuda(cudaError_t e, const char *what, const char *file, int li
 int host_shape_table(int (*e)[3]);
 prism_status configure_plan_kernels(const Plan &pl);
 prism_status configure_attn_kernels();
+prism_status configure_attn_tc_kernels();
 size_t select_smem_bytes(const Plan &pl);
 
 static int log2_exact(int x) {
@@ -112,6 +114,10 @@ static size_t plan_allocs(Plan &pl, Alloc *out) {
     add((void **)&pl.nb, (size_t)g.batch * sizeof(int));
     add((void **)&pl.blk_off, (size_t)g.batch * (g.nbmax + 1) * sizeof(int));
     add((void **)&pl.tile_blk, (size_t)g.batch * g.nbmax * sizeof(int));
+    add((void **)&pl.zone_qt0, (size_t)g.batch * (g.M + 1) * sizeof(int));
+    add((void **)&pl.nqt, (size_t)g.batch * sizeof(int));
+    add((void **)&pl.qt_row, (size_t)g.batch * g.nbmax * sizeof(int));
+    add((void **)&pl.qt_blk, (size_t)g.batch * g.nbmax * sizeof(int));
     add((void **)&pl.perm, (size_t)g.batch * g.N * sizeof(int));
     add((void **)&pl.Qp, BH * g.N * g.D * 2);
     add((void **)&pl.Kp, BH * g.N * g.D * 2);
@@ -258,6 +264,12 @@ prism_status prism_plan_create(const prism_params *params, prism_plan **out) {
     }
     s = configure_plan_kernels(pl);
     if (s == PRISM_OK) s = configure_attn_kernels();
+    if (s == PRISM_OK) s = configure_attn_tc_kernels();
+    if (s == PRISM_OK) s = make_tensor_maps(pl);
+    {
+        const char *env = getenv("PRISM_LEGACY_FWD");
+        pl.use_legacy_fwd = (env && env[0] == '1') ? 1 : 0;
+    }
     if (s != PRISM_OK) {
         release_buffers(pl);
         delete h;
@@ -299,7 +311,8 @@ prism_status prism_attn_fwd(prism_plan *plan, void *O, float *lse, void *stream)
     prism_status s = device_guard(plan->pl);
     if (s != PRISM_OK) return s;
     if ((uintptr_t)O & 15) return fail(PRISM_ERR_INVALID_ARG, "O must be 16-byte aligned");
-    s = launch_attn_fwd(plan->pl, O, lse, static_cast<cudaStream_t>(stream));
+    s = plan->pl.use_legacy_fwd ? launch_attn_fwd(plan->pl, O, lse, static_cast<cudaStream_t>(stream))
+                                : launch_attn_fwd_tc(plan->pl, O, lse, static_cast<cudaStream_t>(stream));
     if (s == PRISM_OK) plan->pl.have_fwd = true;
     return s;
 }

@@ -3,6 +3,7 @@
 // struct below.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -48,6 +49,10 @@ struct Plan {
     int *nb;                // [batch]
     int *blk_off;           // [batch][nbmax+1]
     int *tile_blk;          // [batch][nbmax]  64-row tile -> block
+    int *zone_qt0;          // [batch][M+1]  first 128-row query tile of each zone
+    int *nqt;               // [batch]       number of 128-row query tiles
+    int *qt_row;            // [batch][nbmax] first block-contiguous row of each query tile
+    int *qt_blk;            // [batch][nbmax] block of each query tile
     int *perm;              // [batch][N]  block-contiguous position -> raster token
     // permuted head-major inputs and pooled blocks
     __nv_bfloat16 *Qp, *Kp, *Vp;   // [batch*heads][N][D]
@@ -69,6 +74,9 @@ struct Plan {
     int *status;            // device error word (0 = ok)
     int *host_nb;           // pinned host copy of nb
     TimerState *timers;     // NULL unless timing is on
+    int use_legacy_fwd;     // development switch: warp-MMA forward instead of tcgen05
+    // TMA descriptors of the permuted copies, viewed as [batch*heads*N][D] bf16
+    CUtensorMap tmQ, tmK, tmV;
 };
 
 // Records CUDA events around the launches in its scope when timing is on.
@@ -93,6 +101,8 @@ prism_status fail_cuda(cudaError_t e, const char *what, const char *file, int li
 prism_status launch_plan(Plan &pl, const void *Q, const void *K, const void *V, const float *a,
                          cudaStream_t st);
 prism_status launch_attn_fwd(Plan &pl, void *O, float *lse, cudaStream_t st);
+prism_status launch_attn_fwd_tc(Plan &pl, void *O, float *lse, cudaStream_t st);
+prism_status make_tensor_maps(Plan &pl);
 prism_status launch_attn_bwd(Plan &pl, const void *O, const void *dO, void *dQ, void *dK, void *dV,
                              cudaStream_t st);
 

@@ -93,9 +93,20 @@ def compare_plan(w, pl, view, b=0, heads=None):
     return ties
 
 
+def bf16_half_ulp(x):
+    """Half a bf16 unit in the last place at |x| (8 significant bits)."""
+    ax = np.abs(x)
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    return np.where(ax > 0, np.exp2(e - 8), 0.0)
+
+
 def _err(gpu, ref):
+    """max-abs error beyond the bf16 rounding of the output itself, and the
+    relative L2 error.  Outputs are stored in bf16, so a value of magnitude
+    in [4, 8) can be off by up to 2^-6 from rounding alone; the max-abs bound
+    applies to what the arithmetic adds on top of that."""
     gpu = gpu.astype(np.float64)
-    diff = np.abs(gpu - ref)
+    diff = np.maximum(np.abs(gpu - ref) - bf16_half_ulp(ref), 0.0)
     rel = np.linalg.norm(gpu - ref) / max(np.linalg.norm(ref), 1e-30)
     return float(diff.max()), float(rel)
 
@@ -214,12 +225,25 @@ def test_backward_parity(name):
 def check_gradient_sums(g, inp, b=0):
     """Properties of softmax attention at any size: for every query the dS row
     sums to zero, so sum_t dK_t = 0; the P row sums to one, so
-    sum_t dV_t = sum_q dO_q (per head, over the whole sequence)."""
+    sum_t dV_t = sum_q dO_q (per head, over the whole sequence).
+
+    The kernels form Delta_q = dO_q . O_q from the bf16-rounded O, so each dS
+    row sums to -dDelta_q instead of 0, with dDelta_q of standard deviation at
+    most 2^-8/sqrt(3) |dO_q * O_q|.  Hence sum_t dK_t has standard deviation
+    at most scale 2^-8/sqrt(3) sqrt(sum_q |dO_q * O_q|^2 Q_qc^2) per channel;
+    the bound is six of those plus 2% of |dK| for the bf16 rounding of dS."""
     dK = g["dK"][b].double()
     dV = g["dV"][b].double()
-    dO = inp.dO[b].to(dK.device).double()
+    dev = dK.device
+    dO = inp.dO[b].to(dev).double()
+    O = g["O"][b].double()
+    Q = inp.Q[b].to(dev).double()
+    scale = 1.0 / np.sqrt(Q.shape[-1])
+    w2 = ((dO * O) ** 2).sum(-1, keepdim=True)                 # [N, heads, 1]
+    sigma = scale * 2.0 ** -8 / np.sqrt(3.0) * torch.sqrt((w2 * Q * Q).sum(0))
     sk = dK.sum(0)
-    assert torch.all(sk.abs() <= 0.02 * dK.norm(dim=0) + 1e-3), float((sk.abs() / dK.norm(dim=0)).max())
+    bound = 6.0 * sigma + 0.02 * dK.norm(dim=0) + 1e-3
+    assert torch.all(sk.abs() <= bound), float((sk.abs() / bound).max())
     sv, so = dV.sum(0), dO.sum(0)
     assert torch.all((sv - so).abs() <= 0.02 * dV.norm(dim=0) + 1e-3), float((sv - so).abs().max())
 
