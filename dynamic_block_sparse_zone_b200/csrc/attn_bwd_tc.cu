@@ -1,0 +1,377 @@
+// attn_bwd_tc.cu -- block-sparse attention backward on the tcgen05 tensor
+// cores, key-stationary.
+//
+// Gradient of sum(O * dO) through softmax attention restricted to the
+// selected block pairs [Prism guide, Method section 3; the backward is the
+// standard softmax-attention gradient]:
+//   P = exp(S*scale - LSE), dP = dO V^T, dS = P (dP - Delta),
+//   dV = P^T dO, dK = scale dS^T Q, dQ = scale dS K.
+//
+// Work unit: one 128-key tile of one head (a 64-token key block fills the
+// upper half with rows it ignores).  The CTA walks the query blocks of the
+// key block's CSC column as 64-row chunks.
+//
+// Per chunk c (TMEM buffers alternate with c & 1):
+//   S^T  = K Q_c^T         M=128 keys, N=64 queries   -> TMEM ST[c&1]
+//   dP^T = V dO_c^T        M=128 keys, N=64 queries   -> TMEM DP[c&1]
+//   softmax warps: P^T, dS^T (bf16) over ST / DP, dS^T also to shared memory
+//   dV  += P^T dO_c        A = P^T from TMEM          -> TMEM dV
+//   dK  += dS^T Q_c        A = dS^T from TMEM         -> TMEM dK
+//   dQ^T = K^T dS^T        both operands MN-major     -> TMEM ST[c&1]
+//   drain warps: dQ^T rows (lane = head-dim index) -> fp32 reductions into dQ
+// TMEM columns: dK [0,128), dV [128,256), ST[2] [256,384), DP[2] [384,512).
+//
+// Warp roles (320 threads): warp 0 TMA producer (K, V once; Q, dO, LSE,
+// Delta per chunk into a two-stage ring), warp 1 MMA issuer, warps 2..5
+// softmax (one key row each), warps 6..9 dQ drain (one head-dim row each).
+#include <cuda.h>
+
+#include "tc_common.cuh"
+
+namespace prism {
+
+using namespace tc;
+
+namespace bwdtc {
+
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColDK = 0, kColDV = 128, kColST = 256, kColDP = 384;
+
+template <int D>
+struct Layout {
+    static_assert(D == 128, "tensor-core backward is written for head_dim 128");
+    static constexpr uint32_t kKVHalf = 128 * 128;  // 128 rows x 128 B
+    static constexpr uint32_t kQHalf = 64 * 128;    // 64 rows x 128 B
+    static constexpr uint32_t kK = 0;
+    static constexpr uint32_t kV = kK + 2 * kKVHalf;
+    static constexpr uint32_t kQ0 = kV + 2 * kKVHalf;      // stage s: Q at kQ0 + s*kStage, dO at + 2*kQHalf
+    static constexpr uint32_t kStage = 4 * kQHalf;
+    static constexpr uint32_t kDS = kQ0 + 2 * kStage;      // [2] x 128 key rows x 128 B (64 queries bf16)
+    static constexpr uint32_t kVec = kDS + 2 * 16384;      // stage s: LSE [64] f32 then Delta [64] f32
+    static constexpr uint32_t kBars = kVec + 2 * 512;
+    // kv, q_full[2], q_empty[2], s_full[2], p_full[2], dq_full[2], dq_empty[2], done
+    static constexpr uint32_t kNumBars = 14;
+    static constexpr uint32_t kBytes = kBars + kNumBars * 8 + 16;
+    static constexpr uint32_t kAlloc = kBytes + 1024;
+};
+
+enum { kSiteKV = 11, kSiteQFull, kSiteQEmpty, kSiteS, kSiteP, kSiteDQFull, kSiteDQEmpty, kSiteDone };
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_attn_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO, Geo g,
+                  const int *__restrict__ nqt, const int *__restrict__ qt_row, const int *__restrict__ qt_blk,
+                  const int *__restrict__ blk_off, const int *__restrict__ colT_ptr, const int *__restrict__ rowT,
+                  const int *__restrict__ perm, const float *__restrict__ lse_p, const float *__restrict__ delta,
+                  float *__restrict__ dQacc, __nv_bfloat16 *__restrict__ dK, __nv_bfloat16 *__restrict__ dV,
+                  float scale, float scale_log2, int *__restrict__ status) {
+    using L = Layout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(smem);
+
+    const int tile = blockIdx.x, bh = blockIdx.y, b = bh / g.heads, h = bh % g.heads;
+    if (tile >= nqt[b]) return;
+    if (*reinterpret_cast<volatile int *>(status) != 0) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int *bo = blk_off + (size_t)b * (g.nbmax + 1);
+    const int k0 = qt_row[(size_t)b * g.nbmax + tile];
+    const int jblk = qt_blk[(size_t)b * g.nbmax + tile];
+    const int kvalid = min(128, bo[jblk + 1] - k0);
+    const size_t colid = (size_t)bh * g.nbmax + jblk;
+    const int u_begin = colT_ptr[colid], u_end = colT_ptr[colid + 1];
+
+    int nchunk = 0;  // 64-row query chunks of the column
+    for (int u = u_begin + lane; u < u_end; u += 32) {
+        const int i = rowT[u];
+        nchunk += (bo[i + 1] - bo[i]) >> 6;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nchunk += __shfl_xor_sync(0xffffffffu, nchunk, o);
+
+    const uint32_t bar_kv = sbase + L::kBars;
+    const uint32_t bar_qf = bar_kv + 8, bar_qe = bar_qf + 16, bar_sf = bar_qe + 16, bar_pf = bar_sf + 16;
+    const uint32_t bar_df = bar_pf + 16, bar_de = bar_df + 16, bar_done = bar_de + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBars + L::kNumBars * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kBars + L::kNumBars * 8 + 8);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_init(bar_kv, 1);
+            for (int s = 0; s < 2; ++s) {
+                mbar_init(bar_qf + 8 * s, 1);
+                mbar_init(bar_qe + 8 * s, 1);
+                mbar_init(bar_sf + 8 * s, 1);
+                mbar_init(bar_pf + 8 * s, 128);
+                mbar_init(bar_df + 8 * s, 1);
+                mbar_init(bar_de + 8 * s, 128);
+            }
+            mbar_init(bar_done, 1);
+            *abort_flag = 0;
+            mbar_fence_init();
+            prefetch_map(&tmQ);
+            prefetch_map(&tmK);
+            prefetch_map(&tmV);
+            prefetch_map(&tmdO);
+        }
+        __syncwarp();
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int rowbase = bh * g.N;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            mbar_expect_tx(bar_kv, 2 * 128 * D * 2);
+            for (int hf = 0; hf < 2; ++hf)
+                for (int rh = 0; rh < 2; ++rh) {
+                    tma_load_2d(sbase + L::kK + hf * L::kKVHalf + rh * 8192, &tmK, bar_kv, hf * 64,
+                                rowbase + k0 + rh * 64);
+                    tma_load_2d(sbase + L::kV + hf * L::kKVHalf + rh * 8192, &tmV, bar_kv, hf * 64,
+                                rowbase + k0 + rh * 64);
+                }
+            int u = u_begin, r = 0, r_end = 0;
+            if (u < u_end) {
+                r = bo[rowT[u]];
+                r_end = bo[rowT[u] + 1];
+            }
+            int issued = 0;
+            for (int c = 0; c < nchunk; ++c) {
+                const int st = c & 1;
+                if (c >= 2 && !mbar_wait(bar_qe + 8 * st, ((c >> 1) + 1) & 1, status, kSiteQEmpty, abort_flag))
+                    break;
+                const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + 2 * L::kQHalf;
+                const uint32_t sVec = sbase + L::kVec + st * 512;
+                const uint32_t bar = bar_qf + 8 * st;
+                mbar_expect_tx(bar, 2 * 64 * D * 2 + 512);
+                for (int hf = 0; hf < 2; ++hf) {
+                    tma_load_2d(sQ + hf * L::kQHalf, &tmQ, bar, hf * 64, rowbase + r);
+                    tma_load_2d(sO + hf * L::kQHalf, &tmdO, bar, hf * 64, rowbase + r);
+                }
+                bulk_load(sVec, lse_p + (size_t)rowbase + r, 256, bar);
+                bulk_load(sVec + 256, delta + (size_t)rowbase + r, 256, bar);
+                issued = c + 1;
+                r += 64;
+                if (r >= r_end && ++u < u_end) {
+                    r = bo[rowT[u]];
+                    r_end = bo[rowT[u] + 1];
+                }
+            }
+            for (int c = max(0, issued - 2); c < issued; ++c)
+                mbar_wait(bar_qf + 8 * (c & 1), (c >> 1) & 1, status, kSiteQFull, abort_flag);
+            mbar_wait(bar_kv, 0, status, kSiteKV, abort_flag);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && nchunk > 0) {
+            constexpr uint32_t idST = idesc_bf16(128, 64, false);          // K-major A and B
+            constexpr uint32_t idAcc = idesc_bf16(128, D, true);           // A from TMEM, B MN-major
+            constexpr uint32_t idDQ = idesc_bf16(128, 64, true, true);     // A and B MN-major
+            bool ok = mbar_wait(bar_kv, 0, status, kSiteKV, abort_flag);
+            auto stage_a = [&](int c) -> bool {  // S^T and dP^T of chunk c
+                const int st = c & 1;
+                if (!mbar_wait(bar_qf + 8 * st, (c >> 1) & 1, status, kSiteQFull, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + 2 * L::kQHalf;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t ko = (kk >> 2) * L::kKVHalf + (kk & 3) * 32;
+                    const uint32_t qo = (kk >> 2) * L::kQHalf + (kk & 3) * 32;
+                    mma_ss(tmem + kColST + st * 64, sdesc(sbase + L::kK + ko, 16, 1024), sdesc(sQ + qo, 16, 1024),
+                           idST, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t ko = (kk >> 2) * L::kKVHalf + (kk & 3) * 32;
+                    const uint32_t qo = (kk >> 2) * L::kQHalf + (kk & 3) * 32;
+                    mma_ss(tmem + kColDP + st * 64, sdesc(sbase + L::kV + ko, 16, 1024), sdesc(sO + qo, 16, 1024),
+                           idST, kk > 0);
+                }
+                tc_commit(bar_sf + 8 * st);
+                return true;
+            };
+            if (ok) ok = stage_a(0);
+            if (ok && nchunk > 1) ok = stage_a(1);
+            for (int c = 0; ok && c < nchunk; ++c) {
+                const int st = c & 1;
+                if (!mbar_wait(bar_pf + 8 * st, (c >> 1) & 1, status, kSiteP, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + 2 * L::kQHalf;
+                const uint32_t acc = (c > 0) ? 1u : 0u;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts(tmem + kColDV, tmem + kColST + st * 64 + kk * 8, sdesc(sO + kk * 2048, L::kQHalf, 1024),
+                           idAcc, acc | (kk > 0));
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts(tmem + kColDK, tmem + kColDP + st * 64 + kk * 8, sdesc(sQ + kk * 2048, L::kQHalf, 1024),
+                           idAcc, acc | (kk > 0));
+                tc_commit(bar_qe + 8 * st);
+                const uint32_t sDS = sbase + L::kDS + st * 16384;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tmem + kColST + st * 64, sdesc(sbase + L::kK + kk * 2048, L::kKVHalf, 1024),
+                           sdesc(sDS + kk * 2048, 8192, 1024), idDQ, kk > 0);
+                tc_commit(bar_df + 8 * st);
+                if (c + 2 < nchunk) {
+                    if (!mbar_wait(bar_de + 8 * st, (c >> 1) & 1, status, kSiteDQEmpty, abort_flag)) break;
+                    tc_fence_after();
+                    if (!stage_a(c + 2)) break;
+                }
+            }
+            tc_commit(bar_done);
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ softmax (key rows)
+        const int quad = warp & 3;
+        const int rowid = quad * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const bool live = rowid < kvalid;
+        const float log2e = 1.4426950408889634f;
+        bool ok = true;
+        for (int c = 0; c < nchunk; ++c) {
+            const int st = c & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * st, (c >> 1) & 1, status, kSiteS, abort_flag) &&
+                                             mbar_wait(bar_qf + 8 * st, (c >> 1) & 1, status, kSiteQFull,
+                                                       abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const float *vec = reinterpret_cast<const float *>(smem + L::kVec + st * 512);
+            const uint32_t tST = tmem + kColST + st * 64 + lane_off;
+            const uint32_t tDP = tmem + kColDP + st * 64 + lane_off;
+            uint8_t *dsrow = smem + L::kDS + st * 16384 + rowid * 128;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t sv[32], dv[32];
+                tmem_ld32(tST + hf * 32, sv);
+                tmem_ld32(tDP + hf * 32, dv);
+                tmem_wait_ld();
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int q = hf * 32 + 2 * e;
+                    float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), scale_log2, -vec[q] * log2e));
+                    float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), scale_log2, -vec[q + 1] * log2e));
+                    float d0 = p0 * (__uint_as_float(dv[2 * e]) - vec[64 + q]);
+                    float d1 = p1 * (__uint_as_float(dv[2 * e + 1]) - vec[64 + q + 1]);
+                    if (!live) p0 = p1 = d0 = d1 = 0.f;
+                    pk[e] = pack_bf16x2(p0, p1);
+                    dk[e] = pack_bf16x2(d0, d1);
+                }
+                tmem_st16(tST + hf * 16, pk);
+                tmem_st16(tDP + hf * 16, dk);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int chunk = hf * 4 + j;
+                    *reinterpret_cast<uint4 *>(dsrow + ((chunk ^ (rowid & 7)) << 4)) =
+                        make_uint4(dk[4 * j], dk[4 * j + 1], dk[4 * j + 2], dk[4 * j + 3]);
+                }
+            }
+            tmem_wait_st();
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar_pf + 8 * st);
+        }
+        // epilogue: dK (scaled) and dV rows to the user layout
+        if (ok && nchunk > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, status, kSiteDone, abort_flag));
+        if (ok) {
+            tc_fence_after();
+            const int tok = live ? perm[(size_t)b * g.N + k0 + rowid] : 0;
+            __nv_bfloat16 *dkr = dK + (((size_t)b * g.N + tok) * g.heads + h) * D;
+            __nv_bfloat16 *dvr = dV + (((size_t)b * g.N + tok) * g.heads + h) * D;
+#pragma unroll 1
+            for (int q = 0; q < D / 32; ++q) {
+                uint32_t a[32], v[32];
+                if (nchunk > 0) {
+                    tmem_ld32(tmem + kColDK + lane_off + q * 32, a);
+                    tmem_ld32(tmem + kColDV + lane_off + q * 32, v);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) a[e] = v[e] = 0u;
+                }
+                uint4 pa[4], pv[4];
+                uint32_t *wa = reinterpret_cast<uint32_t *>(pa), *wv = reinterpret_cast<uint32_t *>(pv);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    wa[e] = pack_bf16x2(__uint_as_float(a[2 * e]) * scale, __uint_as_float(a[2 * e + 1]) * scale);
+                    wv[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+                }
+                if (live) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        reinterpret_cast<uint4 *>(dkr + q * 32)[e] = pa[e];
+                        reinterpret_cast<uint4 *>(dvr + q * 32)[e] = pv[e];
+                    }
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ dQ drain (head-dim rows)
+        const int quad = warp & 3;
+        const int d = quad * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        int u = u_begin, r = 0, r_end = 0;
+        if (u < u_end) {
+            r = bo[rowT[u]];
+            r_end = bo[rowT[u] + 1];
+        }
+        for (int c = 0; c < nchunk; ++c) {
+            const int st = c & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(bar_df + 8 * st, (c >> 1) & 1, status, kSiteDQFull, abort_flag)))
+                break;
+            tc_fence_after();
+            uint32_t v[64];
+            tmem_ld32(tmem + kColST + st * 64 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(v));
+            tmem_ld32(tmem + kColST + st * 64 + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(bar_de + 8 * st);
+            float *dst = dQacc + ((size_t)rowbase + r) * D + d;
+#pragma unroll
+            for (int q = 0; q < 64; ++q) atomicAdd(dst + (size_t)q * D, __uint_as_float(v[q]) * scale);
+            r += 64;
+            if (r >= r_end && ++u < u_end) {
+                r = bo[rowT[u]];
+                r_end = bo[rowT[u] + 1];
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace bwdtc
+
+prism_status configure_attn_bwd_tc_kernels() {
+    PRISM_CUDA_OK(cudaFuncSetAttribute(bwdtc::k_attn_bwd_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)bwdtc::Layout<128>::kAlloc));
+    return PRISM_OK;
+}
+
+// Runs the tensor-core key-stationary backward (head_dim 128); the caller has
+// zeroed dQacc and written dOp and delta.
+prism_status launch_attn_bwd_tc_main(Plan &pl, void *dK, void *dV, cudaStream_t st) {
+    const Geo &g = pl.g;
+    const double scale = 1.0 / sqrt((double)g.D);
+    TimerScope ts(pl, kTAttnBwd, st);
+    bwdtc::k_attn_bwd_tc<128><<<dim3(g.nbmax, g.batch * g.heads), bwdtc::kThreads, bwdtc::Layout<128>::kAlloc, st>>>(
+        pl.tmQ, pl.tmK, pl.tmV, pl.tmdO, g, pl.nqt, pl.qt_row, pl.qt_blk, pl.blk_off, pl.colT_ptr, pl.rowT, pl.perm,
+        pl.lse_p, pl.delta, pl.dQacc, static_cast<__nv_bfloat16 *>(dK), static_cast<__nv_bfloat16 *>(dV),
+        (float)scale, (float)(scale * 1.4426950408889634), pl.status);
+    PRISM_CUDA_OK(cudaGetLastError());
+    return PRISM_OK;
+}
+
+}  // namespace prism

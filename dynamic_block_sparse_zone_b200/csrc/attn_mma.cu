@@ -593,7 +593,10 @@ static prism_status bwd_impl(Plan &pl, const void *O, const void *dO, void *dQ, 
                                                              static_cast<const __nv_bfloat16 *>(dO), pl.perm,
                                                              pl.dOp, pl.delta);
     }
-    {
+    if (D == 128 && !pl.use_legacy_fwd) {
+        prism_status s = launch_attn_bwd_tc_main(pl, dK, dV, st);
+        if (s != PRISM_OK) return s;
+    } else {
     TimerScope ts(pl, kTAttnBwd, st);
     k_attn_bwd_mma<D><<<dim3(g.nbmax, g.batch * g.heads), 128, bwd_smem<D>(), st>>>(
         g, pl.Qp, pl.Kp, pl.Vp, pl.dOp, pl.lse_p, pl.delta, pl.blk_off, pl.tile_blk, pl.colT_ptr, pl.rowT,

@@ -386,6 +386,7 @@ prism_status make_tensor_maps(Plan &pl) {
     prism_status s = make_map(&pl.tmQ, pl.Qp, rows, pl.g.D);
     if (s == PRISM_OK) s = make_map(&pl.tmK, pl.Kp, rows, pl.g.D);
     if (s == PRISM_OK) s = make_map(&pl.tmV, pl.Vp, rows, pl.g.D);
+    if (s == PRISM_OK) s = make_map(&pl.tmdO, pl.dOp, rows, pl.g.D);
     return s;
 }
 

@@ -36,6 +36,7 @@ int host_shape_table(int (*e)[3]);
 prism_status configure_plan_kernels(const Plan &pl);
 prism_status configure_attn_kernels();
 prism_status configure_attn_tc_kernels();
+prism_status configure_attn_bwd_tc_kernels();
 size_t select_smem_bytes(const Plan &pl);
 
 static int log2_exact(int x) {
@@ -265,6 +266,7 @@ prism_status prism_plan_create(const prism_params *params, prism_plan **out) {
     s = configure_plan_kernels(pl);
     if (s == PRISM_OK) s = configure_attn_kernels();
     if (s == PRISM_OK) s = configure_attn_tc_kernels();
+    if (s == PRISM_OK) s = configure_attn_bwd_tc_kernels();
     if (s == PRISM_OK) s = make_tensor_maps(pl);
     {
         const char *env = getenv("PRISM_LEGACY_FWD");

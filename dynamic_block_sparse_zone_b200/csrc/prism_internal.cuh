@@ -76,7 +76,7 @@ struct Plan {
     TimerState *timers;     // NULL unless timing is on
     int use_legacy_fwd;     // development switch: warp-MMA forward instead of tcgen05
     // TMA descriptors of the permuted copies, viewed as [batch*heads*N][D] bf16
-    CUtensorMap tmQ, tmK, tmV;
+    CUtensorMap tmQ, tmK, tmV, tmdO;
 };
 
 // Records CUDA events around the launches in its scope when timing is on.
@@ -103,6 +103,7 @@ prism_status launch_plan(Plan &pl, const void *Q, const void *K, const void *V, 
 prism_status launch_attn_fwd(Plan &pl, void *O, float *lse, cudaStream_t st);
 prism_status launch_attn_fwd_tc(Plan &pl, void *O, float *lse, cudaStream_t st);
 prism_status make_tensor_maps(Plan &pl);
+prism_status launch_attn_bwd_tc_main(Plan &pl, void *dK, void *dV, cudaStream_t st);
 prism_status launch_attn_bwd(Plan &pl, const void *O, const void *dO, void *dQ, void *dK, void *dV,
                              cudaStream_t st);
 
