@@ -23,7 +23,7 @@ _STATUS = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_UNSUPPORTED"
 
 EXPORTED = ("prism_plan_create", "prism_plan_bytes", "prism_plan_build", "prism_attn_fwd", "prism_attn_bwd",
             "prism_plan_view_get", "prism_plan_check", "prism_plan_destroy", "prism_last_error",
-            "prism_plan_set_timing", "prism_plan_read_timing", "prism_timer_name")
+            "prism_plan_set_timing", "prism_plan_read_timing", "prism_timer_name", "prism_zone_shapes_noalloc")
 NUM_TIMERS = 10
 
 
@@ -71,6 +71,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.prism_last_error.restype = ctypes.c_char_p
     lib.prism_plan_set_timing.argtypes = [V, ctypes.c_int]
     lib.prism_plan_read_timing.argtypes = [V, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
+    lib.prism_zone_shapes_noalloc.argtypes = [ctypes.POINTER(prism_params), P, P, P, P, P]
+    lib.prism_zone_shapes_noalloc.restype = ctypes.c_int
     lib.prism_timer_name.argtypes = [ctypes.c_int]
     lib.prism_timer_name.restype = ctypes.c_char_p
     for name in ("prism_plan_create", "prism_plan_build", "prism_attn_fwd", "prism_attn_bwd",
@@ -234,6 +236,22 @@ class PrismPlan:
             n_blocks=[int(v.n_blocks[b]) for b in range(p.batch)],
             nbmax=nbmax,
         )
+
+
+def prism_zone_shapes_noalloc(params: Params, V: torch.Tensor, a_norm: torch.Tensor,
+                              zone_B: torch.Tensor, zone_shape: torch.Tensor):
+    """Zone volumes and shapes without any device allocation inside the call
+    (the library's fixed scratch array is used); outputs are caller-owned
+    int32 CUDA tensors of shape [batch, N/512]."""
+    M = params.N // 512
+    _need(V, "V", torch.bfloat16, (params.batch, params.N, params.heads, params.head_dim))
+    _need(a_norm, "a_norm", torch.float32, (params.batch, params.T, params.H, params.W))
+    _need(zone_B, "zone_B", torch.int32, (params.batch, M))
+    _need(zone_shape, "zone_shape", torch.int32, (params.batch, M))
+    c = params.to_c()
+    _check(load_library().prism_zone_shapes_noalloc(ctypes.byref(c), _ptr(V), _ptr(a_norm), _ptr(zone_B),
+                                                    _ptr(zone_shape), _stream()))
+    return zone_B, zone_shape
 
 
 # Module-level names that mirror the C ABI.

@@ -965,4 +965,28 @@ prism_status configure_plan_kernels(const Plan &pl) {
     return upload_shape_table();
 }
 
+// Zone statistics and volume / shape decisions alone, on caller-provided
+// buffers (used by the allocation-free entry point).  Scratch arrays are laid
+// out by the caller; the kernels are the planner's own.
+prism_status launch_zone_decisions(const Geo &g, double eps, int fixed_idx, const __nv_bfloat16 *V, const float *a,
+                                   double *zone_part, double *zone_a, int *zone_B, int *zone_shape, int *zone_blk0,
+                                   int *nb, int *blk_off, int *tile_blk, int *zone_qt0, int *nqt, int *qt_row,
+                                   int *qt_blk, cudaStream_t st) {
+    const int nchunk = (g.C + kStatChunk - 1) / kStatChunk;
+    const size_t smem_v = 2 * 8 * 8 * kStatChunk * sizeof(float);
+    k_zone_stats_v<<<dim3(nchunk, g.M, g.batch), 128, smem_v, st>>>(V, g, zone_part);
+    k_zone_stats_a<<<dim3(g.M, g.batch), 512, 0, st>>>(a, g, zone_a);
+    k_zone_decide<<<g.batch, 1024, 0, st>>>(g, nchunk, zone_part, zone_a, eps, fixed_idx, zone_B, zone_shape,
+                                            zone_blk0, nb, blk_off, tile_blk, zone_qt0, nqt, qt_row, qt_blk);
+    PRISM_CUDA_OK(cudaGetLastError());
+    return PRISM_OK;
+}
+
+// Kernel attributes and the candidate table for launch_zone_decisions.
+prism_status configure_zone_kernels() {
+    PRISM_CUDA_OK(cudaFuncSetAttribute(k_zone_stats_v, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       2 * 8 * 8 * kStatChunk * (int)sizeof(float)));
+    return upload_shape_table();
+}
+
 }  // namespace prism

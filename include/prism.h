@@ -154,6 +154,29 @@ PRISM_API prism_status prism_plan_set_timing(prism_plan *plan, int enable);
 PRISM_API prism_status prism_plan_read_timing(prism_plan *plan, float *total_ms, int *launches);
 PRISM_API const char *prism_timer_name(int id);
 
+/* Allocation-free variant of the planner's first stage (per-zone statistics,
+ * density, block volume B(m) and shape), for callers that cannot call
+ * cudaMalloc: an application whose caching allocator owns all device memory,
+ * or a loop that cannot afford cudaMalloc's implicit device synchronisation.
+ * The paper has no counterpart of this entry point; it writes the same
+ * zone_B / zone_shape that prism_plan_build computes (see prism_plan_view).
+ * Reads params' batch, grid, heads, head_dim, fixed_shape and eps; V (device,
+ * bf16 [batch][N][heads][head_dim]) and a_norm (device, fp32 [batch][T][H][W]).
+ * Writes zone_B and zone_shape (device, int [batch][N/512], caller-owned).
+ * Scratch comes from one fixed device array of PRISM_NOALLOC_SCRATCH_BYTES
+ * compiled into the library, which every GPU that loads the library holds
+ * until the process exits; a problem needing more (about
+ * 24 * batch * N/512 * ceil(heads*head_dim/128) bytes plus 20 bytes per 64
+ * tokens) returns PRISM_ERR_UNSUPPORTED before anything is launched.  The
+ * first call on a device looks up the array's device address and sets kernel
+ * attributes; make that first call before any stream capture.  All calls
+ * share the array (nothing in it has to start at zero), so calls whose work
+ * overlaps on the GPU (other streams or host threads) race: order them.
+ * Only enqueues work on `stream`.                                          */
+#define PRISM_NOALLOC_SCRATCH_BYTES (4u << 20)
+PRISM_API prism_status prism_zone_shapes_noalloc(const prism_params *params, const void *V, const float *a_norm,
+                                                 int *zone_B, int *zone_shape, void *stream);
+
 /* Frees the plan and its device buffers (NULL is ignored).                 */
 PRISM_API void prism_plan_destroy(prism_plan *plan);
 
