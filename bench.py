@@ -127,13 +127,19 @@ def kernel_bytes(name, w, nb, pairs_unused):
     return None
 
 
+def workload_of(args):
+    from dynamic_block_sparse_zone_b200.synth import WORKLOADS, scaled
+    w = WORKLOADS[args.workload]
+    return scaled(w, heads=args.heads) if args.heads else w
+
+
 def run_ours(args, rank, world, dev):
     import torch
     import torch.distributed as dist
     import dynamic_block_sparse_zone_b200 as P
     from dynamic_block_sparse_zone_b200.synth import WORKLOADS, make_inputs
 
-    w = WORKLOADS[args.workload]
+    w = workload_of(args)
     P.load_library()
     inp = make_inputs(w, seed=0, device=dev, with_grad_output=True)
     plan = P.PrismPlan(P.params_for(w))
@@ -360,7 +366,7 @@ def cpu_baseline(w, dev, rows):
 def run_reference(args, dev):
     import oracle
     from dynamic_block_sparse_zone_b200.synth import WORKLOADS
-    w = WORKLOADS[args.workload]
+    w = workload_of(args)
     pl, hb, plan_s = oracle_setup(w, dev)
     rows = args.ref_rows
     for s in range(args.warmup):
@@ -391,8 +397,9 @@ def main():
     ap.add_argument("--workload", default="latent2k_train_24x96x160")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=48)
-    ap.add_argument("--ref-rows", type=int, default=16)
+    ap.add_argument("--heads", type=int, default=0, help="override the workload's head count (profiling)")
+    ap.add_argument("--cpu-rows", type=int, default=6000)
+    ap.add_argument("--ref-rows", type=int, default=1500)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -419,7 +426,7 @@ def main():
         if world == 1 and not args.no_cpu_baseline:
             torch.cuda.empty_cache()
             from dynamic_block_sparse_zone_b200.synth import WORKLOADS
-            res["cpu_baseline"] = cpu_baseline(WORKLOADS[args.workload], dev, args.cpu_rows)
+            res["cpu_baseline"] = cpu_baseline(workload_of(args), dev, args.cpu_rows)
         print(json.dumps(res), flush=True)
     if world > 1:
         import torch.distributed as dist
