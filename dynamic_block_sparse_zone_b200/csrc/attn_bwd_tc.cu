@@ -11,19 +11,27 @@
 // upper half with rows it ignores).  The CTA walks the query blocks of the
 // key block's CSC column as 64-row chunks.
 //
-// Per chunk c (TMEM buffers alternate with c & 1):
-//   S^T  = K Q_c^T         M=128 keys, N=64 queries   -> TMEM ST[c&1]
-//   dP^T = V dO_c^T        M=128 keys, N=64 queries   -> TMEM DP[c&1]
-//   softmax warps: P^T, dS^T (bf16) over ST / DP, dS^T also to shared memory
+// Per chunk c:
+//   S^T  = K Q_c^T         M=128 keys, N=64 queries   -> TMEM ST[c%3]
+//   dP^T = V dO_c^T        M=128 keys, N=64 queries   -> TMEM DP
+//   softmax warps: P^T, dS^T (bf16, packed over their own ST columns),
+//                  dS^T also to shared memory
 //   dV  += P^T dO_c        A = P^T from TMEM          -> TMEM dV
 //   dK  += dS^T Q_c        A = dS^T from TMEM         -> TMEM dK
-//   dQ^T = K^T dS^T        both operands MN-major     -> TMEM ST[c&1]
+//   dQ^T = K^T dS^T        both operands MN-major     -> TMEM ST[c%3]
 //   drain warps: dQ^T rows (lane = head-dim index) -> fp32 reductions into dQ
-// TMEM columns: dK [0,128), dV [128,256), ST[2] [256,384), DP[2] [384,512).
+// Three ST buffers let S^T of chunk c+2 be issued while chunk c's dQ^T waits
+// to be drained; the single DP buffer is refilled (dP^T of chunk c+1) as soon
+// as the softmax of chunk c has read it.
+// TMEM columns: dK [0,128), dV [128,256), ST[3] [256,448), DP [448,512).
+// In an ST buffer, after the softmax, columns [32h, 32h+16) hold P^T and
+// [32h+16, 32h+32) hold dS^T of queries [32h, 32h+32) (h = 0, 1), packed as
+// bf16 pairs.
 //
-// Warp roles (320 threads): warp 0 TMA producer (K, V once; Q, dO, LSE,
-// Delta per chunk into a two-stage ring), warp 1 MMA issuer, warps 2..5
-// softmax (one key row each), warps 6..9 dQ drain (one head-dim row each).
+// Warp roles (448 threads): warp 0 TMA producer (K, V once; Q, dO, LSE,
+// Delta per chunk into a three-stage ring), warp 1 MMA issuer, warps 2..9
+// softmax (a key row and 32 of the 64 query columns each), warps 10..13 dQ
+// drain (one head-dim row each).
 #include <cuda.h>
 
 #include "tc_common.cuh"
@@ -34,9 +42,10 @@ using namespace tc;
 
 namespace bwdtc {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
+constexpr int kStages = 3;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColDK = 0, kColDV = 128, kColST = 256, kColDP = 384;
+constexpr uint32_t kColDK = 0, kColDV = 128, kColST = 256, kColDP = 448;
 
 template <int D>
 struct Layout {
@@ -47,11 +56,11 @@ struct Layout {
     static constexpr uint32_t kV = kK + 2 * kKVHalf;
     static constexpr uint32_t kQ0 = kV + 2 * kKVHalf;      // stage s: Q at kQ0 + s*kStage, dO at + 2*kQHalf
     static constexpr uint32_t kStage = 4 * kQHalf;
-    static constexpr uint32_t kDS = kQ0 + 2 * kStage;      // [2] x 128 key rows x 128 B (64 queries bf16)
-    static constexpr uint32_t kVec = kDS + 2 * 16384;      // stage s: LSE [64] f32 then Delta [64] f32
-    static constexpr uint32_t kBars = kVec + 2 * 512;
-    // kv, q_full[2], q_empty[2], s_full[2], p_full[2], dq_full[2], dq_empty[2], done
-    static constexpr uint32_t kNumBars = 14;
+    static constexpr uint32_t kDS = kQ0 + kStages * kStage;  // [2] x 128 key rows x 128 B (64 queries bf16)
+    static constexpr uint32_t kVec = kDS + 2 * 16384;        // stage s: LSE [64] f32 then Delta [64] f32
+    static constexpr uint32_t kBars = kVec + kStages * 512;
+    // kv, q_full[3], q_empty[3], s_full[2], p_full[2], dq_full[3], dq_empty[3], done
+    static constexpr uint32_t kNumBars = 18;
     static constexpr uint32_t kBytes = kBars + kNumBars * 8 + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;
 };
@@ -92,21 +101,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int o = 16; o > 0; o >>= 1) nchunk += __shfl_xor_sync(0xffffffffu, nchunk, o);
 
     const uint32_t bar_kv = sbase + L::kBars;
-    const uint32_t bar_qf = bar_kv + 8, bar_qe = bar_qf + 16, bar_sf = bar_qe + 16, bar_pf = bar_sf + 16;
-    const uint32_t bar_df = bar_pf + 16, bar_de = bar_df + 16, bar_done = bar_de + 16;
+    const uint32_t bar_qf = bar_kv + 8, bar_qe = bar_qf + 8 * kStages, bar_sf = bar_qe + 8 * kStages;
+    const uint32_t bar_pf = bar_sf + 16, bar_df = bar_pf + 16, bar_de = bar_df + 8 * kStages;
+    const uint32_t bar_done = bar_de + 8 * kStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBars + L::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kBars + L::kNumBars * 8 + 8);
 
     if (warp == 0) {
         if (lane == 0) {
             mbar_init(bar_kv, 1);
-            for (int s = 0; s < 2; ++s) {
+            for (int s = 0; s < kStages; ++s) {
                 mbar_init(bar_qf + 8 * s, 1);
                 mbar_init(bar_qe + 8 * s, 1);
-                mbar_init(bar_sf + 8 * s, 1);
-                mbar_init(bar_pf + 8 * s, 128);
                 mbar_init(bar_df + 8 * s, 1);
                 mbar_init(bar_de + 8 * s, 128);
+            }
+            for (int s = 0; s < 2; ++s) {
+                mbar_init(bar_sf + 8 * s, 1);
+                mbar_init(bar_pf + 8 * s, 256);
             }
             mbar_init(bar_done, 1);
             *abort_flag = 0;
@@ -144,8 +156,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             int issued = 0;
             for (int c = 0; c < nchunk; ++c) {
-                const int st = c & 1;
-                if (c >= 2 && !mbar_wait(bar_qe + 8 * st, ((c >> 1) + 1) & 1, status, kSiteQEmpty, abort_flag))
+                const int st = c % kStages;
+                if (c >= kStages &&
+                    !mbar_wait(bar_qe + 8 * st, ((c / kStages) + 1) & 1, status, kSiteQEmpty, abort_flag))
                     break;
                 const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + 2 * L::kQHalf;
                 const uint32_t sVec = sbase + L::kVec + st * 512;
@@ -164,8 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     r_end = bo[rowT[u] + 1];
                 }
             }
-            for (int c = max(0, issued - 2); c < issued; ++c)
-                mbar_wait(bar_qf + 8 * (c & 1), (c >> 1) & 1, status, kSiteQFull, abort_flag);
+            for (int c = max(0, issued - kStages); c < issued; ++c)
+                mbar_wait(bar_qf + 8 * (c % kStages), (c / kStages) & 1, status, kSiteQFull, abort_flag);
             mbar_wait(bar_kv, 0, status, kSiteKV, abort_flag);
         }
     } else if (warp == 1) {
@@ -175,11 +188,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idAcc = idesc_bf16(128, D, true);           // A from TMEM, B MN-major
             constexpr uint32_t idDQ = idesc_bf16(128, 64, true, true);     // A and B MN-major
             bool ok = mbar_wait(bar_kv, 0, status, kSiteKV, abort_flag);
-            auto stage_a = [&](int c) -> bool {  // S^T and dP^T of chunk c
-                const int st = c & 1;
-                if (!mbar_wait(bar_qf + 8 * st, (c >> 1) & 1, status, kSiteQFull, abort_flag)) return false;
+            auto issue_st = [&](int c) -> bool {  // S^T of chunk c into ST[c % 3]
+                const int st = c % kStages;
+                if (!mbar_wait(bar_qf + 8 * st, (c / kStages) & 1, status, kSiteQFull, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + 2 * L::kQHalf;
+                const uint32_t sQ = sbase + L::kQ0 + st * L::kStage;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ko = (kk >> 2) * L::kKVHalf + (kk & 3) * 32;
@@ -187,129 +200,132 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_ss(tmem + kColST + st * 64, sdesc(sbase + L::kK + ko, 16, 1024), sdesc(sQ + qo, 16, 1024),
                            idST, kk > 0);
                 }
+                return true;
+            };
+            auto issue_dp = [&](int c) {  // dP^T of chunk c into DP (stage already waited by issue_st)
+                const uint32_t sO = sbase + L::kQ0 + (c % kStages) * L::kStage + 2 * L::kQHalf;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ko = (kk >> 2) * L::kKVHalf + (kk & 3) * 32;
                     const uint32_t qo = (kk >> 2) * L::kQHalf + (kk & 3) * 32;
-                    mma_ss(tmem + kColDP + st * 64, sdesc(sbase + L::kV + ko, 16, 1024), sdesc(sO + qo, 16, 1024),
-                           idST, kk > 0);
+                    mma_ss(tmem + kColDP, sdesc(sbase + L::kV + ko, 16, 1024), sdesc(sO + qo, 16, 1024), idST,
+                           kk > 0);
                 }
-                tc_commit(bar_sf + 8 * st);
-                return true;
+                tc_commit(bar_sf + 8 * (c & 1));
             };
-            if (ok) ok = stage_a(0);
-            if (ok && nchunk > 1) ok = stage_a(1);
+            if (ok) {
+                ok = issue_st(0);
+                if (ok) issue_dp(0);
+            }
+            if (ok && nchunk > 1) ok = issue_st(1);
             for (int c = 0; ok && c < nchunk; ++c) {
-                const int st = c & 1;
-                if (!mbar_wait(bar_pf + 8 * st, (c >> 1) & 1, status, kSiteP, abort_flag)) break;
+                const int st = c % kStages;
+                if (!mbar_wait(bar_pf + 8 * (c & 1), (c >> 1) & 1, status, kSiteP, abort_flag)) break;
                 tc_fence_after();
+                if (c + 1 < nchunk) issue_dp(c + 1);
                 const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + 2 * L::kQHalf;
+                const uint32_t tST = tmem + kColST + st * 64;
                 const uint32_t acc = (c > 0) ? 1u : 0u;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + kColDV, tmem + kColST + st * 64 + kk * 8, sdesc(sO + kk * 2048, L::kQHalf, 1024),
+                    mma_ts(tmem + kColDV, tST + 32 * (kk >> 1) + 8 * (kk & 1), sdesc(sO + kk * 2048, L::kQHalf, 1024),
                            idAcc, acc | (kk > 0));
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + kColDK, tmem + kColDP + st * 64 + kk * 8, sdesc(sQ + kk * 2048, L::kQHalf, 1024),
-                           idAcc, acc | (kk > 0));
+                    mma_ts(tmem + kColDK, tST + 32 * (kk >> 1) + 16 + 8 * (kk & 1),
+                           sdesc(sQ + kk * 2048, L::kQHalf, 1024), idAcc, acc | (kk > 0));
                 tc_commit(bar_qe + 8 * st);
-                const uint32_t sDS = sbase + L::kDS + st * 16384;
+                const uint32_t sDS = sbase + L::kDS + (c & 1) * 16384;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tmem + kColST + st * 64, sdesc(sbase + L::kK + kk * 2048, L::kKVHalf, 1024),
-                           sdesc(sDS + kk * 2048, 8192, 1024), idDQ, kk > 0);
+                    mma_ss(tST, sdesc(sbase + L::kK + kk * 2048, L::kKVHalf, 1024), sdesc(sDS + kk * 2048, 8192, 1024),
+                           idDQ, kk > 0);
                 tc_commit(bar_df + 8 * st);
                 if (c + 2 < nchunk) {
-                    if (!mbar_wait(bar_de + 8 * st, (c >> 1) & 1, status, kSiteDQEmpty, abort_flag)) break;
-                    tc_fence_after();
-                    if (!stage_a(c + 2)) break;
+                    const int b2 = (c + 2) % kStages;  // = (c - 1) % 3: the buffer chunk c-1 used
+                    if (c >= 1 &&
+                        !mbar_wait(bar_de + 8 * b2, ((c - 1) / kStages) & 1, status, kSiteDQEmpty, abort_flag))
+                        break;
+                    if (!issue_st(c + 2)) break;
                 }
             }
             tc_commit(bar_done);
         }
-    } else if (warp < 6) {
+    } else if (warp < 10) {
         // ------------------------------------------------------------ softmax (key rows)
         const int quad = warp & 3;
+        const int hh = (warp - 2) >> 2;  // which 32 query columns
         const int rowid = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const bool live = rowid < kvalid;
         const float log2e = 1.4426950408889634f;
         bool ok = true;
         for (int c = 0; c < nchunk; ++c) {
-            const int st = c & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * st, (c >> 1) & 1, status, kSiteS, abort_flag) &&
-                                             mbar_wait(bar_qf + 8 * st, (c >> 1) & 1, status, kSiteQFull,
+            const int st = c % kStages;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * (c & 1), (c >> 1) & 1, status, kSiteS, abort_flag) &&
+                                             mbar_wait(bar_qf + 8 * st, (c / kStages) & 1, status, kSiteQFull,
                                                        abort_flag));
             if (!ok) break;
             tc_fence_after();
-            const float *vec = reinterpret_cast<const float *>(smem + L::kVec + st * 512);
-            const uint32_t tST = tmem + kColST + st * 64 + lane_off;
-            const uint32_t tDP = tmem + kColDP + st * 64 + lane_off;
-            uint8_t *dsrow = smem + L::kDS + st * 16384 + rowid * 128;
+            const float *vec = reinterpret_cast<const float *>(smem + L::kVec + st * 512) + hh * 32;
+            const uint32_t tST = tmem + kColST + st * 64 + 32 * hh + lane_off;
+            const uint32_t tDP = tmem + kColDP + 32 * hh + lane_off;
+            uint32_t sv[32], dv[32];
+            tmem_ld32(tST, sv);
+            tmem_ld32(tDP, dv);
+            tmem_wait_ld();
+            uint32_t pk[16], dk[16];
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t sv[32], dv[32];
-                tmem_ld32(tST + hf * 32, sv);
-                tmem_ld32(tDP + hf * 32, dv);
-                tmem_wait_ld();
-                uint32_t pk[16], dk[16];
+            for (int e = 0; e < 16; ++e) {
+                const int q = 2 * e;
+                float p0 = ex2(fmaf(__uint_as_float(sv[q]), scale_log2, -vec[q] * log2e));
+                float p1 = ex2(fmaf(__uint_as_float(sv[q + 1]), scale_log2, -vec[q + 1] * log2e));
+                float d0 = p0 * (__uint_as_float(dv[q]) - vec[64 + q]);
+                float d1 = p1 * (__uint_as_float(dv[q + 1]) - vec[64 + q + 1]);
+                if (!live) p0 = p1 = d0 = d1 = 0.f;
+                pk[e] = pack_bf16x2(p0, p1);
+                dk[e] = pack_bf16x2(d0, d1);
+            }
+            tmem_st16(tST, pk);
+            tmem_st16(tST + 16, dk);
+            uint8_t *dsrow = smem + L::kDS + (c & 1) * 16384 + rowid * 128;
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int q = hf * 32 + 2 * e;
-                    float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), scale_log2, -vec[q] * log2e));
-                    float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), scale_log2, -vec[q + 1] * log2e));
-                    float d0 = p0 * (__uint_as_float(dv[2 * e]) - vec[64 + q]);
-                    float d1 = p1 * (__uint_as_float(dv[2 * e + 1]) - vec[64 + q + 1]);
-                    if (!live) p0 = p1 = d0 = d1 = 0.f;
-                    pk[e] = pack_bf16x2(p0, p1);
-                    dk[e] = pack_bf16x2(d0, d1);
-                }
-                tmem_st16(tST + hf * 16, pk);
-                tmem_st16(tDP + hf * 16, dk);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int chunk = hf * 4 + j;
-                    *reinterpret_cast<uint4 *>(dsrow + ((chunk ^ (rowid & 7)) << 4)) =
-                        make_uint4(dk[4 * j], dk[4 * j + 1], dk[4 * j + 2], dk[4 * j + 3]);
-                }
+            for (int j = 0; j < 4; ++j) {
+                const int chunk = hh * 4 + j;
+                *reinterpret_cast<uint4 *>(dsrow + ((chunk ^ (rowid & 7)) << 4)) =
+                    make_uint4(dk[4 * j], dk[4 * j + 1], dk[4 * j + 2], dk[4 * j + 3]);
             }
             tmem_wait_st();
             fence_async_smem();
             tc_fence_before();
-            mbar_arrive(bar_pf + 8 * st);
+            mbar_arrive(bar_pf + 8 * (c & 1));
         }
-        // epilogue: dK (scaled) and dV rows to the user layout
+        // epilogue: the first warp group writes dK (scaled), the second dV
         if (ok && nchunk > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, status, kSiteDone, abort_flag));
         if (ok) {
             tc_fence_after();
             const int tok = live ? perm[(size_t)b * g.N + k0 + rowid] : 0;
-            __nv_bfloat16 *dkr = dK + (((size_t)b * g.N + tok) * g.heads + h) * D;
-            __nv_bfloat16 *dvr = dV + (((size_t)b * g.N + tok) * g.heads + h) * D;
+            __nv_bfloat16 *dst = (hh == 0 ? dK : dV) + (((size_t)b * g.N + tok) * g.heads + h) * D;
+            const uint32_t src = tmem + (hh == 0 ? kColDK : kColDV) + lane_off;
+            const float f = (hh == 0) ? scale : 1.0f;
 #pragma unroll 1
             for (int q = 0; q < D / 32; ++q) {
-                uint32_t a[32], v[32];
+                uint32_t a[32];
                 if (nchunk > 0) {
-                    tmem_ld32(tmem + kColDK + lane_off + q * 32, a);
-                    tmem_ld32(tmem + kColDV + lane_off + q * 32, v);
+                    tmem_ld32(src + q * 32, a);
                     tmem_wait_ld();
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) a[e] = v[e] = 0u;
+                    for (int e = 0; e < 32; ++e) a[e] = 0u;
                 }
-                uint4 pa[4], pv[4];
-                uint32_t *wa = reinterpret_cast<uint32_t *>(pa), *wv = reinterpret_cast<uint32_t *>(pv);
+                uint4 pa[4];
+                uint32_t *wa = reinterpret_cast<uint32_t *>(pa);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    wa[e] = pack_bf16x2(__uint_as_float(a[2 * e]) * scale, __uint_as_float(a[2 * e + 1]) * scale);
-                    wv[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-                }
+                for (int e = 0; e < 16; ++e)
+                    wa[e] = pack_bf16x2(__uint_as_float(a[2 * e]) * f, __uint_as_float(a[2 * e + 1]) * f);
                 if (live) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        reinterpret_cast<uint4 *>(dkr + q * 32)[e] = pa[e];
-                        reinterpret_cast<uint4 *>(dvr + q * 32)[e] = pv[e];
-                    }
+                    for (int e = 0; e < 4; ++e) reinterpret_cast<uint4 *>(dst + q * 32)[e] = pa[e];
                 }
             }
         }
@@ -324,8 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             r_end = bo[rowT[u] + 1];
         }
         for (int c = 0; c < nchunk; ++c) {
-            const int st = c & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(bar_df + 8 * st, (c >> 1) & 1, status, kSiteDQFull, abort_flag)))
+            const int st = c % kStages;
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(bar_df + 8 * st, (c / kStages) & 1, status, kSiteDQFull, abort_flag)))
                 break;
             tc_fence_after();
             uint32_t v[64];
