@@ -29,7 +29,7 @@
 // bf16 pairs.
 //
 // Warp roles (448 threads): warp 0 TMA producer (K, V once; Q, dO, LSE,
-// Delta per chunk into a three-stage ring), warp 1 MMA issuer, warps 2..9
+// Delta per chunk into a three-stage ring; LSE is kept in log2 units), warp 1 MMA issuer, warps 2..9
 // softmax (a key row and 32 of the 64 query columns each), warps 10..13 dQ
 // drain (one head-dim row each).
 #include <cuda.h>
@@ -183,14 +183,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && nchunk > 0) {
+        if (nchunk > 0) {  // the whole warp runs the issue loop; elect.sync picks one lane
             constexpr uint32_t idST = idesc_bf16(128, 64, false);          // K-major A and B
             constexpr uint32_t idAcc = idesc_bf16(128, D, true);           // A from TMEM, B MN-major
             constexpr uint32_t idDQ = idesc_bf16(128, 64, true, true);     // A and B MN-major
-            bool ok = mbar_wait(bar_kv, 0, status, kSiteKV, abort_flag);
+            bool ok = __all_sync(0xffffffffu, mbar_wait(bar_kv, 0, status, kSiteKV, abort_flag));
             auto issue_st = [&](int c) -> bool {  // S^T of chunk c into ST[c % 3]
                 const int st = c % kStages;
-                if (!mbar_wait(bar_qf + 8 * st, (c / kStages) & 1, status, kSiteQFull, abort_flag)) return false;
+                if (!__all_sync(0xffffffffu, mbar_wait(bar_qf + 8 * st, (c / kStages) & 1, status, kSiteQFull, abort_flag))) return false;
                 tc_fence_after();
                 const uint32_t sQ = sbase + L::kQ0 + st * L::kStage;
 #pragma unroll
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_ss(tmem + kColDP, sdesc(sbase + L::kV + ko, 16, 1024), sdesc(sO + qo, 16, 1024), idST,
                            kk > 0);
                 }
-                tc_commit(bar_sf + 8 * (c & 1));
+                mma_commit(bar_sf + 8 * (c & 1));
             };
             if (ok) {
                 ok = issue_st(0);
@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok && nchunk > 1) ok = issue_st(1);
             for (int c = 0; ok && c < nchunk; ++c) {
                 const int st = c % kStages;
-                if (!mbar_wait(bar_pf + 8 * (c & 1), (c >> 1) & 1, status, kSiteP, abort_flag)) break;
+                if (!__all_sync(0xffffffffu, mbar_wait(bar_pf + 8 * (c & 1), (c >> 1) & 1, status, kSiteP, abort_flag))) break;
                 tc_fence_after();
                 if (c + 1 < nchunk) issue_dp(c + 1);
                 const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + 2 * L::kQHalf;
@@ -234,22 +234,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < 4; ++kk)
                     mma_ts(tmem + kColDK, tST + 32 * (kk >> 1) + 16 + 8 * (kk & 1),
                            sdesc(sQ + kk * 2048, L::kQHalf, 1024), idAcc, acc | (kk > 0));
-                tc_commit(bar_qe + 8 * st);
+                mma_commit(bar_qe + 8 * st);
                 const uint32_t sDS = sbase + L::kDS + (c & 1) * 16384;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss(tST, sdesc(sbase + L::kK + kk * 2048, L::kKVHalf, 1024), sdesc(sDS + kk * 2048, 8192, 1024),
                            idDQ, kk > 0);
-                tc_commit(bar_df + 8 * st);
+                mma_commit(bar_df + 8 * st);
                 if (c + 2 < nchunk) {
                     const int b2 = (c + 2) % kStages;  // = (c - 1) % 3: the buffer chunk c-1 used
                     if (c >= 1 &&
-                        !mbar_wait(bar_de + 8 * b2, ((c - 1) / kStages) & 1, status, kSiteDQEmpty, abort_flag))
+                        !__all_sync(0xffffffffu, mbar_wait(bar_de + 8 * b2, ((c - 1) / kStages) & 1, status, kSiteDQEmpty, abort_flag)))
                         break;
                     if (!issue_st(c + 2)) break;
                 }
             }
-            tc_commit(bar_done);
+            mma_commit(bar_done);
         }
     } else if (warp < 10) {
         // ------------------------------------------------------------ softmax (key rows)
@@ -258,7 +258,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int rowid = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const bool live = rowid < kvalid;
-        const float log2e = 1.4426950408889634f;
         bool ok = true;
         for (int c = 0; c < nchunk; ++c) {
             const int st = c % kStages;
@@ -278,8 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int q = 2 * e;
-                float p0 = ex2(fmaf(__uint_as_float(sv[q]), scale_log2, -vec[q] * log2e));
-                float p1 = ex2(fmaf(__uint_as_float(sv[q + 1]), scale_log2, -vec[q + 1] * log2e));
+                float p0 = ex2(fmaf(__uint_as_float(sv[q]), scale_log2, -vec[q]));
+                float p1 = ex2(fmaf(__uint_as_float(sv[q + 1]), scale_log2, -vec[q + 1]));
                 float d0 = p0 * (__uint_as_float(dv[q]) - vec[64 + q]);
                 float d1 = p1 * (__uint_as_float(dv[q + 1]) - vec[64 + q + 1]);
                 if (!live) p0 = p1 = d0 = d1 = 0.f;

@@ -256,9 +256,9 @@ __global__ void __launch_bounds__(128, 2)
 #pragma unroll
         for (int rh = 0; rh < 2; ++rh) {
             const int n = tile * 64 + warp * 16 + gr + rh * 8;
-            const float lse = (mrow[rh] + log2f(lrow[rh])) * 0.69314718055994531f;
-            lse_p[(size_t)bh * g.N + n] = lse;
-            if (lse_user) lse_user[(size_t)bh * g.N + perm[(size_t)b * g.N + n]] = lse;
+            const float lse2 = mrow[rh] + log2f(lrow[rh]);  // log2 units
+            lse_p[(size_t)bh * g.N + n] = lse2;
+            if (lse_user) lse_user[(size_t)bh * g.N + perm[(size_t)b * g.N + n]] = lse2 * 0.69314718055994531f;
         }
     }
     __syncwarp();
@@ -340,7 +340,6 @@ __global__ void __launch_bounds__(128, 2)
     const __nv_bfloat16 *dOh = dOp + (size_t)bh * g.N * D;
     const float *Lh = lse_p + (size_t)bh * g.N;
     const float *Dh = delta + (size_t)bh * g.N;
-    const float log2e = 1.4426950408889634f;
 
     ChunkWalk cw;
     cw.init(rowT, colT_ptr[colid], colT_ptr[colid + 1], bo);
@@ -350,7 +349,7 @@ __global__ void __launch_bounds__(128, 2)
         TL::load(sQ0, Qh + (size_t)cw.row() * D, tid);
         TL::load(sO0, dOh + (size_t)cw.row() * D, tid);
         if (tid < 64) {
-            sL[tid] = Lh[cw.row() + tid] * log2e;
+            sL[tid] = Lh[cw.row() + tid];
             sDl[tid] = Dh[cw.row() + tid];
         }
     }
@@ -373,7 +372,7 @@ __global__ void __launch_bounds__(128, 2)
             TL::load(sQ0 + (stage ^ 1) * TL::kBytes, Qh + (size_t)nx.row() * D, tid);
             TL::load(sO0 + (stage ^ 1) * TL::kBytes, dOh + (size_t)nx.row() * D, tid);
             if (tid < 64) {
-                sL[(stage ^ 1) * 64 + tid] = Lh[nx.row() + tid] * log2e;
+                sL[(stage ^ 1) * 64 + tid] = Lh[nx.row() + tid];
                 sDl[(stage ^ 1) * 64 + tid] = Dh[nx.row() + tid];
             }
         }
@@ -397,7 +396,7 @@ __global__ void __launch_bounds__(128, 2)
                 mma16816(st[2 * np + 1], a, bfr[2], bfr[3]);
             }
         }
-        // P^T = exp2(s * scale*log2e - LSE_q*log2e); the column index is the query
+        // P^T = exp2(s * scale*log2e - LSE2_q) (LSE kept in log2 units); the column index is the query
 #pragma unroll
         for (int n = 0; n < 8; ++n) {
             const int q = n * 8 + 2 * t4;

@@ -179,13 +179,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        {  // the whole warp runs the issue loop; elect.sync picks one lane
             constexpr uint32_t idS128 = idesc_bf16(128, 128, false), idS64 = idesc_bf16(128, 64, false);
             constexpr uint32_t idPV = idesc_bf16(128, D, true);
-            bool ok = mbar_wait(bar_q, 0, status, kSiteQ, abort_flag);
+            bool ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, status, kSiteQ, abort_flag));
             auto issue_s = [&](int c) -> bool {
                 const int st = c % kStages;
-                if (!mbar_wait(bar_k + 8 * st, (c / kStages) & 1, status, kSiteK, abort_flag)) return false;
+                if (!__all_sync(0xffffffffu, mbar_wait(bar_k + 8 * st, (c / kStages) & 1, status, kSiteK, abort_flag))) return false;
                 tc_fence_after();
                 const uint32_t sK = sbase + L::kK0 + st * L::kStageBytes;
                 const bool full = (2 * c + 1) < nseg;
@@ -195,23 +195,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_ss(tS0 + (c & 1) * 128, sdesc(sbase + L::kQ + off, 16, 1024), sdesc(sK + off, 16, 1024),
                            full ? idS128 : idS64, kk > 0);
                 }
-                tc_commit(bar_s + 8 * (c & 1));
+                mma_commit(bar_s + 8 * (c & 1));
                 return true;
             };
             if (ok && nchunk > 0) ok = issue_s(0);
             for (int c = 0; ok && c < nchunk; ++c) {
                 if (c + 1 < nchunk && !issue_s(c + 1)) break;
                 const int st = c % kStages;
-                if (!mbar_wait(bar_p + 8 * (c & 1), (c >> 1) & 1, status, kSiteP, abort_flag)) break;
-                if (!mbar_wait(bar_v + 8 * st, (c / kStages) & 1, status, kSiteV, abort_flag)) break;
+                if (!__all_sync(0xffffffffu, mbar_wait(bar_p + 8 * (c & 1), (c >> 1) & 1, status, kSiteP, abort_flag))) break;
+                if (!__all_sync(0xffffffffu, mbar_wait(bar_v + 8 * st, (c / kStages) & 1, status, kSiteV, abort_flag))) break;
                 tc_fence_after();
                 const uint32_t sV = sbase + L::kK0 + st * L::kStageBytes + L::kHalves * L::kTileBytes;
                 const int nk = ((2 * c + 1) < nseg) ? 128 : 64;
                 for (int kk = 0; kk < nk / 16; ++kk)
                     mma_ts(tO, tS0 + (c & 1) * 128 + kk * 8, sdesc(sV + kk * 2048, L::kTileBytes, 1024), idPV,
                            (c > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(bar_e + 8 * st);
-                tc_commit(bar_o);
+                mma_commit(bar_e + 8 * st);
+                mma_commit(bar_o);
             }
         }
     } else {
@@ -330,9 +330,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (write) {
-                const float lse = (m + __log2f(l)) * 0.69314718055994531f;
-                lse_p[(size_t)bh * g.N + n] = lse;
-                if (lse_user) lse_user[(size_t)bh * g.N + tok] = lse;
+                const float lse2 = m + __log2f(l);  // log2 units, as the backward consumes it
+                lse_p[(size_t)bh * g.N + n] = lse2;
+                if (lse_user) lse_user[(size_t)bh * g.N + tok] = lse2 * 0.69314718055994531f;
             }
         }
     }
