@@ -19,7 +19,8 @@
 //   dV  += P^T dO_c        A = P^T from TMEM          -> TMEM dV
 //   dK  += dS^T Q_c        A = dS^T from TMEM         -> TMEM dK
 //   dQ^T = K^T dS^T        both operands MN-major     -> TMEM ST[c%3]
-//   drain warps: dQ^T rows (lane = head-dim index) -> fp32 reductions into dQ
+//   drain warps: dQ^T rows (lane = head-dim index) -> a [64 x D] fp32 tile in
+//                shared memory -> one TMA reduce-add into the dQ accumulator
 // Three ST buffers let S^T of chunk c+2 be issued while chunk c's dQ^T waits
 // to be drained; the single DP buffer is refilled (dP^T of chunk c+1) as soon
 // as the softmax of chunk c has read it.
@@ -58,11 +59,14 @@ struct Layout {
     static constexpr uint32_t kStage = 4 * kQHalf;
     static constexpr uint32_t kDS = kQ0 + kStages * kStage;  // [2] x 128 key rows x 128 B (64 queries bf16)
     static constexpr uint32_t kVec = kDS + 2 * 16384;        // stage s: LSE [64] f32 then Delta [64] f32
-    static constexpr uint32_t kBars = kVec + kStages * 512;
+    static constexpr uint32_t kDQ = kVec + kStages * 512;    // dQ staging tile [64 queries][D] f32 (128-B aligned)
+    static constexpr uint32_t kBars = kDQ + 64 * D * 4;
     // kv, q_full[3], q_empty[3], s_full[2], p_full[2], dq_full[3], dq_empty[3], done
     static constexpr uint32_t kNumBars = 18;
     static constexpr uint32_t kBytes = kBars + kNumBars * 8 + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;
+    static_assert(kAlloc <= 232448, "shared memory per block");
+    static_assert(kDQ % 128 == 0, "TMA source alignment");
 };
 
 enum { kSiteKV = 11, kSiteQFull, kSiteQEmpty, kSiteS, kSiteP, kSiteDQFull, kSiteDQEmpty, kSiteDone };
@@ -70,7 +74,8 @@ enum { kSiteKV = 11, kSiteQFull, kSiteQEmpty, kSiteS, kSiteP, kSiteDQFull, kSite
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO, Geo g,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                  const __grid_constant__ CUtensorMap tmdQ, Geo g,
                   const int *__restrict__ nqt, const int *__restrict__ qt_row, const int *__restrict__ qt_blk,
                   const int *__restrict__ blk_off, const int *__restrict__ colT_ptr, const int *__restrict__ rowT,
                   const int *__restrict__ perm, const float *__restrict__ lse_p, const float *__restrict__ delta,
@@ -127,6 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_map(&tmK);
             prefetch_map(&tmV);
             prefetch_map(&tmdO);
+            prefetch_map(&tmdQ);
         }
         __syncwarp();
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -274,16 +280,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(tDP, dv);
             tmem_wait_ld();
             uint32_t pk[16], dk[16];
+            const float4 *lse4 = reinterpret_cast<const float4 *>(vec);
+            const float4 *del4 = reinterpret_cast<const float4 *>(vec + 64);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int q = 2 * e;
-                float p0 = ex2(fmaf(__uint_as_float(sv[q]), scale_log2, -vec[q]));
-                float p1 = ex2(fmaf(__uint_as_float(sv[q + 1]), scale_log2, -vec[q + 1]));
-                float d0 = p0 * (__uint_as_float(dv[q]) - vec[64 + q]);
-                float d1 = p1 * (__uint_as_float(dv[q + 1]) - vec[64 + q + 1]);
-                if (!live) p0 = p1 = d0 = d1 = 0.f;
-                pk[e] = pack_bf16x2(p0, p1);
-                dk[e] = pack_bf16x2(d0, d1);
+            for (int e4 = 0; e4 < 8; ++e4) {
+                const float4 L4 = lse4[e4], D4 = del4[e4];
+                const int q = 4 * e4;
+                float p0 = ex2(fmaf(__uint_as_float(sv[q]), scale_log2, -L4.x));
+                float p1 = ex2(fmaf(__uint_as_float(sv[q + 1]), scale_log2, -L4.y));
+                float p2 = ex2(fmaf(__uint_as_float(sv[q + 2]), scale_log2, -L4.z));
+                float p3 = ex2(fmaf(__uint_as_float(sv[q + 3]), scale_log2, -L4.w));
+                float d0 = p0 * (__uint_as_float(dv[q]) - D4.x);
+                float d1 = p1 * (__uint_as_float(dv[q + 1]) - D4.y);
+                float d2 = p2 * (__uint_as_float(dv[q + 2]) - D4.z);
+                float d3 = p3 * (__uint_as_float(dv[q + 3]) - D4.w);
+                if (!live) p0 = p1 = p2 = p3 = d0 = d1 = d2 = d3 = 0.f;
+                pk[2 * e4] = pack_bf16x2(p0, p1);
+                pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
+                dk[2 * e4] = pack_bf16x2(d0, d1);
+                dk[2 * e4 + 1] = pack_bf16x2(d2, d3);
             }
             tmem_st16(tST, pk);
             tmem_st16(tST + 16, dk);
@@ -333,6 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp & 3;
         const int d = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const bool leader = (warp == 10 && lane == 0);
         int u = u_begin, r = 0, r_end = 0;
         if (u < u_end) {
             r = bo[rowT[u]];
@@ -350,15 +366,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar_de + 8 * st);
-            float *dst = dQacc + ((size_t)rowbase + r) * D + d;
+            // the staging tile is free once the previous reduce has read it
+            if (leader) bulk_wait_read_all();
+            named_bar_sync(1, 128);
+            float *stage = reinterpret_cast<float *>(smem + L::kDQ) + d;
 #pragma unroll
-            for (int q = 0; q < 64; ++q) atomicAdd(dst + (size_t)q * D, __uint_as_float(v[q]) * scale);
+            for (int q = 0; q < 64; ++q) stage[q * D] = __uint_as_float(v[q]) * scale;
+            fence_async_smem();
+            named_bar_sync(1, 128);
+            if (leader) {
+                tma_reduce_add_2d(&tmdQ, sbase + L::kDQ, 0, rowbase + r);
+                bulk_commit();
+            }
             r += 64;
             if (r >= r_end && ++u < u_end) {
                 r = bo[rowT[u]];
                 r_end = bo[rowT[u] + 1];
             }
         }
+        if (leader) bulk_wait_all();  // every reduce has landed before the CTA exits
     }
     tc_fence_before();
     __syncthreads();
@@ -383,7 +409,7 @@ prism_status launch_attn_bwd_tc_main(Plan &pl, void *dK, void *dV, cudaStream_t 
     const double scale = 1.0 / sqrt((double)g.D);
     TimerScope ts(pl, kTAttnBwd, st);
     bwdtc::k_attn_bwd_tc<128><<<dim3(g.nbmax, g.batch * g.heads), bwdtc::kThreads, bwdtc::Layout<128>::kAlloc, st>>>(
-        pl.tmQ, pl.tmK, pl.tmV, pl.tmdO, g, pl.nqt, pl.qt_row, pl.qt_blk, pl.blk_off, pl.colT_ptr, pl.rowT, pl.perm,
+        pl.tmQ, pl.tmK, pl.tmV, pl.tmdO, pl.tmdQ, g, pl.nqt, pl.qt_row, pl.qt_blk, pl.blk_off, pl.colT_ptr, pl.rowT, pl.perm,
         pl.lse_p, pl.delta, pl.dQacc, static_cast<__nv_bfloat16 *>(dK), static_cast<__nv_bfloat16 *>(dV),
         (float)scale, (float)(scale * 1.4426950408889634), pl.status);
     PRISM_CUDA_OK(cudaGetLastError());

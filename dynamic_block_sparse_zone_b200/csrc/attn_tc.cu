@@ -381,12 +381,29 @@ static prism_status make_map(CUtensorMap *m, const void *base, uint64_t rows, ui
     return PRISM_OK;
 }
 
+// 2D map over a [rows][D] fp32 matrix, boxes of 64 rows x D columns, no
+// swizzle (reduce-add target of the backward's dQ tiles).
+static prism_status make_map_f32_rows(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(PRISM_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 4};
+    cuuint32_t box[2] = {(cuuint32_t)cols, 64};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PRISM_ERR_CUDA, "cuTensorMapEncodeTiled (fp32) failed (%d)", (int)r);
+    return PRISM_OK;
+}
+
 prism_status make_tensor_maps(Plan &pl) {
     const uint64_t rows = (uint64_t)pl.g.batch * pl.g.heads * pl.g.N;
     prism_status s = make_map(&pl.tmQ, pl.Qp, rows, pl.g.D);
     if (s == PRISM_OK) s = make_map(&pl.tmK, pl.Kp, rows, pl.g.D);
     if (s == PRISM_OK) s = make_map(&pl.tmV, pl.Vp, rows, pl.g.D);
     if (s == PRISM_OK) s = make_map(&pl.tmdO, pl.dOp, rows, pl.g.D);
+    if (s == PRISM_OK) s = make_map_f32_rows(&pl.tmdQ, pl.dQacc, rows, pl.g.D);
     return s;
 }
 

@@ -77,6 +77,7 @@ struct Plan {
     int use_legacy_fwd;     // development switch: warp-MMA forward instead of tcgen05
     // TMA descriptors of the permuted copies, viewed as [batch*heads*N][D] bf16
     CUtensorMap tmQ, tmK, tmV, tmdO;
+    CUtensorMap tmdQ;       // fp32 [batch*heads*N][D], 64-row boxes, reduce-add target
 };
 
 // Records CUDA events around the launches in its scope when timing is on.
