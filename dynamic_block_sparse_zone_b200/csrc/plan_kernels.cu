@@ -564,9 +564,11 @@ __device__ __forceinline__ int block_scan_256(int v, int *buf, int *tot) {
     return before + x - v;
 }
 
+constexpr int kSelSlice = 16;  // pooled-key channels staged per pass (128 B of a row)
+
 struct SelSmem {
     // layout inside the dynamic buffer (offsets in bytes)
-    size_t qbar, keys, sk, sj, pr, bits;
+    size_t qbar, keys, sk, sj, pr, bits, tile;
     size_t bytes;
 };
 
@@ -586,6 +588,8 @@ __host__ __device__ inline SelSmem sel_smem_layout(int D, int nbmax, int cap_str
     L.pr = o;   o += (size_t)SP * 8;
     L.sj = o;   o += (size_t)SP * 4;
     L.bits = o; o += (size_t)((nbmax + 31) / 32) * 4;
+    o = (o + 15) & ~(size_t)15;
+    L.tile = o; o += (size_t)kSelThreads * (kSelSlice + 1) * 8;  // [256 rows][16 channels + 1 pad] fp64
     L.bytes = (o + 15) & ~(size_t)15;
     return L;
 }
@@ -622,18 +626,34 @@ __global__ void __launch_bounds__(kSelThreads) k_select(Geo g, const int *__rest
     // scores
     const double sqrtD = __dsqrt_rn((double)g.D);
     const double *kb = Kbar + (size_t)bh * g.nbmax * g.D;
+    double *tile = reinterpret_cast<double *>(sel_raw + L.tile);
     unsigned long long kmax = 0;
-    for (int j = tid; j < nb; j += kSelThreads) {
-        const double2 *kr = reinterpret_cast<const double2 *>(kb + (size_t)j * g.D);
+    // Thread t scores block j0 + t.  Pooled-key rows are staged through shared
+    // memory 16 channels at a time with coalesced loads; each thread still sums
+    // its dot product over the channels in ascending order.
+    for (int j0 = 0; j0 < nb; j0 += kSelThreads) {
+        const int j = j0 + tid;
         double dot = 0.0;
-        for (int c = 0; c < g.D / 2; ++c) {
-            const double2 kv = kr[c];
-            dot = __dadd_rn(dot, __dmul_rn(qbar[2 * c], kv.x));
-            dot = __dadd_rn(dot, __dmul_rn(qbar[2 * c + 1], kv.y));
+        for (int c0 = 0; c0 < g.D; c0 += kSelSlice) {
+            for (int idx = tid; idx < kSelThreads * (kSelSlice / 2); idx += kSelThreads) {
+                const int rr = idx / (kSelSlice / 2), part = idx % (kSelSlice / 2);
+                double2 v = make_double2(0.0, 0.0);
+                if (j0 + rr < nb)
+                    v = *reinterpret_cast<const double2 *>(kb + (size_t)(j0 + rr) * g.D + c0 + 2 * part);
+                tile[rr * (kSelSlice + 1) + 2 * part] = v.x;
+                tile[rr * (kSelSlice + 1) + 2 * part + 1] = v.y;
+            }
+            __syncthreads();
+            const double *tr = tile + tid * (kSelSlice + 1);
+#pragma unroll
+            for (int c = 0; c < kSelSlice; ++c) dot = __dadd_rn(dot, __dmul_rn(qbar[c0 + c], tr[c]));
+            __syncthreads();
         }
-        const uint64_t key = order_key(__ddiv_rn(dot, sqrtD));
-        keys[j] = key;
-        kmax = key > kmax ? key : kmax;
+        if (j < nb) {
+            const uint64_t key = order_key(__ddiv_rn(dot, sqrtD));
+            keys[j] = key;
+            kmax = key > kmax ? key : kmax;
+        }
     }
     kmax = block_max_u64(kmax, ured);
     const double zmax = key_value(kmax);
