@@ -9,16 +9,20 @@
 // are computed and discarded).  The selected key blocks are streamed as
 // 64-row segments; two segments form a 128-key chunk.
 //
+// Two CTAs share an SM (96 KB of shared memory and 256 TMEM columns each), so
+// while one CTA's softmax works the tensor cores run the other CTA's MMAs;
+// inside a CTA the chunk pipeline is strictly ordered:
+//   S_c = Q K_c^T (TMEM S) -> softmax (P_c over S, bf16) -> O += P_c V_c -> S_{c+1}
 // Warp roles (192 threads):
-//   warp 0       TMA producer: Q tile once, then K and V chunks into a
-//                two-stage ring (each stage 128 keys x D, 128-byte swizzle).
-//   warp 1       MMA issuer (one thread): S_c = Q K_c^T into one of two TMEM
-//                S buffers, then O += P_c V_c with P_c read from TMEM.
-//   warps 2..5   softmax, one query row per thread (= TMEM lane): row max,
-//                exp2, running sum; P_c written back over S_c as bf16; O is
-//                rescaled in TMEM only when the running max grows by more
-//                than 2^8.  Epilogue: O / l to the user layout, log-sum-exp.
-// TMEM columns: S buffer 0 [0,128), S buffer 1 [128,256), O [256, 256+D).
+//   warp 0       TMA producer: Q once; K_c into the K buffer once S_{c-1} has
+//                read it, V_c into the V buffer once P_{c-1} V_{c-1} has.
+//   warp 1       MMA issuer (whole warp, one elected lane issues).
+//   warps 2..5   softmax, one query row per thread (= TMEM lane): pass 1 row
+//                max, pass 2 exp2 / running sum / bf16 P written back over S.
+//                O is rescaled in TMEM only when the running max grows by more
+//                than 2^8 (it is current then: S_c was issued after PV_{c-1}).
+//                Epilogue: O / l to the user layout, log-sum-exp.
+// TMEM columns: S / P [0,128), O [128, 128+D).
 #include <cuda.h>
 
 #include "tc_common.cuh"
@@ -30,8 +34,7 @@ using namespace tc;
 namespace fwdtc {
 
 constexpr int kThreads = 192;
-constexpr int kStages = 2;
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemCols = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int D>
@@ -39,20 +42,20 @@ struct Layout {
     static constexpr int kHalves = D / 64;               // 64-column (128 B) swizzle atoms along D
     static constexpr uint32_t kTileBytes = 128 * 128;    // 128 rows x 128 B
     static constexpr uint32_t kQ = 0;
-    static constexpr uint32_t kK0 = kQ + kHalves * kTileBytes;
-    static constexpr uint32_t kStageBytes = 2 * kHalves * kTileBytes;  // K and V
-    static constexpr uint32_t kBars = kK0 + kStages * kStageBytes;
-    // barriers: q, k[S], v[S], kv_empty[S], s[2], p[2], o  (8 B each) + tmem slot + abort
-    static constexpr uint32_t kNumBars = 1 + 3 * kStages + 2 + 2 + 1;
+    static constexpr uint32_t kK = kQ + kHalves * kTileBytes;
+    static constexpr uint32_t kV = kK + kHalves * kTileBytes;
+    static constexpr uint32_t kBars = kV + kHalves * kTileBytes;
+    // barriers: q, k_full, k_empty, v_full, v_empty, s, p, o  (8 B each) + tmem slot + abort
+    static constexpr uint32_t kNumBars = 8;
     static constexpr uint32_t kBytes = kBars + kNumBars * 8 + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;  // slack to align the base to 1024
 };
 
 // Site codes recorded with a timeout.
-enum { kSiteQ = 1, kSiteK, kSiteV, kSiteEmpty, kSiteS, kSiteP, kSiteO };
+enum { kSiteQ = 1, kSiteK, kSiteV, kSiteKEmpty, kSiteVEmpty, kSiteS, kSiteP, kSiteO };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, Geo g, const int *__restrict__ nqt,
                   const int *__restrict__ qt_row, const int *__restrict__ qt_blk, const int *__restrict__ blk_off,
@@ -86,27 +89,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nchunk = (nseg + 1) >> 1;
 
     const uint32_t bar_q = sbase + L::kBars;
-    const uint32_t bar_k = bar_q + 8;                  // [kStages]
-    const uint32_t bar_v = bar_k + 8 * kStages;        // [kStages]
-    const uint32_t bar_e = bar_v + 8 * kStages;        // [kStages] kv stage empty
-    const uint32_t bar_s = bar_e + 8 * kStages;        // [2]
-    const uint32_t bar_p = bar_s + 16;                 // [2]
-    const uint32_t bar_o = bar_p + 16;
+    const uint32_t bar_kf = bar_q + 8, bar_ke = bar_q + 16, bar_vf = bar_q + 24, bar_ve = bar_q + 32;
+    const uint32_t bar_s = bar_q + 40, bar_p = bar_q + 48, bar_o = bar_q + 56;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBars + L::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kBars + L::kNumBars * 8 + 8);
 
     if (warp == 0) {
         if (lane == 0) {
             mbar_init(bar_q, 1);
-            for (int s = 0; s < kStages; ++s) {
-                mbar_init(bar_k + 8 * s, 1);
-                mbar_init(bar_v + 8 * s, 1);
-                mbar_init(bar_e + 8 * s, 1);
-            }
-            for (int s = 0; s < 2; ++s) {
-                mbar_init(bar_s + 8 * s, 1);
-                mbar_init(bar_p + 8 * s, 128);
-            }
+            mbar_init(bar_kf, 1);
+            mbar_init(bar_ke, 1);
+            mbar_init(bar_vf, 1);
+            mbar_init(bar_ve, 1);
+            mbar_init(bar_s, 1);
+            mbar_init(bar_p, 128);
             mbar_init(bar_o, 1);
             *abort_flag = 0;
             mbar_fence_init();
@@ -122,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS0 = tmem, tO = tmem + 256;
+    const uint32_t tS = tmem, tO = tmem + 128;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -138,16 +134,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 r = bo[col[u]];
                 r_end = bo[col[u] + 1];
             }
-            int issued = 0;
+            int kissued = 0, vissued = 0;
             for (int c = 0; c < nchunk; ++c) {
-                const int st = c % kStages;
-                if (c >= kStages && !mbar_wait(bar_e + 8 * st, ((c / kStages) + 1) & 1, status, kSiteEmpty,
-                                               abort_flag))
-                    break;
                 const int nsg = min(2, nseg - 2 * c);
                 const uint32_t bytes = nsg * 64 * D * 2;
-                const uint32_t sK = sbase + L::kK0 + st * L::kStageBytes;
-                const uint32_t sV = sK + L::kHalves * L::kTileBytes;
                 int rows[2];
                 for (int gsg = 0; gsg < nsg; ++gsg) {
                     rows[gsg] = r;
@@ -157,24 +147,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                         r_end = bo[col[u] + 1];
                     }
                 }
-                mbar_expect_tx(bar_k + 8 * st, bytes);
+                // K_c once S_{c-1} has consumed the K buffer
+                if (c > 0 && !mbar_wait(bar_ke, (c - 1) & 1, status, kSiteKEmpty, abort_flag)) break;
+                mbar_expect_tx(bar_kf, bytes);
                 for (int gsg = 0; gsg < nsg; ++gsg)
                     for (int hf = 0; hf < L::kHalves; ++hf)
-                        tma_load_2d(sK + hf * L::kTileBytes + gsg * 8192, &tmK, bar_k + 8 * st, hf * 64,
+                        tma_load_2d(sbase + L::kK + hf * L::kTileBytes + gsg * 8192, &tmK, bar_kf, hf * 64,
                                     rowbase + rows[gsg]);
-                mbar_expect_tx(bar_v + 8 * st, bytes);
+                kissued = c + 1;
+                // V_c once P_{c-1} V_{c-1} has consumed the V buffer
+                if (c > 0 && !mbar_wait(bar_ve, (c - 1) & 1, status, kSiteVEmpty, abort_flag)) break;
+                mbar_expect_tx(bar_vf, bytes);
                 for (int gsg = 0; gsg < nsg; ++gsg)
                     for (int hf = 0; hf < L::kHalves; ++hf)
-                        tma_load_2d(sV + hf * L::kTileBytes + gsg * 8192, &tmV, bar_v + 8 * st, hf * 64,
+                        tma_load_2d(sbase + L::kV + hf * L::kTileBytes + gsg * 8192, &tmV, bar_vf, hf * 64,
                                     rowbase + rows[gsg]);
-                issued = c + 1;
+                vissued = c + 1;
             }
             // drain: every issued load must land before the CTA may exit
-            for (int c = max(0, issued - kStages); c < issued; ++c) {
-                const int st = c % kStages;
-                mbar_wait(bar_k + 8 * st, (c / kStages) & 1, status, kSiteK, abort_flag);
-                mbar_wait(bar_v + 8 * st, (c / kStages) & 1, status, kSiteV, abort_flag);
-            }
+            if (kissued > 0) mbar_wait(bar_kf, (kissued - 1) & 1, status, kSiteK, abort_flag);
+            if (vissued > 0) mbar_wait(bar_vf, (vissued - 1) & 1, status, kSiteV, abort_flag);
             mbar_wait(bar_q, 0, status, kSiteQ, abort_flag);
         }
     } else if (warp == 1) {
@@ -183,34 +175,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idS128 = idesc_bf16(128, 128, false), idS64 = idesc_bf16(128, 64, false);
             constexpr uint32_t idPV = idesc_bf16(128, D, true);
             bool ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, status, kSiteQ, abort_flag));
-            auto issue_s = [&](int c) -> bool {
-                const int st = c % kStages;
-                if (!__all_sync(0xffffffffu, mbar_wait(bar_k + 8 * st, (c / kStages) & 1, status, kSiteK, abort_flag))) return false;
-                tc_fence_after();
-                const uint32_t sK = sbase + L::kK0 + st * L::kStageBytes;
+            for (int c = 0; ok && c < nchunk; ++c) {
                 const bool full = (2 * c + 1) < nseg;
+                if (!__all_sync(0xffffffffu, mbar_wait(bar_kf, c & 1, status, kSiteK, abort_flag))) break;
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::kTileBytes + (kk & 3) * 32;
-                    mma_ss(tS0 + (c & 1) * 128, sdesc(sbase + L::kQ + off, 16, 1024), sdesc(sK + off, 16, 1024),
+                    mma_ss(tS, sdesc(sbase + L::kQ + off, 16, 1024), sdesc(sbase + L::kK + off, 16, 1024),
                            full ? idS128 : idS64, kk > 0);
                 }
-                mma_commit(bar_s + 8 * (c & 1));
-                return true;
-            };
-            if (ok && nchunk > 0) ok = issue_s(0);
-            for (int c = 0; ok && c < nchunk; ++c) {
-                if (c + 1 < nchunk && !issue_s(c + 1)) break;
-                const int st = c % kStages;
-                if (!__all_sync(0xffffffffu, mbar_wait(bar_p + 8 * (c & 1), (c >> 1) & 1, status, kSiteP, abort_flag))) break;
-                if (!__all_sync(0xffffffffu, mbar_wait(bar_v + 8 * st, (c / kStages) & 1, status, kSiteV, abort_flag))) break;
+                mma_commit(bar_s);
+                mma_commit(bar_ke);
+                if (!__all_sync(0xffffffffu, mbar_wait(bar_p, c & 1, status, kSiteP, abort_flag))) break;
+                if (!__all_sync(0xffffffffu, mbar_wait(bar_vf, c & 1, status, kSiteV, abort_flag))) break;
                 tc_fence_after();
-                const uint32_t sV = sbase + L::kK0 + st * L::kStageBytes + L::kHalves * L::kTileBytes;
-                const int nk = ((2 * c + 1) < nseg) ? 128 : 64;
+                const int nk = full ? 128 : 64;
                 for (int kk = 0; kk < nk / 16; ++kk)
-                    mma_ts(tO, tS0 + (c & 1) * 128 + kk * 8, sdesc(sV + kk * 2048, L::kTileBytes, 1024), idPV,
+                    mma_ts(tO, tS + kk * 8, sdesc(sbase + L::kV + kk * 2048, L::kTileBytes, 1024), idPV,
                            (c > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(bar_e + 8 * st);
+                mma_commit(bar_ve);
                 mma_commit(bar_o);
             }
         }
@@ -222,41 +206,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m = -INFINITY, l = 0.f;
         bool ok = true;
         for (int c = 0; c < nchunk; ++c) {
-            const int sb = c & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_s + 8 * sb, (c >> 1) & 1, status, kSiteS, abort_flag));
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_s, c & 1, status, kSiteS, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            const bool full = (2 * c + 1) < nseg;
-            const uint32_t tS = tS0 + sb * 128 + lane_off;
-            uint32_t sr[4][32];
-            tmem_ld32(tS, sr[0]);
-            tmem_ld32(tS + 32, sr[1]);
-            if (full) {
-                tmem_ld32(tS + 64, sr[2]);
-                tmem_ld32(tS + 96, sr[3]);
-            }
-            tmem_wait_ld();
+            const int nq = ((2 * c + 1) < nseg) ? 4 : 2;  // 32-column groups of S in this chunk
+            const uint32_t tSr = tS + lane_off;
+            // pass 1: row max
             float mx = -INFINITY;
+            for (int q = 0; q < nq; ++q) {
+                uint32_t sr[32];
+                tmem_ld32(tSr + q * 32, sr);
+                tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 2; ++q)
-#pragma unroll
-                for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[q][e]));
-            if (full) {
-#pragma unroll
-                for (int q = 2; q < 4; ++q)
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[q][e]));
+                for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[e]));
             }
             const float mx2 = mx * scale_log2;
             const bool need = (c > 0) && (mx2 > m + kRescaleThreshold);
             if (c == 0) m = mx2;
-            // TMEM loads / stores are warp-collective: the whole warp rescales
-            // when any of its rows needs it (a row whose max did not grow gets 1)
+            // TMEM loads / stores are warp-collective: the whole warp rescales when
+            // any of its rows needs it (a row whose max did not grow gets 1).  O
+            // holds every earlier chunk: S_c was issued after P_{c-1} V_{c-1}.
             if (__any_sync(0xffffffffu, need)) {
-                // O must hold every earlier chunk before it is rescaled
-                ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (c - 1) & 1, status, kSiteO, abort_flag));
-                if (!ok) break;
-                tc_fence_after();
                 const float mnew = fmaxf(m, mx2);
                 const float corr = ex2(m - mnew);
 #pragma unroll 1
@@ -268,44 +238,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * corr);
                     tmem_st32(tO + lane_off + q * 32, orr);
                 }
-                tmem_wait_st();
                 l *= corr;
                 m = mnew;
             }
+            // pass 2: P = exp2(S*scale*log2e - m), bf16 pairs written over S.
+            // Group q packs into columns [16q, 16q+16), which pass 2 has already read.
             float sum = 0.f;
-            uint32_t pk[2][32];
-#pragma unroll
-            for (int q = 0; q < 2; ++q)
+            for (int q = 0; q < nq; ++q) {
+                uint32_t sr[32];
+                tmem_ld32(tSr + q * 32, sr);
+                tmem_wait_ld();
+                uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2(fmaf(__uint_as_float(sr[q][2 * e]), scale_log2, -m));
-                    const float p1 = ex2(fmaf(__uint_as_float(sr[q][2 * e + 1]), scale_log2, -m));
+                    const float p0 = ex2(fmaf(__uint_as_float(sr[2 * e]), scale_log2, -m));
+                    const float p1 = ex2(fmaf(__uint_as_float(sr[2 * e + 1]), scale_log2, -m));
                     sum += p0 + p1;
-                    pk[q >> 1][(q & 1) * 16 + e] = pack_bf16x2(p0, p1);
+                    pk[e] = pack_bf16x2(p0, p1);
                 }
-            if (full) {
-#pragma unroll
-                for (int q = 2; q < 4; ++q)
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2(fmaf(__uint_as_float(sr[q][2 * e]), scale_log2, -m));
-                        const float p1 = ex2(fmaf(__uint_as_float(sr[q][2 * e + 1]), scale_log2, -m));
-                        sum += p0 + p1;
-                        pk[q >> 1][(q & 1) * 16 + e] = pack_bf16x2(p0, p1);
-                    }
+                tmem_st16(tSr + q * 16, pk);
             }
             l += sum;
-            tmem_st32(tS, pk[0]);
-            if (full) tmem_st32(tS + 32, pk[1]);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar_p + 8 * sb);
+            mbar_arrive(bar_p);
         }
-        // epilogue: wait for the last two PV products, in phase order
-        if (ok && nchunk > 0) {
-            for (int ph = max(0, nchunk - 2); ph < nchunk && ok; ++ph)
-                ok = __all_sync(0xffffffffu, mbar_wait(bar_o, ph & 1, status, kSiteO, abort_flag));
-        }
+        // epilogue: the last product P V must have landed
+        if (ok && nchunk > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (nchunk - 1) & 1, status, kSiteO, abort_flag));
         if (ok && nchunk > 0) {
             tc_fence_after();
             const float inv = 1.f / l;
