@@ -1,15 +1,14 @@
-// attn_mma.cu -- block-sparse attention forward / backward over the selected
-// key blocks, warp-level bf16 MMA (m16n8k16) with an online softmax.
+// attn_mma.cu -- backward helpers of the block-sparse attention, and the
+// warp-level bf16 MMA (m16n8k16) backward used for head_dim 64.
 //
 // [Prism guide, Method section 3, last sentence]: each query block attends,
 // under one softmax, only to the key blocks of S_i.  Blocks are 64, 128 or 256
 // tokens and start at multiples of 64 in the block-contiguous order, so the
 // kernels work in 64-row tiles with no masking and no ragged tails.
 //
-// Forward : CTA = 4 warps = one 64-query tile; loops over the 64-key chunks of
-//           every selected key block (cp.async double buffer), S = QK^T,
-//           online softmax in registers (exp2 domain), O += P V.
-// Backward: key-stationary.  CTA = one 64-key tile; loops over the query
+// Delta = rowsum(dO * O) and the permuted dO (k_attn_bwd_pre) and the final
+// dQ conversion (k_dq_finalize) serve both backward kernels.
+// Backward (head_dim 64): key-stationary.  CTA = one 64-key tile; loops over the query
 //           tiles of every query block that selected this key block (block
 //           CSC), recomputes P from the forward's log-sum-exp, accumulates
 //           dK, dV in registers and adds dQ into an fp32 buffer.
@@ -110,168 +109,6 @@ struct ChunkWalk {
 }  // namespace mma
 
 using namespace mma;
-
-// ---------------------------------------------------------------------------
-// forward
-// ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(128, 2)
-    k_attn_fwd_mma(Geo g, const __nv_bfloat16 *__restrict__ Qp, const __nv_bfloat16 *__restrict__ Kp,
-                   const __nv_bfloat16 *__restrict__ Vp, const int *__restrict__ blk_off,
-                   const int *__restrict__ tile_blk, const int *__restrict__ row_ptr, const int *__restrict__ col,
-                   const int *__restrict__ perm, __nv_bfloat16 *__restrict__ O, float *__restrict__ lse_user,
-                   float *__restrict__ lse_p, float scale_log2) {
-    extern __shared__ __align__(128) unsigned char smem[];
-    using TL = Tile<D>;
-    const uint32_t sQ = smem_u32(smem);
-    // stage s: K at sQ + (1 + s) * kBytes, V at sQ + (3 + s) * kBytes
-    const uint32_t sK0 = sQ + TL::kBytes, sV0 = sQ + 3 * TL::kBytes;
-    const int tile = blockIdx.x, bh = blockIdx.y, b = bh / g.heads, h = bh % g.heads;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int gr = lane >> 2, t4 = lane & 3, mi = lane >> 3, rr = lane & 7;
-    const int *bo = blk_off + (size_t)b * (g.nbmax + 1);
-    const int i = tile_blk[(size_t)b * g.nbmax + tile];
-    const size_t row = (size_t)bh * g.nbmax + i;
-    const __nv_bfloat16 *Qh = Qp + (size_t)bh * g.N * D;
-    const __nv_bfloat16 *Kh = Kp + (size_t)bh * g.N * D;
-    const __nv_bfloat16 *Vh = Vp + (size_t)bh * g.N * D;
-
-    ChunkWalk cw;
-    cw.init(col, row_ptr[row], row_ptr[row + 1], bo);
-    TL::load(sQ, Qh + (size_t)tile * 64 * D, tid);
-    TL::load(sK0, Kh + (size_t)cw.row() * D, tid);
-    TL::load(sV0, Vh + (size_t)cw.row() * D, tid);
-    cp_commit();
-
-    uint32_t qf[D / 16][4];
-    float o[D / 8][4];
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-    float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
-
-    int stage = 0;
-    bool first = true;
-    while (cw.valid()) {
-        cp_wait<0>();
-        __syncthreads();
-        if (first) {
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-                ldsm4(qf[kk], sQ + TL::off(warp * 16 + (mi & 1) * 8 + rr, kk * 2 + (mi >> 1)));
-            first = false;
-        }
-        ChunkWalk nx = cw;
-        nx.next();
-        if (nx.valid()) {
-            TL::load(sK0 + (stage ^ 1) * TL::kBytes, Kh + (size_t)nx.row() * D, tid);
-            TL::load(sV0 + (stage ^ 1) * TL::kBytes, Vh + (size_t)nx.row() * D, tid);
-        }
-        cp_commit();
-
-        // S = Q K^T for this warp's 16 rows x 64 keys
-        float s[8][4];
-#pragma unroll
-        for (int n = 0; n < 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-#pragma unroll
-            for (int np = 0; np < 4; ++np) {
-                uint32_t bfr[4];
-                ldsm4(bfr, sK0 + stage * TL::kBytes + TL::off(np * 16 + (mi >> 1) * 8 + rr, kk * 2 + (mi & 1)));
-                mma16816(s[2 * np], qf[kk], bfr[0], bfr[1]);
-                mma16816(s[2 * np + 1], qf[kk], bfr[2], bfr[3]);
-            }
-        }
-        // online softmax (rows gr and gr+8)
-#pragma unroll
-        for (int rh = 0; rh < 2; ++rh) {
-            float mx = -INFINITY;
-#pragma unroll
-            for (int n = 0; n < 8; ++n) mx = fmaxf(mx, fmaxf(s[n][2 * rh], s[n][2 * rh + 1]));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float mnew = fmaxf(mrow[rh], mx * scale_log2);
-            const float corr = exp2f(mrow[rh] - mnew);
-            mrow[rh] = mnew;
-            float sum = 0.f;
-#pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                const float p0 = exp2f(s[n][2 * rh] * scale_log2 - mnew);
-                const float p1 = exp2f(s[n][2 * rh + 1] * scale_log2 - mnew);
-                s[n][2 * rh] = p0;
-                s[n][2 * rh + 1] = p1;
-                sum += p0 + p1;
-            }
-            lrow[rh] = lrow[rh] * corr + sum;
-#pragma unroll
-            for (int n = 0; n < D / 8; ++n) {
-                o[n][2 * rh] *= corr;
-                o[n][2 * rh + 1] *= corr;
-            }
-        }
-        // O += P V
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            uint32_t a[4];
-            a[0] = pack_bf16(s[2 * ks][0], s[2 * ks][1]);
-            a[1] = pack_bf16(s[2 * ks][2], s[2 * ks][3]);
-            a[2] = pack_bf16(s[2 * ks + 1][0], s[2 * ks + 1][1]);
-            a[3] = pack_bf16(s[2 * ks + 1][2], s[2 * ks + 1][3]);
-#pragma unroll
-            for (int dp = 0; dp < D / 16; ++dp) {
-                uint32_t bfr[4];
-                ldsm4t(bfr, sV0 + stage * TL::kBytes + TL::off(ks * 16 + (mi & 1) * 8 + rr, dp * 2 + (mi >> 1)));
-                mma16816(o[2 * dp], a, bfr[0], bfr[1]);
-                mma16816(o[2 * dp + 1], a, bfr[2], bfr[3]);
-            }
-        }
-        stage ^= 1;
-        cw = nx;
-    }
-    cp_wait<0>();
-
-    // normalise, stage through shared memory, store rows through perm
-#pragma unroll
-    for (int rh = 0; rh < 2; ++rh) {
-        float l = lrow[rh];
-        l += __shfl_xor_sync(0xffffffffu, l, 1);
-        l += __shfl_xor_sync(0xffffffffu, l, 2);
-        lrow[rh] = l;
-        const float inv = 1.f / l;
-#pragma unroll
-        for (int n = 0; n < D / 8; ++n) {
-            o[n][2 * rh] *= inv;
-            o[n][2 * rh + 1] *= inv;
-        }
-    }
-    __syncthreads();  // every warp is done with sQ's Q tile (fragments are in registers)
-    unsigned char *sOut = smem;
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-        const int r0 = warp * 16 + gr;
-        *reinterpret_cast<uint32_t *>(sOut + TL::off(r0, n) + t4 * 4) = pack_bf16(o[n][0], o[n][1]);
-        *reinterpret_cast<uint32_t *>(sOut + TL::off(r0 + 8, n) + t4 * 4) = pack_bf16(o[n][2], o[n][3]);
-    }
-    if (t4 == 0) {
-#pragma unroll
-        for (int rh = 0; rh < 2; ++rh) {
-            const int n = tile * 64 + warp * 16 + gr + rh * 8;
-            const float lse2 = mrow[rh] + log2f(lrow[rh]);  // log2 units
-            lse_p[(size_t)bh * g.N + n] = lse2;
-            if (lse_user) lse_user[(size_t)bh * g.N + perm[(size_t)b * g.N + n]] = lse2 * 0.69314718055994531f;
-        }
-    }
-    __syncwarp();
-#pragma unroll
-    for (int it = 0; it < 16 * TL::kChunks / 32; ++it) {
-        const int idx = it * 32 + lane;
-        const int r = warp * 16 + idx / TL::kChunks, ch = idx % TL::kChunks;
-        const int n = tile * 64 + r;
-        const int tok = perm[(size_t)b * g.N + n];
-        const uint4 v = *reinterpret_cast<const uint4 *>(sOut + TL::off(r, ch));
-        *reinterpret_cast<uint4 *>(O + (((size_t)b * g.N + tok) * g.heads + h) * D + ch * 8) = v;
-    }
-}
 
 // ---------------------------------------------------------------------------
 // backward, part 1: Delta = rowsum(dO * O) and the permuted copy of dO
@@ -560,24 +397,8 @@ __global__ void __launch_bounds__(256) k_dq_finalize(Geo g, const float *__restr
 // launchers
 // ---------------------------------------------------------------------------
 template <int D>
-static constexpr size_t fwd_smem() {
-    return 5 * Tile<D>::kBytes;
-}
-template <int D>
 static constexpr size_t bwd_smem() {
     return 6 * Tile<D>::kBytes + 64 * 64 * 2 + 4 * 64 * sizeof(float);
-}
-
-template <int D>
-static prism_status fwd_impl(Plan &pl, void *O, float *lse, cudaStream_t st) {
-    const Geo &g = pl.g;
-    const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
-    TimerScope ts(pl, kTAttnFwd, st);
-    k_attn_fwd_mma<D><<<dim3(g.nbmax, g.batch * g.heads), 128, fwd_smem<D>(), st>>>(
-        g, pl.Qp, pl.Kp, pl.Vp, pl.blk_off, pl.tile_blk, pl.row_ptr, pl.col, pl.perm,
-        static_cast<__nv_bfloat16 *>(O), lse, pl.lse_p, scale_log2);
-    PRISM_CUDA_OK(cudaGetLastError());
-    return PRISM_OK;
 }
 
 template <int D>
@@ -592,7 +413,7 @@ static prism_status bwd_impl(Plan &pl, const void *O, const void *dO, void *dQ, 
                                                              static_cast<const __nv_bfloat16 *>(dO), pl.perm,
                                                              pl.dOp, pl.delta);
     }
-    if (D == 128 && !pl.use_legacy_fwd) {
+    if (D == 128) {
         prism_status s = launch_attn_bwd_tc_main(pl, dK, dV, st);
         if (s != PRISM_OK) return s;
     } else {
@@ -610,19 +431,11 @@ static prism_status bwd_impl(Plan &pl, const void *O, const void *dO, void *dQ, 
 }
 
 prism_status configure_attn_kernels() {
-    PRISM_CUDA_OK(cudaFuncSetAttribute(k_attn_fwd_mma<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)fwd_smem<64>()));
-    PRISM_CUDA_OK(cudaFuncSetAttribute(k_attn_fwd_mma<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)fwd_smem<128>()));
     PRISM_CUDA_OK(cudaFuncSetAttribute(k_attn_bwd_mma<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bwd_smem<64>()));
     PRISM_CUDA_OK(cudaFuncSetAttribute(k_attn_bwd_mma<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bwd_smem<128>()));
     return PRISM_OK;
-}
-
-prism_status launch_attn_fwd(Plan &pl, void *O, float *lse, cudaStream_t st) {
-    return pl.g.D == 64 ? fwd_impl<64>(pl, O, lse, st) : fwd_impl<128>(pl, O, lse, st);
 }
 
 prism_status launch_attn_bwd(Plan &pl, const void *O, const void *dO, void *dQ, void *dK, void *dV,

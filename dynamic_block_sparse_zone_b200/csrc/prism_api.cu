@@ -268,10 +268,7 @@ prism_status prism_plan_create(const prism_params *params, prism_plan **out) {
     if (s == PRISM_OK) s = configure_attn_tc_kernels();
     if (s == PRISM_OK) s = configure_attn_bwd_tc_kernels();
     if (s == PRISM_OK) s = make_tensor_maps(pl);
-    {
-        const char *env = getenv("PRISM_LEGACY_FWD");
-        pl.use_legacy_fwd = (env && env[0] == '1') ? 1 : 0;
-    }
+
     if (s != PRISM_OK) {
         release_buffers(pl);
         delete h;
@@ -313,8 +310,7 @@ prism_status prism_attn_fwd(prism_plan *plan, void *O, float *lse, void *stream)
     prism_status s = device_guard(plan->pl);
     if (s != PRISM_OK) return s;
     if ((uintptr_t)O & 15) return fail(PRISM_ERR_INVALID_ARG, "O must be 16-byte aligned");
-    s = plan->pl.use_legacy_fwd ? launch_attn_fwd(plan->pl, O, lse, static_cast<cudaStream_t>(stream))
-                                : launch_attn_fwd_tc(plan->pl, O, lse, static_cast<cudaStream_t>(stream));
+    s = launch_attn_fwd_tc(plan->pl, O, lse, static_cast<cudaStream_t>(stream));
     if (s == PRISM_OK) plan->pl.have_fwd = true;
     return s;
 }

@@ -74,7 +74,6 @@ struct Plan {
     int *status;            // device error word (0 = ok)
     int *host_nb;           // pinned host copy of nb
     TimerState *timers;     // NULL unless timing is on
-    int use_legacy_fwd;     // development switch: warp-MMA forward instead of tcgen05
     // TMA descriptors of the permuted copies, viewed as [batch*heads*N][D] bf16
     CUtensorMap tmQ, tmK, tmV, tmdO;
     CUtensorMap tmdQ;       // fp32 [batch*heads*N][D], 64-row boxes, reduce-add target
@@ -101,7 +100,6 @@ prism_status fail_cuda(cudaError_t e, const char *what, const char *file, int li
 // Launchers (each returns PRISM_OK or an error after checking the launch).
 prism_status launch_plan(Plan &pl, const void *Q, const void *K, const void *V, const float *a,
                          cudaStream_t st);
-prism_status launch_attn_fwd(Plan &pl, void *O, float *lse, cudaStream_t st);
 prism_status launch_attn_fwd_tc(Plan &pl, void *O, float *lse, cudaStream_t st);
 prism_status make_tensor_maps(Plan &pl);
 prism_status launch_attn_bwd_tc_main(Plan &pl, void *dK, void *dV, cudaStream_t st);
