@@ -23,7 +23,8 @@ _STATUS = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_UNSUPPORTED"
 
 EXPORTED = ("prism_plan_create", "prism_plan_bytes", "prism_plan_build", "prism_attn_fwd", "prism_attn_bwd",
             "prism_plan_view_get", "prism_plan_check", "prism_plan_destroy", "prism_last_error",
-            "prism_plan_set_timing", "prism_plan_read_timing", "prism_timer_name", "prism_zone_shapes_noalloc")
+            "prism_plan_set_timing", "prism_plan_read_timing", "prism_timer_name", "prism_zone_shapes_noalloc",
+            "prism_plan_selftest_timeout")
 NUM_TIMERS = 10
 
 
@@ -66,6 +67,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.prism_attn_bwd.argtypes = [V, P, P, P, P, P, P]
     lib.prism_plan_view_get.argtypes = [V, ctypes.POINTER(prism_plan_view), P]
     lib.prism_plan_check.argtypes = [V, P]
+    lib.prism_plan_selftest_timeout.argtypes = [V, P]
+    lib.prism_plan_selftest_timeout.restype = ctypes.c_int
     lib.prism_plan_destroy.argtypes = [V]
     lib.prism_plan_destroy.restype = None
     lib.prism_last_error.restype = ctypes.c_char_p
@@ -217,6 +220,10 @@ class PrismPlan:
     # -- inspection ----------------------------------------------------------
     def check(self):
         _check(load_library().prism_plan_check(self._h, _stream()))
+
+    def selftest_timeout(self):
+        """Enqueues the bounded-wait diagnostic (the next check() raises PRISM_ERR_TIMEOUT)."""
+        _check(load_library().prism_plan_selftest_timeout(self._h, _stream()))
 
     def view(self) -> dict:
         """Copies of the plan's arrays (syncs the current stream)."""

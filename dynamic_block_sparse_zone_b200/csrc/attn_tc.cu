@@ -305,6 +305,26 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 }  // namespace fwdtc
 
+// Exercises the bounded-wait failure path: one thread waits on an mbarrier
+// that nothing arrives on, with the same helper the attention kernels use,
+// and records the timeout in the plan's status word.
+__global__ void k_selftest_bounded_wait(int *status) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(smem_u32(&bar), 1);
+        mbar_fence_init();
+        mbar_wait(smem_u32(&bar), 0, status, 99, &abort_flag);
+    }
+}
+
+prism_status launch_selftest_bounded_wait(Plan &pl, cudaStream_t st) {
+    k_selftest_bounded_wait<<<1, 32, 0, st>>>(pl.status);
+    PRISM_CUDA_OK(cudaGetLastError());
+    return PRISM_OK;
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------

@@ -37,6 +37,7 @@ prism_status configure_plan_kernels(const Plan &pl);
 prism_status configure_attn_kernels();
 prism_status configure_attn_tc_kernels();
 prism_status configure_attn_bwd_tc_kernels();
+prism_status launch_selftest_bounded_wait(Plan &pl, cudaStream_t st);
 size_t select_smem_bytes(const Plan &pl);
 
 static int log2_exact(int x) {
@@ -392,6 +393,14 @@ prism_status prism_plan_read_timing(prism_plan *plan, float *total_ms, int *laun
         ts->rec[k].clear();
     }
     return PRISM_OK;
+}
+
+prism_status prism_plan_selftest_timeout(prism_plan *plan, void *stream) {
+    g_last_error.clear();
+    if (!plan) return fail(PRISM_ERR_INVALID_ARG, "plan is NULL");
+    prism_status s = device_guard(plan->pl);
+    if (s != PRISM_OK) return s;
+    return launch_selftest_bounded_wait(plan->pl, static_cast<cudaStream_t>(stream));
 }
 
 prism_status prism_plan_check(prism_plan *plan, void *stream) {

@@ -16,7 +16,7 @@
 namespace prism {
 namespace tc {
 
-constexpr long long kSpinLimit = 1ll << 23;
+constexpr long long kSpinLimit = 1ll << 18;  // ~1 s: each unsatisfied try_wait suspends a few microseconds
 constexpr int kErrTimeout = 1;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

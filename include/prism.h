@@ -143,6 +143,14 @@ PRISM_API prism_status prism_plan_view_get(prism_plan *plan, prism_plan_view *vi
  * then clears it.                                                          */
 PRISM_API prism_status prism_plan_check(prism_plan *plan, void *stream);
 
+/* Diagnostic of the failure path: enqueues one thread that waits on a
+ * device barrier nothing arrives on, through the same bounded wait the
+ * attention kernels use.  It gives up after its poll limit (about a second)
+ * and records a timeout in the plan's status word,
+ * so the next prism_plan_check returns PRISM_ERR_TIMEOUT; while the word is
+ * set, the plan's attention kernels return at once.  No fault, no hang.   */
+PRISM_API prism_status prism_plan_selftest_timeout(prism_plan *plan, void *stream);
+
 /* Optional per-kernel timing with CUDA events recorded on the launch stream
  * around every kernel of the plan (off by default; adds two event records
  * per launch).  prism_plan_read_timing waits for the recorded events, writes

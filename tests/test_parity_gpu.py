@@ -331,3 +331,27 @@ def test_latent2k_train_full_size_sampled():
     assert_close("dV", g["dV"][0].float().cpu().numpy()[req_t, heads[0]], dV_ref)
     check_gradient_sums(g, inp)
     print("2K near-ties", ties, "blocks", pl.nb)
+
+
+def test_bounded_wait_reports_timeout_and_context_stays_usable():
+    """A device wait that nothing satisfies gives up, the host reads
+    PRISM_ERR_TIMEOUT, the status clears, and the plan keeps working."""
+    import time
+    from dynamic_block_sparse_zone_b200.binding import PrismError
+    w = WORKLOADS["tiny_8x16x16"]
+    inp = make_inputs(w, 0)
+    g = run_gpu(w, inp)
+    plan = g["plan"]
+    t0 = time.time()
+    plan.selftest_timeout()
+    with pytest.raises(PrismError) as ei:
+        plan.check()
+    assert ei.value.status == 4 and "wait gave up" in str(ei.value)
+    assert time.time() - t0 < 60
+    plan.check()  # cleared
+    Q, K, V, a = (x.cuda() for x in (inp.Q, inp.K, inp.V, inp.a))
+    plan.build(Q, K, V, a)
+    O, _ = plan.fwd()
+    torch.cuda.synchronize()
+    plan.check()
+    assert torch.equal(O, g["O"])
