@@ -127,6 +127,25 @@ def kernel_bytes(name, w, nb, pairs_unused):
     return None
 
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Largest value of x over all ranks (timings are taken as the slowest
+    rank's).  The only collective of the benchmark: replicas never exchange
+    data."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(flops_per_step: float, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job TFLOP/s: every rank runs `steps` steps of the same workload
+    (weak scaling), timed by the slowest rank."""
+    return flops_per_step * steps * world / (ms_max * 1e-3) / 1e12
+
+
 def workload_of(args):
     from dynamic_block_sparse_zone_b200.synth import WORKLOADS, scaled
     w = WORKLOADS[args.workload]
@@ -168,12 +187,6 @@ def run_ours(args, rank, world, dev):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # ---- device-resident timed region ----
     plan.set_timing(True)
@@ -191,7 +204,7 @@ def run_ours(args, rank, world, dev):
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    ms = max_over_ranks(e0.elapsed_time(e1))
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     timing = plan.read_timing()
     plan.set_timing(False)
     plan.check()
@@ -222,8 +235,8 @@ def run_ours(args, rank, world, dev):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ms_e2e = max_over_ranks(e0.elapsed_time(e1))
-        e2e = {"value": round(flops_step * args.steps * world / (ms_e2e * 1e-3) / 1e12, 3),
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": round(aggregate_value(flops_step, args.steps, world, ms_e2e), 3),
                "unit": "TFLOP/s", "ms_per_step": round(ms_e2e / args.steps, 3),
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
         del host_in, host_out, dev_in
@@ -260,7 +273,7 @@ def run_ours(args, rank, world, dev):
     launches_per_step = sum(n * (9 if k == "csr_csc" else 1) for k, (t, n) in timing.items()) // max(args.steps, 1)
     result = {
         "metric": METRIC,
-        "value": round(flops_step * args.steps * world / (ms * 1e-3) / 1e12, 3),
+        "value": round(aggregate_value(flops_step, args.steps, world, ms), 3),
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": args.steps,

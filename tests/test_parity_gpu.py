@@ -355,3 +355,48 @@ def test_bounded_wait_reports_timeout_and_context_stays_usable():
     torch.cuda.synchronize()
     plan.check()
     assert torch.equal(O, g["O"])
+
+
+EDGE_CASES = {
+    # fixed non-cubic shapes (volume 64 and 256) exercise the fixed-shape path
+    "fixed_2x4x8": scaled(WORKLOADS["tiny_8x16x16"], fixed_shape=(2, 4, 8)),
+    "fixed_8x8x4": scaled(WORKLOADS["tiny_8x16x16"], T=16, fixed_shape=(8, 8, 4), top_k=1),
+    # one zone, one head: the smallest problem (8 to 2 blocks)
+    "single_zone": scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=8, W=8, heads=1, planted=0, top_k=1, top_p=0.5),
+    # cap equal to k (max_frac so small that floor(frac * N_b) < k)
+    "cap_is_k": scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=2, planted=2, top_k=3, top_p=0.99,
+                       max_frac=0.01),
+    # cap binding at head_dim 64
+    "cap_d64": scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=2, head_dim=64, planted=2, top_k=2,
+                      top_p=0.95, max_frac=0.1),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EDGE_CASES))
+def test_edge_case_plans_and_forward(name):
+    w = EDGE_CASES[name]
+    inp = make_inputs(w, 8)
+    g = run_gpu(w, inp)
+    pl, bits = oracle_plan(w, inp)
+    compare_plan(w, pl, g["view"])
+    if w.max_frac > 0:
+        cap = oracle.cap(pl.nb, w.top_k, _f32(w.max_frac))
+        assert pl.cnt.max() <= cap
+    check_forward(w, inp, g, pl, bits, min(512, w.N * w.heads))
+
+
+def test_capped_backward():
+    w = scaled(EDGE_CASES["cap_is_k"], backward=True)
+    inp = make_inputs(w, 9)
+    g = run_gpu(w, inp, backward=True)
+    pl, bits = oracle_plan(w, inp)
+    compare_plan(w, pl, g["view"])
+    dOb = bf16_bits(inp.dO[0])
+    rs = np.random.default_rng(3)
+    req_h, req_t = sample_rows(rs, w, 256)
+    assert_close("dQ", g["dQ"][0].float().cpu().numpy()[req_t, req_h],
+                 oracle.attn_bwd_dq_rows(pl, *bits, dOb, req_h, req_t))
+    req_h, req_t = sample_rows(rs, w, 128)
+    dK_ref, dV_ref = oracle.attn_bwd_dkv_rows(pl, *bits, dOb, req_h, req_t)
+    assert_close("dK", g["dK"][0].float().cpu().numpy()[req_t, req_h], dK_ref)
+    assert_close("dV", g["dV"][0].float().cpu().numpy()[req_t, req_h], dV_ref)
