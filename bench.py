@@ -118,8 +118,6 @@ def kernel_bytes(name, w, nb, pairs_unused):
         return N * C * 2
     if name == "permute_pool":
         return 6 * N * C * 2 + 2 * h * nb * D * 8 + N * 4
-    if name == "select":
-        return 2 * h * nb * D * 8
     if name == "attn_bwd_pre":
         return 2 * N * C * 2 + N * C * 2 + h * N * 4
     if name == "dq_finalize":
@@ -144,6 +142,10 @@ def aggregate_value(flops_per_step: float, steps: int, world: int, ms_max: float
     """Whole-job TFLOP/s: every rank runs `steps` steps of the same workload
     (weak scaling), timed by the slowest rank."""
     return flops_per_step * steps * world / (ms_max * 1e-3) / 1e12
+
+
+def steps_or_1(args):
+    return max(args.steps, 1)
 
 
 def workload_of(args):
@@ -249,6 +251,9 @@ def run_ours(args, rank, world, dev):
             continue
         avg = tms / n
         rec = {"launches": n, "avg_ms": round(avg, 4), "share": round(tms / total_k, 4)}
+        if name == "select":
+            rec["fp64_tflops"] = round(2.0 * w.head_dim * nb * nb * w.heads * w.batch * steps_or_1(args) /
+                                       (tms * 1e-3) / 1e12, 3)
         if name == "attn_fwd":
             rec["tflops"] = round(flops_fwd / (avg * 1e-3) / 1e12, 2)
         elif name == "attn_bwd":
@@ -270,6 +275,7 @@ def run_ours(args, rank, world, dev):
         ach = kernels[dom].get("gbs", 0.0)
         roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
                 "frac": round(ach / peak, 4), "peak_kind": f"HBM copy ({peak_src})", "traffic": traffic_for(dom)}
+    # one timer record per kernel launch, except the CSR/CSC scope (9 kernels)
     launches_per_step = sum(n * (9 if k == "csr_csc" else 1) for k, (t, n) in timing.items()) // max(args.steps, 1)
     result = {
         "metric": METRIC,

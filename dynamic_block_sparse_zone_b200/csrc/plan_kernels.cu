@@ -564,11 +564,9 @@ __device__ __forceinline__ int block_scan_256(int v, int *buf, int *tot) {
     return before + x - v;
 }
 
-constexpr int kSelSlice = 16;  // pooled-key channels staged per pass (128 B of a row)
-
 struct SelSmem {
     // layout inside the dynamic buffer (offsets in bytes)
-    size_t qbar, keys, sk, sj, pr, bits, tile;
+    size_t keys, sk, sj, pr, bits;
     size_t bytes;
 };
 
@@ -582,30 +580,84 @@ __host__ __device__ inline SelSmem sel_smem_layout(int D, int nbmax, int cap_str
     SelSmem L;
     const int SP = pow2_at_least(cap_stride);
     size_t o = 0;
-    L.qbar = o; o += (size_t)D * 8;
     L.keys = o; o += (size_t)nbmax * 8;
     L.sk = o;   o += (size_t)SP * 8;
     L.pr = o;   o += (size_t)SP * 8;
     L.sj = o;   o += (size_t)SP * 4;
     L.bits = o; o += (size_t)((nbmax + 31) / 32) * 4;
-    o = (o + 15) & ~(size_t)15;
-    L.tile = o; o += (size_t)kSelThreads * (kSelSlice + 1) * 8;  // [256 rows][16 channels + 1 pad] fp64
     L.bytes = (o + 15) & ~(size_t)15;
     return L;
 }
 
+// Pooled block scores of a group of heads: z_ij = Qbar_i . Kbar_j / sqrt(D),
+// stored as order-preserving u64 keys in keys[head of group][i][j].  A CTA
+// computes a 64 x 64 block; each thread keeps 16 scores in flight, each one
+// summed over the channels in ascending order with explicitly rounded fp64
+// operations (the oracle's order).
+constexpr int kScoreTile = 64;
+constexpr int kScoreSlice = 32;
+
+__global__ void __launch_bounds__(256) k_scores(Geo g, const int *__restrict__ nb_arr,
+                                                const double *__restrict__ Qbar, const double *__restrict__ Kbar,
+                                                int bh0, unsigned long long *__restrict__ keys) {
+    __shared__ double sq[kScoreTile][kScoreSlice + 1], sk[kScoreTile][kScoreSlice + 1];
+    const int jt = blockIdx.x, it = blockIdx.y, bh = bh0 + blockIdx.z;
+    if (bh >= g.batch * g.heads) return;
+    const int nb = nb_arr[bh / g.heads];
+    const int i0 = it * kScoreTile, j0 = jt * kScoreTile;
+    if (i0 >= nb || j0 >= nb) return;
+    const int tid = threadIdx.x, ti = tid >> 4, tj = tid & 15;
+    const double *qb = Qbar + (size_t)bh * g.nbmax * g.D;
+    const double *kb = Kbar + (size_t)bh * g.nbmax * g.D;
+    double acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[a][c] = 0.0;
+    for (int c0 = 0; c0 < g.D; c0 += kScoreSlice) {
+        for (int idx = tid; idx < kScoreTile * kScoreSlice; idx += 256) {
+            const int r = idx / kScoreSlice, c = idx % kScoreSlice;
+            sq[r][c] = (i0 + r < nb) ? qb[(size_t)(i0 + r) * g.D + c0 + c] : 0.0;
+            sk[r][c] = (j0 + r < nb) ? kb[(size_t)(j0 + r) * g.D + c0 + c] : 0.0;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int c = 0; c < kScoreSlice; ++c) {
+            double qa[4], kc[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) qa[a] = sq[ti + 16 * a][c];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) kc[e] = sk[tj + 16 * e][c];
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[a][e] = __dadd_rn(acc[a][e], __dmul_rn(qa[a], kc[e]));
+        }
+        __syncthreads();
+    }
+    const double sqrtD = __dsqrt_rn((double)g.D);
+    unsigned long long *out = keys + (size_t)blockIdx.z * g.nbmax * g.nbmax;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int i = i0 + ti + 16 * a, j = j0 + tj + 16 * e;
+            if (i < nb && j < nb) out[(size_t)i * g.nbmax + j] = order_key(__ddiv_rn(acc[a][e], sqrtD));
+        }
+}
+
 __global__ void __launch_bounds__(kSelThreads) k_select(Geo g, const int *__restrict__ nb_arr,
-                                                        const double *__restrict__ Qbar,
-                                                        const double *__restrict__ Kbar, int top_k, double top_p,
-                                                        float max_frac, int cap_stride, int *__restrict__ cnt,
-                                                        int *__restrict__ cols_pad) {
+                                                        const unsigned long long *__restrict__ keys_in, int bh0,
+                                                        int top_k, double top_p, float max_frac, int cap_stride,
+                                                        int *__restrict__ cnt, int *__restrict__ cols_pad) {
     extern __shared__ __align__(16) unsigned char sel_raw[];
     __shared__ int hist[256];
     __shared__ int ibuf[64];
     __shared__ double dred[32];
     __shared__ unsigned long long ured[32];
     __shared__ int s_digit, s_rem, s_done, s_fill, s_np;
-    const int i = blockIdx.x, bh = blockIdx.y, b = bh / g.heads;
+    const int i = blockIdx.x, bh = bh0 + blockIdx.y, b = bh / g.heads;
+    if (bh >= g.batch * g.heads) return;
     const int tid = threadIdx.x;
     const size_t row = (size_t)bh * g.nbmax + i;
     const int nb = nb_arr[b];
@@ -614,46 +666,19 @@ __global__ void __launch_bounds__(kSelThreads) k_select(Geo g, const int *__rest
         return;
     }
     const SelSmem L = sel_smem_layout(g.D, g.nbmax, cap_stride);
-    double *qbar = reinterpret_cast<double *>(sel_raw + L.qbar);
     uint64_t *keys = reinterpret_cast<uint64_t *>(sel_raw + L.keys);
     uint64_t *sk = reinterpret_cast<uint64_t *>(sel_raw + L.sk);
     double *pr = reinterpret_cast<double *>(sel_raw + L.pr);
     int *sj = reinterpret_cast<int *>(sel_raw + L.sj);
     uint32_t *bits = reinterpret_cast<uint32_t *>(sel_raw + L.bits);
 
-    for (int c = tid; c < g.D; c += kSelThreads) qbar[c] = Qbar[row * g.D + c];
-    __syncthreads();
-    // scores
-    const double sqrtD = __dsqrt_rn((double)g.D);
-    const double *kb = Kbar + (size_t)bh * g.nbmax * g.D;
-    double *tile = reinterpret_cast<double *>(sel_raw + L.tile);
+    // scores of this row (written by k_scores)
+    const unsigned long long *krow = keys_in + ((size_t)blockIdx.y * g.nbmax + i) * g.nbmax;
     unsigned long long kmax = 0;
-    // Thread t scores block j0 + t.  Pooled-key rows are staged through shared
-    // memory 16 channels at a time with coalesced loads; each thread still sums
-    // its dot product over the channels in ascending order.
-    for (int j0 = 0; j0 < nb; j0 += kSelThreads) {
-        const int j = j0 + tid;
-        double dot = 0.0;
-        for (int c0 = 0; c0 < g.D; c0 += kSelSlice) {
-            for (int idx = tid; idx < kSelThreads * (kSelSlice / 2); idx += kSelThreads) {
-                const int rr = idx / (kSelSlice / 2), part = idx % (kSelSlice / 2);
-                double2 v = make_double2(0.0, 0.0);
-                if (j0 + rr < nb)
-                    v = *reinterpret_cast<const double2 *>(kb + (size_t)(j0 + rr) * g.D + c0 + 2 * part);
-                tile[rr * (kSelSlice + 1) + 2 * part] = v.x;
-                tile[rr * (kSelSlice + 1) + 2 * part + 1] = v.y;
-            }
-            __syncthreads();
-            const double *tr = tile + tid * (kSelSlice + 1);
-#pragma unroll
-            for (int c = 0; c < kSelSlice; ++c) dot = __dadd_rn(dot, __dmul_rn(qbar[c0 + c], tr[c]));
-            __syncthreads();
-        }
-        if (j < nb) {
-            const uint64_t key = order_key(__ddiv_rn(dot, sqrtD));
-            keys[j] = key;
-            kmax = key > kmax ? key : kmax;
-        }
+    for (int j = tid; j < nb; j += kSelThreads) {
+        const unsigned long long key = krow[j];
+        keys[j] = key;
+        kmax = key > kmax ? key : kmax;
     }
     kmax = block_max_u64(kmax, ured);
     const double zmax = key_value(kmax);
@@ -953,10 +978,25 @@ prism_status launch_plan(Plan &pl, const void *Qv, const void *Kv, const void *V
                                                                    pl.perm, pl.Qp, pl.Kp, pl.Vp, pl.Qbar, pl.Kbar); }
     PRISM_CUDA_OK(cudaGetLastError());
     const size_t rows = (size_t)g.batch * g.heads * g.nbmax;
-    { TimerScope ts(pl, kTSelect, st);
-    k_select<<<dim3(g.nbmax, g.batch * g.heads), kSelThreads, select_smem_bytes(pl), st>>>(
-        g, pl.nb, pl.Qbar, pl.Kbar, pl.p.top_k, (double)pl.p.top_p, pl.p.max_frac, pl.cap_stride, pl.cnt,
-        pl.cols_pad); }
+    {
+        // scores and selection, a group of heads at a time (the score scratch
+        // holds score_group heads of N_b x N_b keys); one timer record per launch
+        const int BH = g.batch * g.heads;
+        const int nt = (g.nbmax + kScoreTile - 1) / kScoreTile;
+        for (int bh0 = 0; bh0 < BH; bh0 += pl.score_group) {
+            const int G = BH - bh0 < pl.score_group ? BH - bh0 : pl.score_group;
+            {
+                TimerScope ts(pl, kTSelect, st);
+                k_scores<<<dim3(nt, nt, G), 256, 0, st>>>(g, pl.nb, pl.Qbar, pl.Kbar, bh0, pl.score_keys);
+            }
+            {
+                TimerScope ts(pl, kTSelect, st);
+                k_select<<<dim3(g.nbmax, G), kSelThreads, select_smem_bytes(pl), st>>>(
+                    g, pl.nb, pl.score_keys, bh0, pl.p.top_k, (double)pl.p.top_p, pl.p.max_frac, pl.cap_stride,
+                    pl.cnt, pl.cols_pad);
+            }
+        }
+    }
     PRISM_CUDA_OK(cudaGetLastError());
     TimerScope ts_csr(pl, kTCsr, st);
     prism_status s = scan_into(pl.cnt, rows, pl.row_ptr, pl.scan_tmp, st);

@@ -93,7 +93,19 @@ static prism_status check_params(const prism_params *p, Geo *g, int *fixed_idx, 
         return fail(PRISM_ERR_UNSUPPORTED, "selection too large for 32-bit CSR offsets (%lld x %d)", rows, *cap_stride);
     if ((long long)g->batch * g->heads * g->N * g->D >= (1ll << 40))
         return fail(PRISM_ERR_UNSUPPORTED, "tensors too large");
+    const double head_scores = (double)g->nbmax * g->nbmax * 8.0;  // bytes of one head's block scores
+    if (head_scores > 2.0 * (1ull << 30))
+        return fail(PRISM_ERR_UNSUPPORTED, "too many blocks for the score scratch (%d blocks per sample)", g->nbmax);
     return PRISM_OK;
+}
+
+// Heads whose block scores are held at once: as many as fit in 1 GiB.
+static int score_group_for(const Geo &g) {
+    const double head_scores = (double)g.nbmax * g.nbmax * 8.0;
+    int G = (int)((double)(1ull << 30) / head_scores);
+    if (G < 1) G = 1;
+    if (G > g.batch * g.heads) G = g.batch * g.heads;
+    return G;
 }
 
 struct Alloc {
@@ -126,6 +138,7 @@ static size_t plan_allocs(Plan &pl, Alloc *out) {
     add((void **)&pl.Vp, BH * g.N * g.D * 2);
     add((void **)&pl.Qbar, rows * g.D * sizeof(double));
     add((void **)&pl.Kbar, rows * g.D * sizeof(double));
+    add((void **)&pl.score_keys, (size_t)pl.score_group * g.nbmax * g.nbmax * sizeof(unsigned long long));
     add((void **)&pl.cnt, rows * sizeof(int));
     add((void **)&pl.cols_pad, nnz * sizeof(int));
     add((void **)&pl.row_ptr, (rows + 1) * sizeof(int));
@@ -213,6 +226,7 @@ size_t prism_plan_bytes(const prism_params *params) {
     Plan pl;
     memset(&pl, 0, sizeof pl);
     if (check_params(params, &pl.g, &pl.fixed_idx, &pl.cap_stride) != PRISM_OK) return 0;
+    pl.score_group = score_group_for(pl.g);
     Alloc a[64];
     const size_t n = plan_allocs(pl, a);
     size_t tot = 0;
@@ -235,6 +249,7 @@ prism_status prism_plan_create(const prism_params *params, prism_plan **out) {
     }
     pl.p = *params;
     if (!(pl.p.eps > 0.0)) pl.p.eps = 1e-6;
+    pl.score_group = score_group_for(pl.g);
     if (select_smem_bytes(pl) > 220 * 1024) {
         delete h;
         return fail(PRISM_ERR_UNSUPPORTED, "selection working set (%zu bytes of shared memory) too large",

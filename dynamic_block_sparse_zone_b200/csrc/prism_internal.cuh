@@ -58,6 +58,8 @@ struct Plan {
     __nv_bfloat16 *Qp, *Kp, *Vp;   // [batch*heads][N][D]
     double *Qbar, *Kbar;           // [batch*heads][nbmax][D]
     // selection
+    unsigned long long *score_keys;  // [score_group][nbmax][nbmax] order-preserving score keys
+    int score_group;        // heads scored per pass
     int *cnt;               // [batch*heads*nbmax]
     int *cols_pad;          // [batch*heads*nbmax][cap_stride]
     int *row_ptr;           // [rows+1]
