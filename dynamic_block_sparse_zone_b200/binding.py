@@ -24,7 +24,7 @@ _STATUS = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_UNSUPPORTED"
 EXPORTED = ("prism_plan_create", "prism_plan_bytes", "prism_plan_build", "prism_attn_fwd", "prism_attn_bwd",
             "prism_plan_view_get", "prism_plan_check", "prism_plan_destroy", "prism_last_error",
             "prism_plan_set_timing", "prism_plan_read_timing", "prism_timer_name", "prism_zone_shapes_noalloc",
-            "prism_plan_selftest_timeout")
+            "prism_plan_selftest_timeout", "prism_plan_update_qkv")
 NUM_TIMERS = 10
 
 
@@ -64,6 +64,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.prism_plan_bytes.restype = ctypes.c_size_t
     lib.prism_plan_build.argtypes = [V, P, P, P, P, P]
     lib.prism_attn_fwd.argtypes = [V, P, P, P]
+    lib.prism_plan_update_qkv.argtypes = [V, P, P, P, P]
+    lib.prism_plan_update_qkv.restype = ctypes.c_int
     lib.prism_attn_bwd.argtypes = [V, P, P, P, P, P, P]
     lib.prism_plan_view_get.argtypes = [V, ctypes.POINTER(prism_plan_view), P]
     lib.prism_plan_check.argtypes = [V, P]
@@ -179,6 +181,13 @@ class PrismPlan:
             _need(t, n, torch.bfloat16, self._qkv_shape())
         _need(a_norm, "a_norm", torch.float32, (p.batch, p.T, p.H, p.W))
         _check(load_library().prism_plan_build(self._h, _ptr(Q), _ptr(K), _ptr(V), _ptr(a_norm), _stream()))
+        return self
+
+    def update_qkv(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor):
+        """Reuse the plan (zones, shapes, permutation, selection) for new Q, K, V."""
+        for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+            _need(t, n, torch.bfloat16, self._qkv_shape())
+        _check(load_library().prism_plan_update_qkv(self._h, _ptr(Q), _ptr(K), _ptr(V), _stream()))
         return self
 
     def fwd(self, O: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, want_lse: bool = True):

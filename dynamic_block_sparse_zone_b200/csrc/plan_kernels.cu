@@ -1025,6 +1025,21 @@ prism_status configure_plan_kernels(const Plan &pl) {
     return upload_shape_table();
 }
 
+// Re-gathers new Q, K, V into the plan's block-contiguous copies with the
+// plan's existing block table (the selection is kept; the pooled means are
+// refreshed by the same kernel but not used again).
+prism_status launch_regather(Plan &pl, const void *Qv, const void *Kv, const void *Vv, cudaStream_t st) {
+    const Geo &g = pl.g;
+    const int pp_threads = g.C / 8 >= 384 ? 384 : ((g.C / 8 + 31) / 32) * 32;
+    TimerScope ts(pl, kTPermutePool, st);
+    k_permute_pool<<<dim3(g.nbmax, g.batch), pp_threads, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(Qv), static_cast<const __nv_bfloat16 *>(Kv),
+        static_cast<const __nv_bfloat16 *>(Vv), g, pl.nb, pl.blk_off, pl.zone_shape, pl.perm, pl.Qp, pl.Kp, pl.Vp,
+        pl.Qbar, pl.Kbar);
+    PRISM_CUDA_OK(cudaGetLastError());
+    return PRISM_OK;
+}
+
 // Zone statistics and volume / shape decisions alone, on caller-provided
 // buffers (used by the allocation-free entry point).  Scratch arrays are laid
 // out by the caller; the kernels are the planner's own.

@@ -317,7 +317,21 @@ prism_status prism_plan_build(prism_plan *plan, const void *Q, const void *K, co
     const uintptr_t al = (uintptr_t)Q | (uintptr_t)K | (uintptr_t)V;
     if (al & 15) return fail(PRISM_ERR_INVALID_ARG, "Q, K, V must be 16-byte aligned");
     plan->pl.have_fwd = false;
-    return launch_plan(plan->pl, Q, K, V, a_norm, static_cast<cudaStream_t>(stream));
+    s = launch_plan(plan->pl, Q, K, V, a_norm, static_cast<cudaStream_t>(stream));
+    if (s == PRISM_OK) plan->pl.built = true;
+    return s;
+}
+
+prism_status prism_plan_update_qkv(prism_plan *plan, const void *Q, const void *K, const void *V, void *stream) {
+    g_last_error.clear();
+    if (!plan || !Q || !K || !V) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_plan_update_qkv");
+    prism_status s = device_guard(plan->pl);
+    if (s != PRISM_OK) return s;
+    if (!plan->pl.built) return fail(PRISM_ERR_STATE, "prism_plan_update_qkv needs a built plan");
+    const uintptr_t al = (uintptr_t)Q | (uintptr_t)K | (uintptr_t)V;
+    if (al & 15) return fail(PRISM_ERR_INVALID_ARG, "Q, K, V must be 16-byte aligned");
+    plan->pl.have_fwd = false;
+    return launch_regather(plan->pl, Q, K, V, static_cast<cudaStream_t>(stream));
 }
 
 prism_status prism_attn_fwd(prism_plan *plan, void *O, float *lse, void *stream) {
@@ -325,6 +339,7 @@ prism_status prism_attn_fwd(prism_plan *plan, void *O, float *lse, void *stream)
     if (!plan || !O) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_attn_fwd");
     prism_status s = device_guard(plan->pl);
     if (s != PRISM_OK) return s;
+    if (!plan->pl.built) return fail(PRISM_ERR_STATE, "prism_attn_fwd needs a built plan");
     if ((uintptr_t)O & 15) return fail(PRISM_ERR_INVALID_ARG, "O must be 16-byte aligned");
     s = launch_attn_fwd_tc(plan->pl, O, lse, static_cast<cudaStream_t>(stream));
     if (s == PRISM_OK) plan->pl.have_fwd = true;
@@ -337,7 +352,8 @@ prism_status prism_attn_bwd(prism_plan *plan, const void *O, const void *dO, voi
     if (!plan || !O || !dO || !dQ || !dK || !dV) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_attn_bwd");
     prism_status s = device_guard(plan->pl);
     if (s != PRISM_OK) return s;
-    if (!plan->pl.have_fwd) return fail(PRISM_ERR_STATE, "prism_attn_bwd needs a prism_attn_fwd after the build");
+    if (!plan->pl.have_fwd)
+        return fail(PRISM_ERR_STATE, "prism_attn_bwd needs a prism_attn_fwd after the last build or update");
     const uintptr_t al = (uintptr_t)O | (uintptr_t)dO | (uintptr_t)dQ | (uintptr_t)dK | (uintptr_t)dV;
     if (al & 15) return fail(PRISM_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
     return launch_attn_bwd(plan->pl, O, dO, dQ, dK, dV, static_cast<cudaStream_t>(stream));

@@ -40,6 +40,7 @@ struct Plan {
     int cap_stride;         // worst-case selected blocks per row
     int device;
     bool have_fwd;
+    bool built;
     // zone statistics and decisions
     double *zone_part;      // [batch][M][nchunk][3]  sum_c of directional variances
     double *zone_a;         // [batch][M][5]  sigma2_a T,H,W, mean a, max a
@@ -103,6 +104,7 @@ prism_status fail_cuda(cudaError_t e, const char *what, const char *file, int li
 prism_status launch_plan(Plan &pl, const void *Q, const void *K, const void *V, const float *a,
                          cudaStream_t st);
 prism_status launch_attn_fwd_tc(Plan &pl, void *O, float *lse, cudaStream_t st);
+prism_status launch_regather(Plan &pl, const void *Q, const void *K, const void *V, cudaStream_t st);
 prism_status make_tensor_maps(Plan &pl);
 prism_status launch_attn_bwd_tc_main(Plan &pl, void *dK, void *dV, cudaStream_t st);
 prism_status launch_attn_bwd(Plan &pl, const void *O, const void *dO, void *dQ, void *dK, void *dV,

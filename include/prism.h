@@ -118,10 +118,20 @@ PRISM_API size_t prism_plan_bytes(const prism_params *params);
 PRISM_API prism_status prism_plan_build(prism_plan *plan, const void *Q, const void *K, const void *V,
                               const float *a_norm, void *stream);
 
+/* Plan reuse: gathers new Q, K, V (device, layouts above) into the plan's
+ * block-contiguous copies using the plan's existing zone shapes, permutation
+ * and selection, which are not recomputed.  Subsequent prism_attn_fwd /
+ * prism_attn_bwd attend with the new inputs under the cached plan -- the
+ * reuse of a sparsity plan across diffusion steps or layers that the DFSAttn
+ * page describes as adaptive mask caching (its third component).  Returns
+ * PRISM_ERR_STATE before the first prism_plan_build.                       */
+PRISM_API prism_status prism_plan_update_qkv(prism_plan *plan, const void *Q, const void *K, const void *V,
+                                             void *stream);
+
 /* Sparse attention forward over the selected blocks of the last build
  * [Prism guide, Method section 3, last sentence]: each query token of block
  * i attends under one online softmax to every token of the key blocks in
- * S_i.  Reads the permuted Q, K, V of the last build.  Writes O (device,
+ * S_i.  Reads the permuted Q, K, V of the last build or update.  Writes O (device,
  * bf16, user layout) and, if lse != NULL, the natural-log log-sum-exp of the
  * scaled scores (device, fp32 [batch][heads][N], raster token order).  The
  * plan keeps its own copy of the statistics for prism_attn_bwd.           */

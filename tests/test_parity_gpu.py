@@ -400,3 +400,31 @@ def test_capped_backward():
     dK_ref, dV_ref = oracle.attn_bwd_dkv_rows(pl, *bits, dOb, req_h, req_t)
     assert_close("dK", g["dK"][0].float().cpu().numpy()[req_t, req_h], dK_ref)
     assert_close("dV", g["dV"][0].float().cpu().numpy()[req_t, req_h], dV_ref)
+
+
+def test_plan_reuse_with_new_inputs():
+    """prism_plan_update_qkv keeps the plan of the first inputs and attends with
+    the second: compare with the oracle's plan of the first inputs applied to
+    the second inputs' Q, K, V."""
+    w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=2, planted=2, backward=True)
+    first = make_inputs(w, 21)
+    second = make_inputs(w, 22)
+    P = _lib()
+    plan = P.PrismPlan(P.params_for(w))
+    plan.build(*(x.cuda() for x in (first.Q, first.K, first.V, first.a)))
+    with pytest.raises(P.PrismError):
+        plan.bwd(torch.zeros_like(first.Q).cuda(), first.dO.cuda())  # no forward yet
+    plan.update_qkv(*(x.cuda() for x in (second.Q, second.K, second.V)))
+    O, lse = plan.fwd()
+    dQ, dK, dV = plan.bwd(O, second.dO.cuda())
+    torch.cuda.synchronize()
+    plan.check()
+    pl, _ = oracle_plan(w, first)
+    compare_plan(w, pl, plan.view())
+    bits2 = tuple(bf16_bits(x[0]) for x in (second.Q, second.K, second.V))
+    rs = np.random.default_rng(4)
+    req_h, req_t = sample_rows(rs, w, 512)
+    O_ref, _ = oracle.attn_fwd_rows(pl, *bits2, req_h, req_t)
+    assert_close("O", O[0].float().cpu().numpy()[req_t, req_h], O_ref)
+    dQ_ref = oracle.attn_bwd_dq_rows(pl, *bits2, bf16_bits(second.dO[0]), req_h[:128], req_t[:128])
+    assert_close("dQ", dQ[0].float().cpu().numpy()[req_t[:128], req_h[:128]], dQ_ref)
