@@ -50,13 +50,14 @@ constexpr uint32_t kColDK = 0, kColDV = 128, kColST = 256, kColDP = 448;
 
 template <int D>
 struct Layout {
-    static_assert(D == 128, "tensor-core backward is written for head_dim 128");
+    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    static constexpr int kHalves = D / 64;          // 64-column (128 B) swizzle atoms along D
     static constexpr uint32_t kKVHalf = 128 * 128;  // 128 rows x 128 B
     static constexpr uint32_t kQHalf = 64 * 128;    // 64 rows x 128 B
     static constexpr uint32_t kK = 0;
-    static constexpr uint32_t kV = kK + 2 * kKVHalf;
-    static constexpr uint32_t kQ0 = kV + 2 * kKVHalf;      // stage s: Q at kQ0 + s*kStage, dO at + 2*kQHalf
-    static constexpr uint32_t kStage = 4 * kQHalf;
+    static constexpr uint32_t kV = kK + kHalves * kKVHalf;
+    static constexpr uint32_t kQ0 = kV + kHalves * kKVHalf;  // stage s: Q at kQ0 + s*kStage, dO at + kHalves*kQHalf
+    static constexpr uint32_t kStage = 2 * kHalves * kQHalf;
     static constexpr uint32_t kDS = kQ0 + kStages * kStage;  // [2] x 128 key rows x 128 B (64 queries bf16)
     static constexpr uint32_t kVec = kDS + 2 * 16384;        // stage s: LSE [64] f32 then Delta [64] f32
     static constexpr uint32_t kDQ = kVec + kStages * 512;    // dQ staging tile [64 queries][D] f32 (128-B aligned)
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             mbar_expect_tx(bar_kv, 2 * 128 * D * 2);
-            for (int hf = 0; hf < 2; ++hf)
+            for (int hf = 0; hf < L::kHalves; ++hf)
                 for (int rh = 0; rh < 2; ++rh) {
                     tma_load_2d(sbase + L::kK + hf * L::kKVHalf + rh * 8192, &tmK, bar_kv, hf * 64,
                                 rowbase + k0 + rh * 64);
@@ -166,11 +167,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (c >= kStages &&
                     !mbar_wait(bar_qe + 8 * st, ((c / kStages) + 1) & 1, status, kSiteQEmpty, abort_flag))
                     break;
-                const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + 2 * L::kQHalf;
+                const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + L::kHalves * L::kQHalf;
                 const uint32_t sVec = sbase + L::kVec + st * 512;
                 const uint32_t bar = bar_qf + 8 * st;
                 mbar_expect_tx(bar, 2 * 64 * D * 2 + 512);
-                for (int hf = 0; hf < 2; ++hf) {
+                for (int hf = 0; hf < L::kHalves; ++hf) {
                     tma_load_2d(sQ + hf * L::kQHalf, &tmQ, bar, hf * 64, rowbase + r);
                     tma_load_2d(sO + hf * L::kQHalf, &tmdO, bar, hf * 64, rowbase + r);
                 }
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return true;
             };
             auto issue_dp = [&](int c) {  // dP^T of chunk c into DP (stage already waited by issue_st)
-                const uint32_t sO = sbase + L::kQ0 + (c % kStages) * L::kStage + 2 * L::kQHalf;
+                const uint32_t sO = sbase + L::kQ0 + (c % kStages) * L::kStage + L::kHalves * L::kQHalf;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ko = (kk >> 2) * L::kKVHalf + (kk & 3) * 32;
@@ -229,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!__all_sync(0xffffffffu, mbar_wait(bar_pf + 8 * (c & 1), (c >> 1) & 1, status, kSiteP, abort_flag))) break;
                 tc_fence_after();
                 if (c + 1 < nchunk) issue_dp(c + 1);
-                const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + 2 * L::kQHalf;
+                const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + L::kHalves * L::kQHalf;
                 const uint32_t tST = tmem + kColST + st * 64;
                 const uint32_t acc = (c > 0) ? 1u : 0u;
 #pragma unroll
@@ -370,8 +371,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (leader) bulk_wait_read_all();
             named_bar_sync(1, 128);
             float *stage = reinterpret_cast<float *>(smem + L::kDQ) + d;
+            if (d < D) {  // head_dim 64: dQ^T rows 64..127 are padding
 #pragma unroll
-            for (int q = 0; q < 64; ++q) stage[q * D] = __uint_as_float(v[q]) * scale;
+                for (int q = 0; q < 64; ++q) stage[q * D] = __uint_as_float(v[q]) * scale;
+            }
             fence_async_smem();
             named_bar_sync(1, 128);
             if (leader) {
@@ -397,23 +400,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace bwdtc
 
 prism_status configure_attn_bwd_tc_kernels() {
+    PRISM_CUDA_OK(cudaFuncSetAttribute(bwdtc::k_attn_bwd_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)bwdtc::Layout<64>::kAlloc));
     PRISM_CUDA_OK(cudaFuncSetAttribute(bwdtc::k_attn_bwd_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bwdtc::Layout<128>::kAlloc));
     return PRISM_OK;
 }
 
-// Runs the tensor-core key-stationary backward (head_dim 128); the caller has
-// zeroed dQacc and written dOp and delta.
-prism_status launch_attn_bwd_tc_main(Plan &pl, void *dK, void *dV, cudaStream_t st) {
+// Runs the tensor-core key-stationary backward; the caller has zeroed dQacc
+// and written dOp and delta.
+template <int D>
+static prism_status bwd_tc_main(Plan &pl, void *dK, void *dV, cudaStream_t st) {
     const Geo &g = pl.g;
-    const double scale = 1.0 / sqrt((double)g.D);
+    const double scale = 1.0 / sqrt((double)D);
     TimerScope ts(pl, kTAttnBwd, st);
-    bwdtc::k_attn_bwd_tc<128><<<dim3(g.nbmax, g.batch * g.heads), bwdtc::kThreads, bwdtc::Layout<128>::kAlloc, st>>>(
-        pl.tmQ, pl.tmK, pl.tmV, pl.tmdO, pl.tmdQ, g, pl.nqt, pl.qt_row, pl.qt_blk, pl.blk_off, pl.colT_ptr, pl.rowT, pl.perm,
-        pl.lse_p, pl.delta, pl.dQacc, static_cast<__nv_bfloat16 *>(dK), static_cast<__nv_bfloat16 *>(dV),
+    bwdtc::k_attn_bwd_tc<D><<<dim3(g.nbmax, g.batch * g.heads), bwdtc::kThreads, bwdtc::Layout<D>::kAlloc, st>>>(
+        pl.tmQ, pl.tmK, pl.tmV, pl.tmdO, pl.tmdQ, g, pl.nqt, pl.qt_row, pl.qt_blk, pl.blk_off, pl.colT_ptr, pl.rowT,
+        pl.perm, pl.lse_p, pl.delta, pl.dQacc, static_cast<__nv_bfloat16 *>(dK), static_cast<__nv_bfloat16 *>(dV),
         (float)scale, (float)(scale * 1.4426950408889634), pl.status);
     PRISM_CUDA_OK(cudaGetLastError());
     return PRISM_OK;
+}
+
+prism_status launch_attn_bwd_tc_main(Plan &pl, void *dK, void *dV, cudaStream_t st) {
+    return pl.g.D == 64 ? bwd_tc_main<64>(pl, dK, dV, st) : bwd_tc_main<128>(pl, dK, dV, st);
 }
 
 }  // namespace prism

@@ -34,7 +34,6 @@ prism_status fail_cuda(cudaError_t e, const char *what, const char *file, int li
 
 int host_shape_table(int (*e)[3]);
 prism_status configure_plan_kernels(const Plan &pl);
-prism_status configure_attn_kernels();
 prism_status configure_attn_tc_kernels();
 prism_status configure_attn_bwd_tc_kernels();
 prism_status launch_selftest_bounded_wait(Plan &pl, cudaStream_t st);
@@ -280,7 +279,6 @@ prism_status prism_plan_create(const prism_params *params, prism_plan **out) {
         return fail_cuda(e, "plan setup", __FILE__, __LINE__);
     }
     s = configure_plan_kernels(pl);
-    if (s == PRISM_OK) s = configure_attn_kernels();
     if (s == PRISM_OK) s = configure_attn_tc_kernels();
     if (s == PRISM_OK) s = configure_attn_bwd_tc_kernels();
     if (s == PRISM_OK) s = make_tensor_maps(pl);
