@@ -172,7 +172,8 @@ def run_ours(args, rank, world, dev):
     def step(Q, K, V, a, dO):
         plan.build(Q, K, V, a)
         plan.fwd(O, lse)
-        plan.bwd(O, dO, dQ, dK, dV)
+        if not args.fwd_only:
+            plan.bwd(O, dO, dQ, dK, dV)
 
     for _ in range(args.warmup):
         step(inp.Q, inp.K, inp.V, inp.a, inp.dO)
@@ -183,7 +184,7 @@ def run_ours(args, rank, world, dev):
     nb = view["n_blocks"][0]
     flops_fwd = 4.0 * w.head_dim * pairs
     flops_bwd = 10.0 * w.head_dim * pairs
-    flops_step = flops_fwd + flops_bwd
+    flops_step = flops_fwd + (0.0 if args.fwd_only else flops_bwd)
 
     def barrier():
         if world > 1:
@@ -214,8 +215,9 @@ def run_ours(args, rank, world, dev):
     # ---- end to end through the public API with pinned host buffers ----
     e2e = None
     if not args.no_e2e:
-        host_in = [x.cpu().pin_memory() for x in (inp.Q, inp.K, inp.V, inp.a, inp.dO)]
-        host_out = [torch.empty(shp, dtype=torch.bfloat16).pin_memory() for _ in range(4)]
+        host_in = [x.cpu().pin_memory() for x in ((inp.Q, inp.K, inp.V, inp.a) if args.fwd_only else
+                                                  (inp.Q, inp.K, inp.V, inp.a, inp.dO))]
+        host_out = [torch.empty(shp, dtype=torch.bfloat16).pin_memory() for _ in range(1 if args.fwd_only else 4)]
         dev_in = [torch.empty_like(x, device=dev) for x in host_in]
         h2d = sum(x.numel() * x.element_size() for x in host_in)
         d2h = sum(x.numel() * x.element_size() for x in host_out)
@@ -223,8 +225,8 @@ def run_ours(args, rank, world, dev):
         def e2e_step():
             for d, h in zip(dev_in, host_in):
                 d.copy_(h, non_blocking=True)
-            step(*dev_in)
-            for h, d in zip(host_out, (O, dQ, dK, dV)):
+            step(*dev_in) if not args.fwd_only else step(*dev_in, None)
+            for h, d in zip(host_out, (O,) if args.fwd_only else (O, dQ, dK, dV)):
                 h.copy_(d, non_blocking=True)
 
         for _ in range(max(1, args.warmup // 2)):
@@ -291,7 +293,8 @@ def run_ours(args, rank, world, dev):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "grid": [w.T, w.H, w.W], "tokens": w.N, "heads": w.heads,
+        "config": {"workload": w.name, "pass": "forward" if args.fwd_only else "forward+backward",
+                   "grid": [w.T, w.H, w.W], "tokens": w.N, "heads": w.heads,
                    "head_dim": w.head_dim, "top_k": w.top_k, "top_p": w.top_p, "max_frac": w.max_frac,
                    "n_blocks": nb, "selected_token_pairs": pairs, "flops_per_step": flops_step,
                    "l2": "inputs larger than L2 (Q,K,V,dO 2.26 GB each)", "parallelism": f"replicas x{world}"},
@@ -415,6 +418,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="latent2k_train_24x96x160")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--fwd-only", action="store_true", help="step = plan + forward (forward-only workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the workload's head count (profiling)")
     ap.add_argument("--cpu-rows", type=int, default=6000)
