@@ -25,14 +25,18 @@
 // to be drained; the single DP buffer is refilled (dP^T of chunk c+1) as soon
 // as the softmax of chunk c has read it.
 // TMEM columns: dK [0,128), dV [128,256), ST[3] [256,448), DP [448,512).
-// In an ST buffer, after the softmax, columns [32h, 32h+16) hold P^T and
-// [32h+16, 32h+32) hold dS^T of queries [32h, 32h+32) (h = 0, 1), packed as
+// In an ST buffer, after the softmax, columns [16g, 16g+8) hold P^T and
+// [16g+8, 16g+16) hold dS^T of queries [16g, 16g+16) (g = 0..3), packed as
 // bf16 pairs.
 //
-// Warp roles (448 threads): warp 0 TMA producer (K, V once; Q, dO, LSE,
-// Delta per chunk into a three-stage ring; LSE is kept in log2 units), warp 1 MMA issuer, warps 2..9
-// softmax (a key row and 32 of the 64 query columns each), warps 10..13 dQ
-// drain (one head-dim row each).
+// The softmax is the loop's critical path (dP^T of chunk c+1 waits for it,
+// and the softmax of c+1 waits for that), so it is spread over 16 warps, each
+// owning one TMEM lane quadrant (32 key rows) and 16 query columns: many short
+// independent exp2 chains instead of a few long ones.
+// Warp roles (704 threads): warp 0 TMA producer (K, V once; Q, dO, LSE,
+// Delta per chunk into a three-stage ring; LSE is kept in log2 units), warp 1
+// MMA issuer, warps 2..17 softmax, warps 18..21 dQ drain (one head-dim row
+// each).
 #include <cuda.h>
 
 #include "tc_common.cuh"
@@ -43,7 +47,8 @@ using namespace tc;
 
 namespace bwdtc {
 
-constexpr int kThreads = 448;
+constexpr int kSoftmaxWarps = 16;
+constexpr int kThreads = 32 * (2 + kSoftmaxWarps + 4);
 constexpr int kStages = 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDK = 0, kColDV = 128, kColST = 256, kColDP = 448;
@@ -69,6 +74,16 @@ struct Layout {
     static_assert(kAlloc <= 232448, "shared memory per block");
     static_assert(kDQ % 128 == 0, "TMA source alignment");
 };
+
+// S^T / dP^T: contraction over the head dimension, A (K or V rows) and B (Q or
+// dO rows) K-major, their 64-column halves kKVHalf and kQHalf bytes apart.
+template <int D>
+__device__ __forceinline__ void mma_over_d(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc) {
+    if constexpr (D == 128)
+        mma_ss8<2, 4, 6, 1024, 1026, 1028, 1030, 2, 4, 6, 512, 514, 516, 518>(d_tmem, adesc, bdesc, idesc, 0u);
+    else
+        mma_ss4<2, 4, 6, 2, 4, 6>(d_tmem, adesc, bdesc, idesc, 0u);
+}
 
 enum { kSiteKV = 11, kSiteQFull, kSiteQEmpty, kSiteS, kSiteP, kSiteDQFull, kSiteDQEmpty, kSiteDone };
 
@@ -124,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int s = 0; s < 2; ++s) {
                 mbar_init(bar_sf + 8 * s, 1);
-                mbar_init(bar_pf + 8 * s, 256);
+                mbar_init(bar_pf + 8 * s, 32 * kSoftmaxWarps);
             }
             mbar_init(bar_done, 1);
             *abort_flag = 0;
@@ -200,24 +215,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!__all_sync(0xffffffffu, mbar_wait(bar_qf + 8 * st, (c / kStages) & 1, status, kSiteQFull, abort_flag))) return false;
                 tc_fence_after();
                 const uint32_t sQ = sbase + L::kQ0 + st * L::kStage;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t ko = (kk >> 2) * L::kKVHalf + (kk & 3) * 32;
-                    const uint32_t qo = (kk >> 2) * L::kQHalf + (kk & 3) * 32;
-                    mma_ss(tmem + kColST + st * 64, sdesc(sbase + L::kK + ko, 16, 1024), sdesc(sQ + qo, 16, 1024),
-                           idST, kk > 0);
-                }
+                mma_over_d<D>(tmem + kColST + st * 64, sdesc(sbase + L::kK, 16, 1024), sdesc(sQ, 16, 1024), idST);
                 return true;
             };
             auto issue_dp = [&](int c) {  // dP^T of chunk c into DP (stage already waited by issue_st)
                 const uint32_t sO = sbase + L::kQ0 + (c % kStages) * L::kStage + L::kHalves * L::kQHalf;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t ko = (kk >> 2) * L::kKVHalf + (kk & 3) * 32;
-                    const uint32_t qo = (kk >> 2) * L::kQHalf + (kk & 3) * 32;
-                    mma_ss(tmem + kColDP, sdesc(sbase + L::kV + ko, 16, 1024), sdesc(sO + qo, 16, 1024), idST,
-                           kk > 0);
-                }
+                mma_over_d<D>(tmem + kColDP, sdesc(sbase + L::kV, 16, 1024), sdesc(sO, 16, 1024), idST);
                 mma_commit(bar_sf + 8 * (c & 1));
             };
             if (ok) {
@@ -233,20 +236,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + L::kHalves * L::kQHalf;
                 const uint32_t tST = tmem + kColST + st * 64;
                 const uint32_t acc = (c > 0) ? 1u : 0u;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + kColDV, tST + 32 * (kk >> 1) + 8 * (kk & 1), sdesc(sO + kk * 2048, L::kQHalf, 1024),
-                           idAcc, acc | (kk > 0));
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + kColDK, tST + 32 * (kk >> 1) + 16 + 8 * (kk & 1),
-                           sdesc(sQ + kk * 2048, L::kQHalf, 1024), idAcc, acc | (kk > 0));
+                // k-step kk of P^T / dS^T: columns 16 kk (+8 for dS^T);
+                // of dO / Q: 16 rows = 2048 B further
+                mma_ts4x2<16, 32, 48, 128, 256, 384>(tmem + kColDV, tST, sdesc(sO, L::kQHalf, 1024), tmem + kColDK,
+                                                      tST + 8, sdesc(sQ, L::kQHalf, 1024), idAcc, acc);
                 mma_commit(bar_qe + 8 * st);
                 const uint32_t sDS = sbase + L::kDS + (c & 1) * 16384;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tST, sdesc(sbase + L::kK + kk * 2048, L::kKVHalf, 1024), sdesc(sDS + kk * 2048, 8192, 1024),
-                           idDQ, kk > 0);
+                // K^T and dS^T MN-major: k-step kk (16 keys) 2048 B further in both
+                mma_ss8<128, 256, 384, 512, 640, 768, 896, 128, 256, 384, 512, 640, 768, 896>(
+                    tST, sdesc(sbase + L::kK, L::kKVHalf, 1024), sdesc(sDS, 8192, 1024), idDQ, 0u);
                 mma_commit(bar_df + 8 * st);
                 if (c + 2 < nchunk) {
                     const int b2 = (c + 2) % kStages;  // = (c - 1) % 3: the buffer chunk c-1 used
@@ -258,10 +256,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             mma_commit(bar_done);
         }
-    } else if (warp < 10) {
+    } else if (warp < 2 + kSoftmaxWarps) {
         // ------------------------------------------------------------ softmax (key rows)
-        const int quad = warp & 3;
-        const int hh = (warp - 2) >> 2;  // which 32 query columns
+        const int quad = warp & 3;          // TMEM lane quadrant this warp may access
+        const int cg = (warp - 2) >> 2;     // its 16 query columns [16 cg, 16 cg + 16)
         const int rowid = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const bool live = rowid < kvalid;
@@ -273,58 +271,59 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                        abort_flag));
             if (!ok) break;
             tc_fence_after();
-            const float *vec = reinterpret_cast<const float *>(smem + L::kVec + st * 512) + hh * 32;
-            const uint32_t tST = tmem + kColST + st * 64 + 32 * hh + lane_off;
-            const uint32_t tDP = tmem + kColDP + 32 * hh + lane_off;
-            uint32_t sv[32], dv[32];
-            tmem_ld32(tST, sv);
-            tmem_ld32(tDP, dv);
-            tmem_wait_ld();
-            uint32_t pk[16], dk[16];
-            const float4 *lse4 = reinterpret_cast<const float4 *>(vec);
-            const float4 *del4 = reinterpret_cast<const float4 *>(vec + 64);
-#pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-                const float4 L4 = lse4[e4], D4 = del4[e4];
-                const int q = 4 * e4;
-                float p0 = ex2(fmaf(__uint_as_float(sv[q]), scale_log2, -L4.x));
-                float p1 = ex2(fmaf(__uint_as_float(sv[q + 1]), scale_log2, -L4.y));
-                float p2 = ex2(fmaf(__uint_as_float(sv[q + 2]), scale_log2, -L4.z));
-                float p3 = ex2(fmaf(__uint_as_float(sv[q + 3]), scale_log2, -L4.w));
-                float d0 = p0 * (__uint_as_float(dv[q]) - D4.x);
-                float d1 = p1 * (__uint_as_float(dv[q + 1]) - D4.y);
-                float d2 = p2 * (__uint_as_float(dv[q + 2]) - D4.z);
-                float d3 = p3 * (__uint_as_float(dv[q + 3]) - D4.w);
-                if (!live) p0 = p1 = p2 = p3 = d0 = d1 = d2 = d3 = 0.f;
-                pk[2 * e4] = pack_bf16x2(p0, p1);
-                pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
-                dk[2 * e4] = pack_bf16x2(d0, d1);
-                dk[2 * e4 + 1] = pack_bf16x2(d2, d3);
-            }
-            tmem_st16(tST, pk);
-            tmem_st16(tST + 16, dk);
-            uint8_t *dsrow = smem + L::kDS + (c & 1) * 16384 + rowid * 128;
+            const uint32_t tST = tmem + kColST + st * 64 + 16 * cg + lane_off;
+            uint32_t sv[16], dv[16];
+            tmem_ld16(tST, sv);
+            tmem_ld16(tmem + kColDP + 16 * cg + lane_off, dv);
+            // LSE (log2 units) and Delta of the 16 queries: the same for every lane
+            const uint32_t vec = sbase + L::kVec + st * 512 + cg * 64;
+            float4 L4[4], D4[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int chunk = hh * 4 + j;
-                *reinterpret_cast<uint4 *>(dsrow + ((chunk ^ (rowid & 7)) << 4)) =
-                    make_uint4(dk[4 * j], dk[4 * j + 1], dk[4 * j + 2], dk[4 * j + 3]);
+                L4[j] = lds_f4(vec + 16 * j);
+                D4[j] = lds_f4(vec + 256 + 16 * j);
             }
+            tmem_wait_ld();
+            uint32_t pd[16];  // P^T pairs then dS^T pairs
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int q = 4 * j;
+                float p0 = ex2(fmaf(__uint_as_float(sv[q]), scale_log2, -L4[j].x));
+                float p1 = ex2(fmaf(__uint_as_float(sv[q + 1]), scale_log2, -L4[j].y));
+                float p2 = ex2(fmaf(__uint_as_float(sv[q + 2]), scale_log2, -L4[j].z));
+                float p3 = ex2(fmaf(__uint_as_float(sv[q + 3]), scale_log2, -L4[j].w));
+                float d0 = p0 * (__uint_as_float(dv[q]) - D4[j].x);
+                float d1 = p1 * (__uint_as_float(dv[q + 1]) - D4[j].y);
+                float d2 = p2 * (__uint_as_float(dv[q + 2]) - D4[j].z);
+                float d3 = p3 * (__uint_as_float(dv[q + 3]) - D4[j].w);
+                if (!live) p0 = p1 = p2 = p3 = d0 = d1 = d2 = d3 = 0.f;
+                pd[2 * j] = pack_bf16x2(p0, p1);
+                pd[2 * j + 1] = pack_bf16x2(p2, p3);
+                pd[8 + 2 * j] = pack_bf16x2(d0, d1);
+                pd[8 + 2 * j + 1] = pack_bf16x2(d2, d3);
+            }
+            // P^T over columns [16 cg, 16 cg + 8), dS^T over [16 cg + 8, 16 cg + 16): this warp's own S^T columns
+            tmem_st16(tST, pd);
+            // dS^T row to shared memory for dQ^T: 16-byte chunks 2 cg, 2 cg + 1 of the 128-byte row, swizzled
+            const uint32_t dsrow = sbase + L::kDS + (c & 1) * 16384 + rowid * 128;
+            sts_u4(dsrow + (((2 * cg) ^ (rowid & 7)) << 4), pd[8], pd[9], pd[10], pd[11]);
+            sts_u4(dsrow + (((2 * cg + 1) ^ (rowid & 7)) << 4), pd[12], pd[13], pd[14], pd[15]);
             tmem_wait_st();
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(bar_pf + 8 * (c & 1));
         }
-        // epilogue: the first warp group writes dK (scaled), the second dV
+        // epilogue: column groups 0, 1 write halves of dK (scaled), 2, 3 halves of dV
         if (ok && nchunk > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, status, kSiteDone, abort_flag));
         if (ok) {
             tc_fence_after();
             const int tok = live ? perm[(size_t)b * g.N + k0 + rowid] : 0;
-            __nv_bfloat16 *dst = (hh == 0 ? dK : dV) + (((size_t)b * g.N + tok) * g.heads + h) * D;
-            const uint32_t src = tmem + (hh == 0 ? kColDK : kColDV) + lane_off;
-            const float f = (hh == 0) ? scale : 1.0f;
+            const int c0 = (cg & 1) * (D / 2);
+            __nv_bfloat16 *dst = (cg < 2 ? dK : dV) + (((size_t)b * g.N + tok) * g.heads + h) * D + c0;
+            const uint32_t src = tmem + (cg < 2 ? kColDK : kColDV) + c0 + lane_off;
+            const float f = (cg < 2) ? scale : 1.0f;
 #pragma unroll 1
-            for (int q = 0; q < D / 32; ++q) {
+            for (int q = 0; q < D / 64; ++q) {
                 uint32_t a[32];
                 if (nchunk > 0) {
                     tmem_ld32(src + q * 32, a);
@@ -349,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp & 3;
         const int d = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const bool leader = (warp == 10 && lane == 0);
+        const bool leader = (warp == 2 + kSoftmaxWarps && lane == 0);
         int u = u_begin, r = 0, r_end = 0;
         if (u < u_end) {
             r = bo[rowT[u]];
@@ -361,19 +360,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mbar_wait(bar_df + 8 * st, (c / kStages) & 1, status, kSiteDQFull, abort_flag)))
                 break;
             tc_fence_after();
-            uint32_t v[64];
-            tmem_ld32(tmem + kColST + st * 64 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(v));
-            tmem_ld32(tmem + kColST + st * 64 + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+            uint32_t v[32], w[32];
+            tmem_ld32(tmem + kColST + st * 64 + lane_off, v);
+            tmem_ld32(tmem + kColST + st * 64 + lane_off + 32, w);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar_de + 8 * st);
             // the staging tile is free once the previous reduce has read it
             if (leader) bulk_wait_read_all();
             named_bar_sync(1, 128);
-            float *stage = reinterpret_cast<float *>(smem + L::kDQ) + d;
+            const uint32_t stage = sbase + L::kDQ + d * 4;
             if (d < D) {  // head_dim 64: dQ^T rows 64..127 are padding
 #pragma unroll
-                for (int q = 0; q < 64; ++q) stage[q * D] = __uint_as_float(v[q]) * scale;
+                for (int q = 0; q < 32; ++q) sts_f32(stage + q * D * 4, __uint_as_float(v[q]) * scale);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) sts_f32(stage + (q + 32) * D * 4, __uint_as_float(w[q]) * scale);
             }
             fence_async_smem();
             named_bar_sync(1, 128);

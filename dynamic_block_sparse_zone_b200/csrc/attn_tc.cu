@@ -179,21 +179,24 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const bool full = (2 * c + 1) < nseg;
                 if (!__all_sync(0xffffffffu, mbar_wait(bar_kf, c & 1, status, kSiteK, abort_flag))) break;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * L::kTileBytes + (kk & 3) * 32;
-                    mma_ss(tS, sdesc(sbase + L::kQ + off, 16, 1024), sdesc(sbase + L::kK + off, 16, 1024),
-                           full ? idS128 : idS64, kk > 0);
-                }
+                // k-step kk: 32 B along a 128-B row, the second 64 columns a tile further
+                const uint64_t aQ = sdesc(sbase + L::kQ, 16, 1024), bK = sdesc(sbase + L::kK, 16, 1024);
+                if constexpr (D == 128)
+                    mma_ss8<2, 4, 6, 1024, 1026, 1028, 1030, 2, 4, 6, 1024, 1026, 1028, 1030>(
+                        tS, aQ, bK, full ? idS128 : idS64, 0u);
+                else
+                    mma_ss4<2, 4, 6, 2, 4, 6>(tS, aQ, bK, full ? idS128 : idS64, 0u);
                 mma_commit(bar_s);
                 mma_commit(bar_ke);
                 if (!__all_sync(0xffffffffu, mbar_wait(bar_p, c & 1, status, kSiteP, abort_flag))) break;
                 if (!__all_sync(0xffffffffu, mbar_wait(bar_vf, c & 1, status, kSiteV, abort_flag))) break;
                 tc_fence_after();
-                const int nk = full ? 128 : 64;
-                for (int kk = 0; kk < nk / 16; ++kk)
-                    mma_ts(tO, tS + kk * 8, sdesc(sbase + L::kV + kk * 2048, L::kTileBytes, 1024), idPV,
-                           (c > 0 || kk > 0) ? 1u : 0u);
+                // k-step kk (16 keys): P columns 8 kk, V rows 2048 B further
+                const uint64_t bV = sdesc(sbase + L::kV, L::kTileBytes, 1024);
+                if (full)
+                    mma_ts8<8, 16, 24, 32, 40, 48, 56, 128, 256, 384, 512, 640, 768, 896>(tO, tS, bV, idPV, c > 0);
+                else
+                    mma_ts4<8, 16, 24, 128, 256, 384>(tO, tS, bV, idPV, c > 0);
                 mma_commit(bar_ve);
                 mma_commit(bar_o);
             }

@@ -89,6 +89,18 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(nthreads) : "memory");
 }
+// shared-memory accesses by 32-bit shared-window address
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];\n" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void sts_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
+    asm volatile("st.shared.f32 [%0], %1;\n" ::"r"(addr), "f"(v) : "memory");
+}
 // generic-proxy shared-memory writes -> visible to the async proxy (tensor cores)
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 __device__ __forceinline__ void prefetch_map(const CUtensorMap *map) {
@@ -140,31 +152,92 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 
 // ---- MMA ----
 // The issuing helpers are executed by a whole, converged warp: operands are
-// warp-uniform (they stay in the uniform datapath) and elect.sync picks the
-// single lane that issues.  The same lane is elected every time (lowest lane
-// of a full mask), so a commit tracks the MMAs issued before it.
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T   (kind::f16, one CTA)
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
+// warp-uniform and elect.sync picks the single lane that issues.  The same
+// lane is elected every time (lowest lane of a full mask), so a commit tracks
+// the MMAs issued before it.  kind::f16: D[tmem] (+)= A * B^T, one CTA.
+// Batched issue.  A run of MMAs issued from ONE inline-asm block, with the
+// descriptor steps computed inside it, issues at the tensor-core rate on
+// sm_100a; the same MMAs issued one asm block each measured 1.5-2x slower per
+// instruction (an issue-rate probe: 8 x M128 N128 K16 smem-operand MMAs took
+// 64 cycles each batched and about 105 one by one).  Offsets are template
+// immediates: descriptor offsets in 16-byte units (the start-address field),
+// TMEM offsets in columns.  The first MMA of a run takes `accumulate`; the
+// rest accumulate.
+#define PRISM_MMA_HEAD                   \
+    "{\n\t.reg .pred p, e, t;\n\t"       \
+    ".reg .b64 x, y;\n\t.reg .b32 z;\n\t" \
+    "setp.ne.b32 p, %4, 0;\n\t"          \
+    "setp.ne.b32 t, %3, 0;\n\t"          \
+    "elect.sync _|e, 0xffffffff;\n\t"
+#define PRISM_MMA_SS_FIRST "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+#define PRISM_MMA_SS_NEXT(ia, ib) \
+    "add.s64 x, %1, %" #ia ";\n\tadd.s64 y, %2, %" #ib ";\n\t@e tcgen05.mma.cta_group::1.kind::f16 [%0], x, y, %3, t;\n\t"
+
+// Eight smem-operand MMAs into one accumulator: A = a + A_i, B = b + B_i.
+template <uint32_t A1, uint32_t A2, uint32_t A3, uint32_t A4, uint32_t A5, uint32_t A6, uint32_t A7, uint32_t B1,
+          uint32_t B2, uint32_t B3, uint32_t B4, uint32_t B5, uint32_t B6, uint32_t B7>
+__device__ __forceinline__ void mma_ss8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(PRISM_MMA_HEAD PRISM_MMA_SS_FIRST PRISM_MMA_SS_NEXT(5, 12) PRISM_MMA_SS_NEXT(6, 13)
+                     PRISM_MMA_SS_NEXT(7, 14) PRISM_MMA_SS_NEXT(8, 15) PRISM_MMA_SS_NEXT(9, 16)
+                         PRISM_MMA_SS_NEXT(10, 17) PRISM_MMA_SS_NEXT(11, 18) "}\n" ::"r"(d_tmem),
+                 "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "n"(A1), "n"(A2), "n"(A3), "n"(A4), "n"(A5),
+                 "n"(A6), "n"(A7), "n"(B1), "n"(B2), "n"(B3), "n"(B4), "n"(B5), "n"(B6), "n"(B7)
+                 : "memory");
 }
-// D[tmem] (+)= A[tmem] * B[smem desc]^T
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
+// Four smem-operand MMAs into one accumulator.
+template <uint32_t A1, uint32_t A2, uint32_t A3, uint32_t B1, uint32_t B2, uint32_t B3>
+__device__ __forceinline__ void mma_ss4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(PRISM_MMA_HEAD PRISM_MMA_SS_FIRST PRISM_MMA_SS_NEXT(5, 8) PRISM_MMA_SS_NEXT(6, 9)
+                     PRISM_MMA_SS_NEXT(7, 10) "}\n" ::"r"(d_tmem),
+                 "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "n"(A1), "n"(A2), "n"(A3), "n"(B1), "n"(B2),
+                 "n"(B3)
+                 : "memory");
 }
+#define PRISM_MMA_TS_FIRST(dd) "@e tcgen05.mma.cta_group::1.kind::f16 [%" #dd "], [%1], %2, %3, p;\n\t"
+#define PRISM_MMA_TS_NEXT(dd, ia, ib, pr)                                                 \
+    "add.u32 z, %1, %" #ia ";\n\tadd.s64 y, %2, %" #ib ";\n\t@e tcgen05.mma.cta_group::1.kind::f16 [%" #dd \
+    "], [z], y, %3, " #pr ";\n\t"
+#define PRISM_MMA_TS2_FIRST "@e tcgen05.mma.cta_group::1.kind::f16 [%5], [%6], %7, %3, p;\n\t"
+#define PRISM_MMA_TS2_NEXT(ia, ib)                                                                   \
+    "add.u32 z, %6, %" #ia ";\n\tadd.s64 y, %7, %" #ib ";\n\t@e tcgen05.mma.cta_group::1.kind::f16 [%5], [z], y, %3, " \
+    "t;\n\t"
+// Two runs of four MMAs with A from TMEM and B from shared memory, the same
+// steps in both: d0 (+)= [a0 + A_i] * (b0 + B_i), then d1 (+)= [a1 + A_i] *
+// (b1 + B_i).  Each run's first MMA takes `accumulate`.
+template <uint32_t A1, uint32_t A2, uint32_t A3, uint32_t B1, uint32_t B2, uint32_t B3>
+__device__ __forceinline__ void mma_ts4x2(uint32_t d0, uint32_t a0, uint64_t b0, uint32_t d1, uint32_t a1,
+                                          uint64_t b1, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(PRISM_MMA_HEAD PRISM_MMA_TS_FIRST(0) PRISM_MMA_TS_NEXT(0, 8, 11, t) PRISM_MMA_TS_NEXT(0, 9, 12, t)
+                     PRISM_MMA_TS_NEXT(0, 10, 13, t) PRISM_MMA_TS2_FIRST PRISM_MMA_TS2_NEXT(8, 11)
+                         PRISM_MMA_TS2_NEXT(9, 12) PRISM_MMA_TS2_NEXT(10, 13) "}\n" ::"r"(d0),
+                 "r"(a0), "l"(b0), "r"(idesc), "r"(accumulate), "r"(d1), "r"(a1), "l"(b1), "n"(A1), "n"(A2), "n"(A3),
+                 "n"(B1), "n"(B2), "n"(B3)
+                 : "memory");
+}
+// Eight (or four) MMAs with A from TMEM into one accumulator.
+template <uint32_t A1, uint32_t A2, uint32_t A3, uint32_t A4, uint32_t A5, uint32_t A6, uint32_t A7, uint32_t B1,
+          uint32_t B2, uint32_t B3, uint32_t B4, uint32_t B5, uint32_t B6, uint32_t B7>
+__device__ __forceinline__ void mma_ts8(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(PRISM_MMA_HEAD PRISM_MMA_TS_FIRST(0) PRISM_MMA_TS_NEXT(0, 5, 12, t) PRISM_MMA_TS_NEXT(0, 6, 13, t)
+                     PRISM_MMA_TS_NEXT(0, 7, 14, t) PRISM_MMA_TS_NEXT(0, 8, 15, t) PRISM_MMA_TS_NEXT(0, 9, 16, t)
+                         PRISM_MMA_TS_NEXT(0, 10, 17, t) PRISM_MMA_TS_NEXT(0, 11, 18, t) "}\n" ::"r"(d_tmem),
+                 "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "n"(A1), "n"(A2), "n"(A3), "n"(A4), "n"(A5),
+                 "n"(A6), "n"(A7), "n"(B1), "n"(B2), "n"(B3), "n"(B4), "n"(B5), "n"(B6), "n"(B7)
+                 : "memory");
+}
+template <uint32_t A1, uint32_t A2, uint32_t A3, uint32_t B1, uint32_t B2, uint32_t B3>
+__device__ __forceinline__ void mma_ts4(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(PRISM_MMA_HEAD PRISM_MMA_TS_FIRST(0) PRISM_MMA_TS_NEXT(0, 5, 8, t) PRISM_MMA_TS_NEXT(0, 6, 9, t)
+                     PRISM_MMA_TS_NEXT(0, 7, 10, t) "}\n" ::"r"(d_tmem),
+                 "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "n"(A1), "n"(A2), "n"(A3), "n"(B1), "n"(B2),
+                 "n"(B3)
+                 : "memory");
+}
+
 // Arrive on `bar` once every MMA issued so far by the elected lane completes.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile(
