@@ -69,7 +69,7 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.f.close()
-        sms, mx, reasons = [], None, set()
+        sms, watts, mx, reasons = [], [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
             for line in f:
@@ -81,6 +81,10 @@ class ClockSampler:
                     mx = float(parts[2])
                 except ValueError:
                     continue
+                try:
+                    watts.append(float(parts[3]))
+                except ValueError:
+                    pass
                 for n, v in zip(names, parts[5:9]):
                     if v.lower().startswith("active"):
                         reasons.add(n)
@@ -88,7 +92,7 @@ class ClockSampler:
         if not sms:
             return None
         return {"sm_mhz": statistics.median(sms), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sms)}
+                "power_w": statistics.median(watts) if watts else None, "samples": len(sms)}
 
 
 # --------------------------------------------------------------------------

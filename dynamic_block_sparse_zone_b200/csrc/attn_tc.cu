@@ -17,7 +17,8 @@
 //   warp 0       TMA producer: Q once; K_c into the K buffer once S_{c-1} has
 //                read it, V_c into the V buffer once P_{c-1} V_{c-1} has.
 //   warp 1       MMA issuer (whole warp, one elected lane issues).
-//   warps 2..5   softmax, one query row per thread (= TMEM lane): pass 1 row
+//   warps 2..5   softmax, one query row per thread (= TMEM lane): the S row
+//                comes into registers in one TMEM round trip; pass 1 row
 //                max, pass 2 exp2 / running sum / bf16 P written back over S.
 //                O is rescaled in TMEM only when the running max grows by more
 //                than 2^8 (it is current then: S_c was issued after PV_{c-1}).
@@ -214,15 +215,20 @@ __global__ void __launch_bounds__(kThreads, 2)
             tc_fence_after();
             const int nq = ((2 * c + 1) < nseg) ? 4 : 2;  // 32-column groups of S in this chunk
             const uint32_t tSr = tS + lane_off;
+            // the whole S row into registers: one TMEM round trip for both passes
+            uint32_t sr[128];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (q < nq) tmem_ld32(tSr + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * q]));
+            tmem_wait_ld();
             // pass 1: row max
             float mx = -INFINITY;
-            for (int q = 0; q < nq; ++q) {
-                uint32_t sr[32];
-                tmem_ld32(tSr + q * 32, sr);
-                tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[e]));
-            }
+            for (int q = 0; q < 4; ++q)
+                if (q < nq) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[32 * q + e]));
+                }
             const float mx2 = mx * scale_log2;
             const bool need = (c > 0) && (mx2 > m + kRescaleThreshold);
             if (c == 0) m = mx2;
@@ -233,34 +239,33 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const float mnew = fmaxf(m, mx2);
                 const float corr = ex2(m - mnew);
 #pragma unroll 1
-                for (int q = 0; q < D / 32; ++q) {
-                    uint32_t orr[32];
-                    tmem_ld32(tO + lane_off + q * 32, orr);
+                for (int q = 0; q < D / 16; ++q) {
+                    uint32_t orr[16];
+                    tmem_ld16(tO + lane_off + q * 16, orr);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * corr);
-                    tmem_st32(tO + lane_off + q * 32, orr);
+                    for (int e = 0; e < 16; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * corr);
+                    tmem_st16(tO + lane_off + q * 16, orr);
                 }
                 l *= corr;
                 m = mnew;
             }
-            // pass 2: P = exp2(S*scale*log2e - m), bf16 pairs written over S.
-            // Group q packs into columns [16q, 16q+16), which pass 2 has already read.
+            // pass 2: P = exp2(S*scale*log2e - m), bf16 pairs written over S
+            // (group q packs into columns [16q, 16q+16); all of S is in registers).
             float sum = 0.f;
-            for (int q = 0; q < nq; ++q) {
-                uint32_t sr[32];
-                tmem_ld32(tSr + q * 32, sr);
-                tmem_wait_ld();
-                uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2(fmaf(__uint_as_float(sr[2 * e]), scale_log2, -m));
-                    const float p1 = ex2(fmaf(__uint_as_float(sr[2 * e + 1]), scale_log2, -m));
-                    sum += p0 + p1;
-                    pk[e] = pack_bf16x2(p0, p1);
+            for (int q = 0; q < 4; ++q)
+                if (q < nq) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = ex2(fmaf(__uint_as_float(sr[32 * q + 2 * e]), scale_log2, -m));
+                        const float p1 = ex2(fmaf(__uint_as_float(sr[32 * q + 2 * e + 1]), scale_log2, -m));
+                        sum += p0 + p1;
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(tSr + q * 16, pk);
                 }
-                tmem_st16(tSr + q * 16, pk);
-            }
             l += sum;
             tmem_wait_st();
             tc_fence_before();
