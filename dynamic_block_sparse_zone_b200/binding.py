@@ -24,7 +24,8 @@ _STATUS = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_UNSUPPORTED"
 EXPORTED = ("prism_plan_create", "prism_plan_bytes", "prism_plan_build", "prism_attn_fwd", "prism_attn_bwd",
             "prism_plan_view_get", "prism_plan_check", "prism_plan_destroy", "prism_last_error",
             "prism_plan_set_timing", "prism_plan_read_timing", "prism_timer_name", "prism_zone_shapes_noalloc",
-            "prism_plan_selftest_timeout", "prism_plan_update_qkv")
+            "prism_plan_selftest_timeout", "prism_plan_update_qkv", "prism_step_host", "prism_step_join",
+            "prism_step_wait")
 NUM_TIMERS = 10
 
 
@@ -50,6 +51,10 @@ class prism_plan_view(ctypes.Structure):
 _lib = None
 
 
+class prism_host_io(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("Q", "K", "V", "a_norm", "dO", "O", "lse", "dQ", "dK", "dV")]
+
+
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     """Loads libprism.so; raises if it has not been built."""
     global _lib
@@ -71,6 +76,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.prism_plan_check.argtypes = [V, P]
     lib.prism_plan_selftest_timeout.argtypes = [V, P]
     lib.prism_plan_selftest_timeout.restype = ctypes.c_int
+    lib.prism_step_host.argtypes = [V, ctypes.POINTER(prism_host_io), P, ctypes.POINTER(ctypes.c_ulonglong)]
+    lib.prism_step_host.restype = ctypes.c_int
+    lib.prism_step_join.argtypes = [V, ctypes.c_ulonglong, P]
+    lib.prism_step_join.restype = ctypes.c_int
+    lib.prism_step_wait.argtypes = [V, ctypes.c_ulonglong]
+    lib.prism_step_wait.restype = ctypes.c_int
     lib.prism_plan_destroy.argtypes = [V]
     lib.prism_plan_destroy.restype = None
     lib.prism_last_error.restype = ctypes.c_char_p
@@ -157,11 +168,13 @@ class PrismPlan:
         h = ctypes.c_void_p()
         _check(load_library().prism_plan_create(ctypes.byref(self._c), ctypes.byref(h)))
         self._h = h
+        self._held = {}  # ticket -> host tensors a queued step reads or writes
 
     def close(self):
         if getattr(self, "_h", None) is not None and self._h.value:
-            load_library().prism_plan_destroy(self._h)
+            load_library().prism_plan_destroy(self._h)  # waits for queued host steps
             self._h = None
+        self._held = {}
 
     def __del__(self):
         try:
@@ -213,6 +226,39 @@ class PrismPlan:
             _need(t, n, torch.bfloat16, shp)
         _check(load_library().prism_attn_bwd(self._h, _ptr(O), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _stream()))
         return dQ, dK, dV
+
+    # -- steps from host memory (pipelined across calls) ---------------------
+    def step_host(self, Q, K, V, a_norm, O, lse=None, dO=None, dQ=None, dK=None, dV=None) -> int:
+        """Enqueues one layer step on host tensors (page-locked for overlap) and
+        returns its ticket; the tensors are kept alive until step_wait covers it."""
+        p = self.params
+        shp = self._qkv_shape()
+        host = [(Q, "Q", torch.bfloat16, shp), (K, "K", torch.bfloat16, shp), (V, "V", torch.bfloat16, shp),
+                (a_norm, "a_norm", torch.float32, (p.batch, p.T, p.H, p.W)), (O, "O", torch.bfloat16, shp)]
+        if lse is not None:
+            host.append((lse, "lse", torch.float32, (p.batch, p.heads, p.N)))
+        if dO is not None:
+            if dQ is None or dK is None or dV is None:
+                raise ValueError("a step with dO needs dQ, dK and dV")
+            host += [(t, n, torch.bfloat16, shp) for t, n in ((dO, "dO"), (dQ, "dQ"), (dK, "dK"), (dV, "dV"))]
+        for t, n, dt, sh in host:
+            if t.is_cuda or t.dtype != dt or tuple(t.shape) != tuple(sh) or not t.is_contiguous():
+                raise ValueError(f"{n}: expected a contiguous host tensor {dt} {tuple(sh)}")
+        io = prism_host_io(*(None if t is None else t.data_ptr() for t in (Q, K, V, a_norm, dO, O, lse, dQ, dK, dV)))
+        tk = ctypes.c_ulonglong()
+        _check(load_library().prism_step_host(self._h, ctypes.byref(io), _stream(), ctypes.byref(tk)))
+        self._held[tk.value] = [t for t, *_ in host]
+        return tk.value
+
+    def step_join(self, ticket: int):
+        """The current CUDA stream waits (on the device) for step `ticket`."""
+        _check(load_library().prism_step_join(self._h, ticket, _stream()))
+
+    def step_wait(self, ticket: int):
+        """Blocks until step `ticket` (and every earlier one) has its outputs in host memory."""
+        _check(load_library().prism_step_wait(self._h, ticket))
+        for t in [t for t in self._held if t <= ticket]:
+            del self._held[t]
 
     # -- per-kernel event timing ---------------------------------------------
     def set_timing(self, enable: bool = True):

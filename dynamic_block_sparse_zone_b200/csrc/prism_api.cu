@@ -194,6 +194,7 @@ TimerScope::~TimerScope() {
 }
 
 static void release_buffers(Plan &pl) {
+    release_host_pipe(pl);  // first: its streams may still use the plan's buffers
     Alloc a[64];
     const size_t n = plan_allocs(pl, a);
     for (size_t k = 0; k < n; ++k)
@@ -355,6 +356,34 @@ prism_status prism_attn_bwd(prism_plan *plan, const void *O, const void *dO, voi
     const uintptr_t al = (uintptr_t)O | (uintptr_t)dO | (uintptr_t)dQ | (uintptr_t)dK | (uintptr_t)dV;
     if (al & 15) return fail(PRISM_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
     return launch_attn_bwd(plan->pl, O, dO, dQ, dK, dV, static_cast<cudaStream_t>(stream));
+}
+
+prism_status prism_step_host(prism_plan *plan, const prism_host_io *io, void *stream, unsigned long long *ticket) {
+    g_last_error.clear();
+    if (!plan || !io || !ticket) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_step_host");
+    if (!io->Q || !io->K || !io->V || !io->a_norm || !io->O)
+        return fail(PRISM_ERR_INVALID_ARG, "prism_step_host needs Q, K, V, a_norm and O");
+    if (io->dO && (!io->dQ || !io->dK || !io->dV))
+        return fail(PRISM_ERR_INVALID_ARG, "prism_step_host with dO needs dQ, dK and dV");
+    prism_status s = device_guard(plan->pl);
+    if (s != PRISM_OK) return s;
+    return host_step(plan->pl, *io, static_cast<cudaStream_t>(stream), ticket);
+}
+
+prism_status prism_step_join(prism_plan *plan, unsigned long long ticket, void *stream) {
+    g_last_error.clear();
+    if (!plan) return fail(PRISM_ERR_INVALID_ARG, "plan is NULL");
+    prism_status s = device_guard(plan->pl);
+    if (s != PRISM_OK) return s;
+    return host_step_join(plan->pl, ticket, static_cast<cudaStream_t>(stream));
+}
+
+prism_status prism_step_wait(prism_plan *plan, unsigned long long ticket) {
+    g_last_error.clear();
+    if (!plan) return fail(PRISM_ERR_INVALID_ARG, "plan is NULL");
+    prism_status s = device_guard(plan->pl);
+    if (s != PRISM_OK) return s;
+    return host_step_wait(plan->pl, ticket);
 }
 
 prism_status prism_plan_view_get(prism_plan *plan, prism_plan_view *view, void *stream) {

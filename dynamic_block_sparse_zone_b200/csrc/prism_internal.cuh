@@ -25,6 +25,7 @@ enum TimerId {
 static_assert(kTCount == PRISM_NUM_TIMERS, "timer count");
 
 struct TimerState;  // event pools, defined in prism_api.cu
+struct HostPipe;    // host-buffer step pipeline, defined in host_pipeline.cu
 
 // Per-launch problem geometry, passed by value to kernels.
 struct Geo {
@@ -77,6 +78,7 @@ struct Plan {
     int *status;            // device error word (0 = ok)
     int *host_nb;           // pinned host copy of nb
     TimerState *timers;     // NULL unless timing is on
+    HostPipe *pipe;         // NULL until the first host-buffer step
     // TMA descriptors of the permuted copies, viewed as [batch*heads*N][D] bf16
     CUtensorMap tmQ, tmK, tmV, tmdO;
     CUtensorMap tmdQ;       // fp32 [batch*heads*N][D], 64-row boxes, reduce-add target
@@ -109,6 +111,12 @@ prism_status make_tensor_maps(Plan &pl);
 prism_status launch_attn_bwd_tc_main(Plan &pl, void *dK, void *dV, cudaStream_t st);
 prism_status launch_attn_bwd(Plan &pl, const void *O, const void *dO, void *dQ, void *dK, void *dV,
                              cudaStream_t st);
+
+// Host-buffer steps (host_pipeline.cu).
+prism_status host_step(Plan &pl, const prism_host_io &io, cudaStream_t user, unsigned long long *ticket);
+prism_status host_step_join(Plan &pl, unsigned long long ticket, cudaStream_t st);
+prism_status host_step_wait(Plan &pl, unsigned long long ticket);
+void release_host_pipe(Plan &pl);
 
 __host__ __device__ inline int cap_for(int nb, int k, float max_frac) {
     if (!(max_frac > 0.0f)) return nb;

@@ -145,6 +145,47 @@ PRISM_API prism_status prism_attn_fwd(prism_plan *plan, void *O, float *lse, voi
 PRISM_API prism_status prism_attn_bwd(prism_plan *plan, const void *O, const void *dO, void *dQ, void *dK,
                             void *dV, void *stream);
 
+/* One layer step from HOST buffers: copy the inputs to the device, build the
+ * plan, run the forward and (when dO is given) the backward, and copy the
+ * outputs back -- the same computation as prism_plan_build + prism_attn_fwd
+ * + prism_attn_bwd on device tensors.  The pages define no such call; it is
+ * the runtime that feeds the hot path from host memory.
+ *
+ * Every field is a HOST pointer in the layouts above; the caller owns all of
+ * them.  Q, K, V, a_norm, O are required; lse may be NULL; dO == NULL means
+ * forward only, otherwise dQ, dK, dV are required.  Page-locked buffers
+ * (cudaHostAlloc / cudaHostRegister) let the copies run asynchronously;
+ * pageable ones work but their copies are not overlapped.
+ *
+ * prism_step_host only enqueues work and returns *ticket (1, 2, ...).  The
+ * plan runs steps on three streams of its own -- host->device copies into
+ * one of two device staging sets, the plan + attention kernels, and
+ * device->host copies -- so the copies of one step overlap the kernels of
+ * the next and the previous one.  The step's first copy waits for the work
+ * enqueued on `stream` before the call.  The caller must leave the input
+ * buffers unchanged, and must not read the output buffers, until the step has
+ * completed: prism_step_wait blocks the host until then; prism_step_join makes
+ * `stream` wait for it on the device.  At most 8 steps are in flight: the
+ * ninth call first waits on the host for the first one.  Staging buffers are
+ * allocated on the first step that needs them: two sets of the inputs and
+ * outputs used (2 x 9 bf16 tensors of batch*N*heads*head_dim at most) and
+ * freed with the plan.  Do not interleave host steps with the device-pointer
+ * calls on one plan without prism_step_wait in between: both use the plan's
+ * internal buffers.  PRISM_ERR_INVALID_ARG for a NULL required field or a
+ * ticket that was never issued.                                            */
+typedef struct prism_host_io {
+    const void *Q, *K, *V;  /* bf16, host                                     */
+    const float *a_norm;    /* fp32, host                                     */
+    const void *dO;         /* bf16, host; NULL = forward only                */
+    void *O;                /* bf16, host, written                            */
+    float *lse;             /* fp32, host, written; may be NULL               */
+    void *dQ, *dK, *dV;     /* bf16, host, written when dO != NULL            */
+} prism_host_io;
+PRISM_API prism_status prism_step_host(prism_plan *plan, const prism_host_io *io, void *stream,
+                                       unsigned long long *ticket);
+PRISM_API prism_status prism_step_join(prism_plan *plan, unsigned long long ticket, void *stream);
+PRISM_API prism_status prism_step_wait(prism_plan *plan, unsigned long long ticket);
+
 /* Synchronises `stream`, then fills *view (device pointers + host n_blocks).*/
 PRISM_API prism_status prism_plan_view_get(prism_plan *plan, prism_plan_view *view, void *stream);
 

@@ -82,3 +82,14 @@ def test_null_arguments_are_rejected(lib):
     assert lib.prism_attn_bwd(None, None, None, None, None, None, None) == 1
     assert b"NULL" in lib.prism_last_error()
     lib.prism_plan_destroy(None)  # no-op
+
+
+def test_host_step_arguments_are_checked_on_the_host(lib):
+    from dynamic_block_sparse_zone_b200.binding import prism_host_io
+    io = prism_host_io()
+    tk = ctypes.c_ulonglong()
+    assert lib.prism_step_host(None, ctypes.byref(io), None, ctypes.byref(tk)) == 1
+    assert lib.prism_step_host(None, None, None, None) == 1
+    assert lib.prism_step_join(None, 1, None) == 1
+    assert lib.prism_step_wait(None, 1) == 1
+    assert b"NULL" in lib.prism_last_error()

@@ -428,3 +428,55 @@ def test_plan_reuse_with_new_inputs():
     assert_close("O", O[0].float().cpu().numpy()[req_t, req_h], O_ref)
     dQ_ref = oracle.attn_bwd_dq_rows(pl, *bits2, bf16_bits(second.dO[0]), req_h[:128], req_t[:128])
     assert_close("dQ", dQ[0].float().cpu().numpy()[req_t[:128], req_h[:128]], dQ_ref)
+
+
+def test_host_steps_match_the_device_path():
+    """Pipelined steps from page-locked host buffers (prism_step_host) give the
+    outputs of prism_plan_build + prism_attn_fwd + prism_attn_bwd on device
+    tensors: forward outputs, lse, dK and dV bit for bit (same kernels, same
+    order), dQ up to the order of its fp32 reduce-adds.  Ten steps cycle the
+    two staging sets and wrap the ring of eight completion events."""
+    P = _lib()
+    w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=2, planted=2, backward=True)
+    inputs = [make_inputs(w, seed, with_grad_output=True) for seed in range(3)]
+    refs = []
+    plan = P.PrismPlan(P.params_for(w))
+    for inp in inputs:
+        Q, K, V, a, dO = (x.cuda() for x in (inp.Q, inp.K, inp.V, inp.a, inp.dO))
+        plan.build(Q, K, V, a)
+        O, lse = plan.fwd()
+        dQ, dK, dV = plan.bwd(O, dO)
+        refs.append([t.cpu() for t in (O, lse, dQ, dK, dV)])
+    torch.cuda.synchronize()
+    plan.check()
+
+    shp, lshp = inputs[0].Q.shape, refs[0][1].shape
+    pin = [[x.pin_memory() for x in (inp.Q, inp.K, inp.V, inp.a, inp.dO)] for inp in inputs]
+    outs, tickets = [], []
+    for step in range(10):
+        k = step % 3
+        bwd = step % 4 != 3  # some forward-only steps
+        O = torch.empty(shp, dtype=torch.bfloat16).pin_memory()
+        lse = torch.empty(lshp, dtype=torch.float32).pin_memory() if step % 2 == 0 else None
+        grads = [torch.empty(shp, dtype=torch.bfloat16).pin_memory() for _ in range(3)] if bwd else [None] * 3
+        Q, K, V, a, dO = pin[k]
+        tickets.append(plan.step_host(Q, K, V, a, O, lse=lse, dO=dO if bwd else None,
+                                      dQ=grads[0], dK=grads[1], dV=grads[2]))
+        outs.append((k, bwd, O, lse, grads))
+    assert tickets == list(range(1, 11))
+    plan.step_wait(tickets[-1])
+    plan.check()
+    for k, bwd, O, lse, (dQ, dK, dV) in outs:
+        rO, rl, rdQ, rdK, rdV = refs[k]
+        assert torch.equal(O, rO)
+        if lse is not None:
+            assert torch.equal(lse, rl)
+        if bwd:
+            assert torch.equal(dK, rdK) and torch.equal(dV, rdV)
+            assert torch.allclose(dQ.float(), rdQ.float(), rtol=1e-2, atol=1e-3)
+    with pytest.raises(P.PrismError):
+        plan.step_wait(11)
+    with pytest.raises(P.PrismError):
+        plan.step_wait(0)
+    plan.step_wait(1)  # long completed: fine
+    plan.close()
