@@ -34,7 +34,7 @@
 // owning one TMEM lane quadrant (32 key rows) and 16 query columns: many short
 // independent exp2 chains instead of a few long ones.
 // Warp roles (704 threads): warp 0 TMA producer (K, V once; Q, dO, LSE,
-// Delta per chunk into a three-stage ring; LSE is kept in log2 units), warp 1
+// Delta per chunk into a three-stage ring; LSE is kept negated, in log2 units), warp 1
 // MMA issuer, warps 2..17 softmax, warps 18..21 dQ drain (one head-dim row
 // each).
 #include <cuda.h>
@@ -64,7 +64,7 @@ struct Layout {
     static constexpr uint32_t kQ0 = kV + kHalves * kKVHalf;  // stage s: Q at kQ0 + s*kStage, dO at + kHalves*kQHalf
     static constexpr uint32_t kStage = 2 * kHalves * kQHalf;
     static constexpr uint32_t kDS = kQ0 + kStages * kStage;  // [2] x 128 key rows x 128 B (64 queries bf16)
-    static constexpr uint32_t kVec = kDS + 2 * 16384;        // stage s: LSE [64] f32 then Delta [64] f32
+    static constexpr uint32_t kVec = kDS + 2 * 16384;        // stage s: -LSE [64] f32 then Delta [64] f32
     static constexpr uint32_t kDQ = kVec + kStages * 512;    // dQ staging tile [64 queries][D] f32 (128-B aligned)
     static constexpr uint32_t kBars = kDQ + 64 * D * 4;
     // kv, q_full[3], q_empty[3], s_full[2], p_full[2], dq_full[3], dq_empty[3], done
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tmdQ, Geo g,
                   const int *__restrict__ nqt, const int *__restrict__ qt_row, const int *__restrict__ qt_blk,
                   const int *__restrict__ blk_off, const int *__restrict__ colT_ptr, const int *__restrict__ rowT,
-                  const int *__restrict__ perm, const float *__restrict__ lse_p, const float *__restrict__ delta,
+                  const int *__restrict__ perm, const float *__restrict__ nlse_p, const float *__restrict__ delta,
                   float *__restrict__ dQacc, __nv_bfloat16 *__restrict__ dK, __nv_bfloat16 *__restrict__ dV,
                   float scale, float scale_log2, int *__restrict__ status) {
     using L = Layout<D>;
@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(sQ + hf * L::kQHalf, &tmQ, bar, hf * 64, rowbase + r);
                     tma_load_2d(sO + hf * L::kQHalf, &tmdO, bar, hf * 64, rowbase + r);
                 }
-                bulk_load(sVec, lse_p + (size_t)rowbase + r, 256, bar);
+                bulk_load(sVec, nlse_p + (size_t)rowbase + r, 256, bar);
                 bulk_load(sVec + 256, delta + (size_t)rowbase + r, 256, bar);
                 issued = c + 1;
                 r += 64;
@@ -275,32 +275,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t sv[16], dv[16];
             tmem_ld16(tST, sv);
             tmem_ld16(tmem + kColDP + 16 * cg + lane_off, dv);
-            // LSE (log2 units) and Delta of the 16 queries: the same for every lane
+            // -LSE (log2 units) and Delta of the 16 queries: the same for every lane
             const uint32_t vec = sbase + L::kVec + st * 512 + cg * 64;
-            float4 L4[4], D4[4];
+            float4 N4[4], D4[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                L4[j] = lds_f4(vec + 16 * j);
+                N4[j] = lds_f4(vec + 16 * j);
                 D4[j] = lds_f4(vec + 256 + 16 * j);
             }
             tmem_wait_ld();
             uint32_t pd[16];  // P^T pairs then dS^T pairs
+            // key rows past the block (a 64-token key block fills half the tile) are
+            // a whole warp's rows, so the branch is warp-uniform
+            if (live) {
+                const uint64_t s2 = splat2(scale_log2);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int q = 4 * j;
-                float p0 = ex2(fmaf(__uint_as_float(sv[q]), scale_log2, -L4[j].x));
-                float p1 = ex2(fmaf(__uint_as_float(sv[q + 1]), scale_log2, -L4[j].y));
-                float p2 = ex2(fmaf(__uint_as_float(sv[q + 2]), scale_log2, -L4[j].z));
-                float p3 = ex2(fmaf(__uint_as_float(sv[q + 3]), scale_log2, -L4[j].w));
-                float d0 = p0 * (__uint_as_float(dv[q]) - D4[j].x);
-                float d1 = p1 * (__uint_as_float(dv[q + 1]) - D4[j].y);
-                float d2 = p2 * (__uint_as_float(dv[q + 2]) - D4[j].z);
-                float d3 = p3 * (__uint_as_float(dv[q + 3]) - D4[j].w);
-                if (!live) p0 = p1 = p2 = p3 = d0 = d1 = d2 = d3 = 0.f;
-                pd[2 * j] = pack_bf16x2(p0, p1);
-                pd[2 * j + 1] = pack_bf16x2(p2, p3);
-                pd[8 + 2 * j] = pack_bf16x2(d0, d1);
-                pd[8 + 2 * j + 1] = pack_bf16x2(d2, d3);
+                for (int j = 0; j < 4; ++j) {
+                    const int q = 4 * j;
+                    float x0, x1, x2, x3, d0, d1, d2, d3;
+                    fma2(__uint_as_float(sv[q]), __uint_as_float(sv[q + 1]), s2, pair2(N4[j].x, N4[j].y), x0, x1);
+                    fma2(__uint_as_float(sv[q + 2]), __uint_as_float(sv[q + 3]), s2, pair2(N4[j].z, N4[j].w), x2, x3);
+                    const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+                    // dS = P (dP - Delta), two lanes per instruction
+                    mul_sub2(p0, p1, __uint_as_float(dv[q]), __uint_as_float(dv[q + 1]), D4[j].x, D4[j].y, d0, d1);
+                    mul_sub2(p2, p3, __uint_as_float(dv[q + 2]), __uint_as_float(dv[q + 3]), D4[j].z, D4[j].w, d2, d3);
+                    pd[2 * j] = pack_bf16x2(p0, p1);
+                    pd[2 * j + 1] = pack_bf16x2(p2, p3);
+                    pd[8 + 2 * j] = pack_bf16x2(d0, d1);
+                    pd[8 + 2 * j + 1] = pack_bf16x2(d2, d3);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) pd[e] = 0u;
             }
             // P^T over columns [16 cg, 16 cg + 8), dS^T over [16 cg + 8, 16 cg + 16): this warp's own S^T columns
             tmem_st16(tST, pd);
@@ -417,7 +423,7 @@ static prism_status bwd_tc_main(Plan &pl, void *dK, void *dV, cudaStream_t st) {
     TimerScope ts(pl, kTAttnBwd, st);
     bwdtc::k_attn_bwd_tc<D><<<dim3(g.nbmax, g.batch * g.heads), bwdtc::kThreads, bwdtc::Layout<D>::kAlloc, st>>>(
         pl.tmQ, pl.tmK, pl.tmV, pl.tmdO, pl.tmdQ, g, pl.nqt, pl.qt_row, pl.qt_blk, pl.blk_off, pl.colT_ptr, pl.rowT,
-        pl.perm, pl.lse_p, pl.delta, pl.dQacc, static_cast<__nv_bfloat16 *>(dK), static_cast<__nv_bfloat16 *>(dV),
+        pl.perm, pl.nlse_p, pl.delta, pl.dQacc, static_cast<__nv_bfloat16 *>(dK), static_cast<__nv_bfloat16 *>(dV),
         (float)scale, (float)(scale * 1.4426950408889634), pl.status);
     PRISM_CUDA_OK(cudaGetLastError());
     return PRISM_OK;

@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                   const __grid_constant__ CUtensorMap tmV, Geo g, const int *__restrict__ nqt,
                   const int *__restrict__ qt_row, const int *__restrict__ qt_blk, const int *__restrict__ blk_off,
                   const int *__restrict__ row_ptr, const int *__restrict__ col, const int *__restrict__ perm,
-                  __nv_bfloat16 *__restrict__ O, float *__restrict__ lse_user, float *__restrict__ lse_p,
+                  __nv_bfloat16 *__restrict__ O, float *__restrict__ lse_user, float *__restrict__ nlse_p,
                   float scale_log2, int *__restrict__ status) {
     using L = Layout<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -221,14 +221,21 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int q = 0; q < 4; ++q)
                 if (q < nq) tmem_ld32(tSr + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * q]));
             tmem_wait_ld();
-            // pass 1: row max
-            float mx = -INFINITY;
+            // pass 1: row max (three-input max, four independent chains)
+            float mxa = -INFINITY, mxb = -INFINITY, mxc = -INFINITY, mxd = -INFINITY;
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 if (q < nq) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[32 * q + e]));
+                    for (int e = 0; e < 32; e += 8) {
+                        const float *v = reinterpret_cast<const float *>(&sr[32 * q + e]);
+                        mxa = fmax3(mxa, v[0], v[1]);
+                        mxb = fmax3(mxb, v[2], v[3]);
+                        mxc = fmax3(mxc, v[4], v[5]);
+                        mxd = fmax3(mxd, v[6], v[7]);
+                    }
                 }
+            const float mx = fmaxf(fmaxf(mxa, mxb), fmaxf(mxc, mxd));
             const float mx2 = mx * scale_log2;
             const bool need = (c > 0) && (mx2 > m + kRescaleThreshold);
             if (c == 0) m = mx2;
@@ -252,20 +259,25 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             // pass 2: P = exp2(S*scale*log2e - m), bf16 pairs written over S
             // (group q packs into columns [16q, 16q+16); all of S is in registers).
-            float sum = 0.f;
+            // (scale, -m) and the running sum as packed fp32 pairs
+            const uint64_t s2 = splat2(scale_log2), c2 = splat2(-m);
+            uint64_t acc2 = 0;
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 if (q < nq) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2(fmaf(__uint_as_float(sr[32 * q + 2 * e]), scale_log2, -m));
-                        const float p1 = ex2(fmaf(__uint_as_float(sr[32 * q + 2 * e + 1]), scale_log2, -m));
-                        sum += p0 + p1;
+                        float x0, x1;
+                        fma2(__uint_as_float(sr[32 * q + 2 * e]), __uint_as_float(sr[32 * q + 2 * e + 1]), s2, c2, x0,
+                             x1);
+                        const float p0 = ex2(x0), p1 = ex2(x1);
+                        add2(acc2, p0, p1);
                         pk[e] = pack_bf16x2(p0, p1);
                     }
                     tmem_st16(tSr + q * 16, pk);
                 }
+            const float sum = sum2(acc2);
             l += sum;
             tmem_wait_st();
             tc_fence_before();
@@ -297,8 +309,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
             }
             if (write) {
-                const float lse2 = m + __log2f(l);  // log2 units, as the backward consumes it
-                lse_p[(size_t)bh * g.N + n] = lse2;
+                const float lse2 = m + __log2f(l);
+                nlse_p[(size_t)bh * g.N + n] = -lse2;  // negated, log2 units: the backward's exp2 addend
                 if (lse_user) lse_user[(size_t)bh * g.N + tok] = lse2 * 0.69314718055994531f;
             }
         }
@@ -401,7 +413,7 @@ static prism_status fwd_tc_impl(Plan &pl, void *O, float *lse, cudaStream_t st) 
     TimerScope ts(pl, kTAttnFwd, st);
     fwdtc::k_attn_fwd_tc<D><<<dim3(g.nbmax, g.batch * g.heads), fwdtc::kThreads, fwdtc::Layout<D>::kAlloc, st>>>(
         pl.tmQ, pl.tmK, pl.tmV, g, pl.nqt, pl.qt_row, pl.qt_blk, pl.blk_off, pl.row_ptr, pl.col, pl.perm,
-        static_cast<__nv_bfloat16 *>(O), lse, pl.lse_p, scale_log2, pl.status);
+        static_cast<__nv_bfloat16 *>(O), lse, pl.nlse_p, scale_log2, pl.status);
     PRISM_CUDA_OK(cudaGetLastError());
     return PRISM_OK;
 }

@@ -146,7 +146,7 @@ static size_t plan_allocs(Plan &pl, Alloc *out) {
     add((void **)&pl.rowT, nnz * sizeof(int));
     add((void **)&pl.colT_cursor, rows * sizeof(int));
     add((void **)&pl.scan_tmp, ((rows + 1023) / 1024 + 1) * sizeof(int));
-    add((void **)&pl.lse_p, BH * g.N * sizeof(float));
+    add((void **)&pl.nlse_p, BH * g.N * sizeof(float));
     add((void **)&pl.dOp, BH * g.N * g.D * 2);
     add((void **)&pl.delta, BH * g.N * sizeof(float));
     add((void **)&pl.dQacc, BH * g.N * g.D * sizeof(float));

@@ -71,7 +71,7 @@ struct Plan {
     int *colT_cursor;       // [rows]
     int *scan_tmp;          // block partial sums for scans
     // attention statistics / backward scratch
-    float *lse_p;           // [batch*heads][N] log2-unit LSE of the scaled scores, permuted order
+    float *nlse_p;          // [batch*heads][N] minus the log2-unit LSE of the scaled scores, permuted order
     __nv_bfloat16 *dOp;     // [batch*heads][N][D]
     float *delta;           // [batch*heads][N]
     float *dQacc;           // [batch*heads][N][D]

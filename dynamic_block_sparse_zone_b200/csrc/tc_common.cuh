@@ -274,6 +274,41 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction for two lanes,
+// where the softmax loops are instruction-issue bound.  (y0, y1) = (x0, x1) * s2 + c2.
+__device__ __forceinline__ void fma2(float x0, float x1, uint64_t s2, uint64_t c2, float &y0, float &y1) {
+    asm("{\n\t.reg .b64 x, y;\n\tmov.b64 x, {%2, %3};\n\tfma.rn.f32x2 y, x, %4, %5;\n\tmov.b64 {%0, %1}, y;\n\t}\n"
+        : "=f"(y0), "=f"(y1)
+        : "f"(x0), "f"(x1), "l"(s2), "l"(c2));
+}
+// (d0, d1) = (p0, p1) * ((a0, a1) - (b0, b1)), each step rounded as in scalar code
+__device__ __forceinline__ void mul_sub2(float p0, float p1, float a0, float a1, float b0, float b1, float &d0,
+                                         float &d1) {
+    asm("{\n\t.reg .b64 p, a, b, t;\n\tmov.b64 p, {%2, %3};\n\tmov.b64 a, {%4, %5};\n\tmov.b64 b, {%6, %7};\n\t"
+        "sub.rn.f32x2 t, a, b;\n\tmul.rn.f32x2 t, p, t;\n\tmov.b64 {%0, %1}, t;\n\t}\n"
+        : "=f"(d0), "=f"(d1)
+        : "f"(p0), "f"(p1), "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ uint64_t pair2(float lo, float hi) {
+    return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+// acc2 += (p0, p1)
+__device__ __forceinline__ void add2(uint64_t &acc2, float p0, float p1) {
+    asm("{\n\t.reg .b64 p;\n\tmov.b64 p, {%1, %2};\n\tadd.rn.f32x2 %0, %0, p;\n\t}\n" : "+l"(acc2) : "f"(p0), "f"(p1));
+}
+__device__ __forceinline__ uint64_t splat2(float v) {
+    return (uint64_t)__float_as_uint(v) | ((uint64_t)__float_as_uint(v) << 32);
+}
+__device__ __forceinline__ float sum2(uint64_t acc2) {
+    return __uint_as_float((uint32_t)acc2) + __uint_as_float((uint32_t)(acc2 >> 32));
+}
+// max of three
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
