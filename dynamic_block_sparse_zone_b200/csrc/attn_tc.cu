@@ -19,7 +19,9 @@
 //   warp 1       MMA issuer (whole warp, one elected lane issues).
 //   warps 2..5   softmax, one query row per thread (= TMEM lane): the S row
 //                comes into registers in one TMEM round trip; pass 1 row
-//                max, pass 2 exp2 / running sum / bf16 P written back over S.
+//                max, pass 2 exp2 / running sum / bf16 P written back over S;
+//                P of the first 64 keys is published as soon as it is stored,
+//                so the first half of P V overlaps the rest of the softmax.
 //                O is rescaled in TMEM only when the running max grows by more
 //                than 2^8 (it is current then: S_c was issued after PV_{c-1}).
 //                Epilogue: O / l to the user layout, log-sum-exp.
@@ -47,7 +49,7 @@ struct Layout {
     static constexpr uint32_t kV = kK + kHalves * kTileBytes;
     static constexpr uint32_t kBars = kV + kHalves * kTileBytes;
     // barriers: q, k_full, k_empty, v_full, v_empty, s, p, o  (8 B each) + tmem slot + abort
-    static constexpr uint32_t kNumBars = 8;
+    static constexpr uint32_t kNumBars = 9;
     static constexpr uint32_t kBytes = kBars + kNumBars * 8 + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;  // slack to align the base to 1024
 };
@@ -92,6 +94,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t bar_q = sbase + L::kBars;
     const uint32_t bar_kf = bar_q + 8, bar_ke = bar_q + 16, bar_vf = bar_q + 24, bar_ve = bar_q + 32;
     const uint32_t bar_s = bar_q + 40, bar_p = bar_q + 48, bar_o = bar_q + 56;
+    const uint32_t bar_p2 = bar_q + 64;  // P of keys 64..127 (bar_p: keys 0..63)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBars + L::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kBars + L::kNumBars * 8 + 8);
 
@@ -104,6 +107,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_init(bar_ve, 1);
             mbar_init(bar_s, 1);
             mbar_init(bar_p, 128);
+            mbar_init(bar_p2, 128);
             mbar_init(bar_o, 1);
             *abort_flag = 0;
             mbar_fence_init();
@@ -189,15 +193,17 @@ __global__ void __launch_bounds__(kThreads, 2)
                     mma_ss4<2, 4, 6, 2, 4, 6>(tS, aQ, bK, full ? idS128 : idS64, 0u);
                 mma_commit(bar_s);
                 mma_commit(bar_ke);
+                // P V in two halves: keys 0..63 as soon as the softmax has stored their P
+                // (it goes on with keys 64..127 meanwhile), then keys 64..127
                 if (!__all_sync(0xffffffffu, mbar_wait(bar_p, c & 1, status, kSiteP, abort_flag))) break;
                 if (!__all_sync(0xffffffffu, mbar_wait(bar_vf, c & 1, status, kSiteV, abort_flag))) break;
                 tc_fence_after();
-                // k-step kk (16 keys): P columns 8 kk, V rows 2048 B further
+                // k-step kk (16 keys): P columns 8 kk, V rows 2048 B (128 descriptor units) further
                 const uint64_t bV = sdesc(sbase + L::kV, L::kTileBytes, 1024);
-                if (full)
-                    mma_ts8<8, 16, 24, 32, 40, 48, 56, 128, 256, 384, 512, 640, 768, 896>(tO, tS, bV, idPV, c > 0);
-                else
-                    mma_ts4<8, 16, 24, 128, 256, 384>(tO, tS, bV, idPV, c > 0);
+                mma_ts4<8, 16, 24, 128, 256, 384>(tO, tS, bV, idPV, c > 0);
+                if (!__all_sync(0xffffffffu, mbar_wait(bar_p2, c & 1, status, kSiteP, abort_flag))) break;
+                tc_fence_after();
+                if (full) mma_ts4<8, 16, 24, 128, 256, 384>(tO, tS + 32, bV + 512, idPV, 1u);
                 mma_commit(bar_ve);
                 mma_commit(bar_o);
             }
@@ -276,12 +282,17 @@ __global__ void __launch_bounds__(kThreads, 2)
                         pk[e] = pack_bf16x2(p0, p1);
                     }
                     tmem_st16(tSr + q * 16, pk);
+                    if (q == 1) {  // P of keys 0..63 is in TMEM: the first half of P V may start
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(bar_p);
+                    }
                 }
             const float sum = sum2(acc2);
             l += sum;
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar_p);
+            mbar_arrive(bar_p2);
         }
         // epilogue: the last product P V must have landed
         if (ok && nchunk > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (nchunk - 1) & 1, status, kSiteO, abort_flag));
