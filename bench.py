@@ -148,6 +148,9 @@ def aggregate_value(flops_per_step: float, steps: int, world: int, ms_max: float
     return flops_per_step * steps * world / (ms_max * 1e-3) / 1e12
 
 
+L2_BYTES = 128 << 20  # B200 L2: 126 MB
+
+
 def steps_or_1(args):
     return max(args.steps, 1)
 
@@ -196,25 +199,71 @@ def run_ours(args, rank, world, dev):
 
 
     # ---- device-resident timed region ----
-    plan.set_timing(True)
-    plan.read_timing()
-    clocks = ClockSampler(torch.cuda.current_device())
+    # Inputs larger than L2 stream from HBM every step; smaller ones would stay
+    # in L2 between steps, so then L2 is flushed (a 256 MB write) before each
+    # step and the steps are timed one by one, the flush outside the events.
+    in_bytes = sum(x.numel() * x.element_size() for x in (inp.Q, inp.K, inp.V, inp.a)) + (
+        0 if args.fwd_only else inp.dO.numel() * inp.dO.element_size())
+    flush = None if in_bytes > L2_BYTES else torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    l2_note = (f"inputs larger than L2 ({in_bytes / 1e9:.2f} GB per step vs 126 MB)" if flush is None else
+               f"L2 flushed (256 MB write) before each timed step, steps timed one by one (inputs {in_bytes / 1e6:.1f} MB)")
     stream = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    e0.record(stream)
-    for _ in range(args.steps):
-        step(inp.Q, inp.K, inp.V, inp.a, inp.dO)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    clk = clocks.stop()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+
+    def timed(run):
+        """Device time of args.steps calls of run(), max over ranks, with clocks sampled."""
+        clocks = ClockSampler(torch.cuda.current_device())
+        barrier()
+        torch.cuda.synchronize()
+        clocks.start()
+        if flush is None:
+            e0.record(stream)
+            for _ in range(args.steps):
+                run()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            total = e0.elapsed_time(e1)
+        else:
+            pairs = []
+            for _ in range(args.steps):
+                flush.fill_(1)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                run()
+                b.record(stream)
+                pairs.append((a, b))
+            torch.cuda.synchronize()
+            total = sum(a.elapsed_time(b) for a, b in pairs)
+        barrier()
+        return max_over_ranks(total, world, dev), clocks.stop()
+
+    plan.set_timing(True)
+    plan.read_timing()
+    ms, clk = timed(lambda: step(inp.Q, inp.K, inp.V, inp.a, inp.dO))
     timing = plan.read_timing()
     plan.set_timing(False)
     plan.check()
+
+    # ---- the same step captured once in a CUDA graph and replayed ----
+    # (the per-kernel times above come from the eager loop: event timers do
+    # not run inside a graph; the kernels are the same)
+    launch = "eager"
+    if args.graph:
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step(inp.Q, inp.K, inp.V, inp.a, inp.dO)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step(inp.Q, inp.K, inp.V, inp.a, inp.dO)
+        for _ in range(args.warmup):
+            graph.replay()
+        ms, clk = timed(graph.replay)
+        plan.check()
+        del graph
+        launch = "cuda graph (one step captured, replayed)"
 
     # ---- end to end through the C ABI with page-locked host buffers ----
     # prism_step_host: every step copies its inputs host->device, runs the
@@ -307,7 +356,7 @@ def run_ours(args, rank, world, dev):
                    "grid": [w.T, w.H, w.W], "tokens": w.N, "heads": w.heads,
                    "head_dim": w.head_dim, "top_k": w.top_k, "top_p": w.top_p, "max_frac": w.max_frac,
                    "n_blocks": nb, "selected_token_pairs": pairs, "flops_per_step": flops_step,
-                   "l2": "inputs larger than L2 (Q,K,V,dO 2.26 GB each)", "parallelism": f"replicas x{world}"},
+                   "l2": l2_note, "launch": launch, "parallelism": f"replicas x{world}"},
         "kernels": kernels,
         "roofline": roof,
         "gpu_launches": launches_per_step * args.steps,
@@ -430,6 +479,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--fwd-only", action="store_true", help="step = plan + forward (forward-only workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true", help="time replays of the step captured in a CUDA graph")
     ap.add_argument("--heads", type=int, default=0, help="override the workload's head count (profiling)")
     ap.add_argument("--cpu-rows", type=int, default=6000)
     ap.add_argument("--ref-rows", type=int, default=1500)
