@@ -22,17 +22,17 @@
 //   drain warps: dQ^T rows (lane = head-dim index) -> a [64 x D] fp32 tile in
 //                shared memory -> one TMA reduce-add into the dQ accumulator
 // Three ST buffers let S^T of chunk c+2 be issued while chunk c's dQ^T waits
-// to be drained; the single DP buffer is refilled (dP^T of chunk c+1) as soon
-// as the softmax of chunk c has read it.
+// to be drained; the single DP buffer is refilled (dP^T of chunk c+1) once the
+// softmax of chunk c has published its P^T / dS^T.
 // TMEM columns: dK [0,128), dV [128,256), ST[3] [256,448), DP [448,512).
 // In an ST buffer, after the softmax, columns [16g, 16g+8) hold P^T and
 // [16g+8, 16g+16) hold dS^T of queries [16g, 16g+16) (g = 0..3), packed as
 // bf16 pairs.
 //
-// The softmax is the loop's critical path (dP^T of chunk c+1 waits for it,
-// and the softmax of c+1 waits for that), so it is spread over 16 warps, each
-// owning one TMEM lane quadrant (32 key rows) and 16 query columns: many short
-// independent exp2 chains instead of a few long ones.
+// dP^T of chunk c+1 waits for the softmax of chunk c, and the softmax of c+1
+// for that dP^T, so the softmax is spread over 16 warps, each owning one TMEM
+// lane quadrant (32 key rows) and 16 query columns, and does its arithmetic in
+// packed fp32 pairs.
 // Warp roles (704 threads): warp 0 TMA producer (K, V once; Q, dO, LSE,
 // Delta per chunk into a three-stage ring; LSE is kept negated, in log2 units), warp 1
 // MMA issuer, warps 2..17 softmax, warps 18..21 dQ drain (one head-dim row
