@@ -67,6 +67,7 @@ def _load():
                                             _I, _I, _P, _P, _P]),
             "orc_attn_bwd_dkv_rows": (None, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P,
                                              _I, _I, _P, _P, _P, _P]),
+            "orc_audio_norms": (None, [_P, _P, ctypes.c_longlong, _I]),
             "orc_num_threads": (_I, []),
         }
         for name, (res, args) in sigs.items():
@@ -251,6 +252,17 @@ def plan(Q_bits, K_bits, V_bits, a, T, H, W, heads, D, k, p, max_frac=0.0,
     return OraclePlan(T, H, W, heads, D, sv, sa, am, amax, dec["g"], dec["rho"], dec["lstar"],
                       dec["zone_B"], dec["zone_shape"], dec["gap_shape"], dec["gap_rho"], box, pm,
                       Qb, Kb, cnt, cols, diag)
+
+
+def audio_norms(h_bits: np.ndarray) -> np.ndarray:
+    """a_{t,h,w} = ||h^_{t,h,w}||_2 over the last axis of bf16 bits h_bits [..., C]
+    (fp64, channel order) [Prism guide, Method section 1]."""
+    C = h_bits.shape[-1]
+    hb = _c(h_bits.reshape(-1, C), np.uint16)
+    out = np.empty(hb.shape[0], np.float64)
+    lib = _load()
+    lib.orc_audio_norms(_ptr(hb), _ptr(out), ctypes.c_longlong(hb.shape[0]), _I(C))
+    return out.reshape(h_bits.shape[:-1])
 
 
 # --------------------------------------------------------------------------

@@ -42,6 +42,10 @@
  *   orc_attn_*                                     pinned (dense reduction vs
  *                                                  library SDPA, masked dense,
  *                                                  finite differences)
+ *   orc_audio_norms                                pinned (closed forms: constant
+ *                                                  rows, one-hot rows, integer
+ *                                                  norms; an exact rational sum
+ *                                                  on random rows)
  */
 #include <math.h>
 #include <stdint.h>
@@ -728,4 +732,24 @@ int orc_num_threads(void)
 #else
     return 1;
 #endif
+}
+
+/* ------------------------------------------------------------------------ */
+/* Audio guidance a_{t,h,w} = || h^_{t,h,w} ||_2 [Prism guide, Method section
+ * 1, the sentence before the g_d equation]: the L2 norm, over the channels,
+ * of the audio-to-video cross-attention output of each video token, which the
+ * layer caches for the next layer's plan.  h is [rows][C] bf16 bits, a is
+ * [rows] (rows = batch * T * H * W in raster order).  The squares are summed
+ * in channel order.                                                        */
+void orc_audio_norms(const uint16_t *h, double *a, long long rows, int C)
+{
+#pragma omp parallel for schedule(static)
+    for (long long r = 0; r < rows; ++r) {
+        double s = 0.0;
+        for (int c = 0; c < C; ++c) {
+            const double x = widen_bf16(h[r * (long long)C + c]);
+            s += x * x;
+        }
+        a[r] = sqrt(s);
+    }
 }

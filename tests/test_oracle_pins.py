@@ -407,3 +407,39 @@ def test_planted_zones_raise_directional_variation():
     others = [m for m in range(w.zones) if m not in planted]
     for z, ax in planted.items():
         assert sv[z, ax] >= 4.0 * np.median(sv[others, ax])
+
+
+def test_audio_norms_closed_forms_and_exact_sums():
+    """a_{t,h,w} = ||h^_{t,h,w}||_2 [Prism guide, Method section 1]: closed forms
+    (constant rows, one-hot rows, rows with integer norms) and, on random bf16
+    rows, the exact rational sum of squares with a 50-digit square root."""
+    from decimal import Decimal, getcontext
+    from fractions import Fraction
+    C = 3072
+    rows = [np.full(C, 0.75, np.float32), np.full(C, -1.5, np.float32)]
+    onehot = np.zeros(C, np.float32)
+    onehot[1234] = -2.25
+    rows.append(onehot)
+    for trip, n in (((3, 4), 5), ((2, 3, 6), 7), ((1, 4, 8), 9), ((2, 6, 9), 11)):
+        r = np.zeros(C, np.float32)
+        r[[5, 700, 3000][:len(trip)]] = trip
+        rows.append(r)
+    h = f32_bits(np.stack(rows))
+    a = oracle.audio_norms(h)
+    assert a[0] == pytest.approx(0.75 * math.sqrt(C), rel=1e-15)
+    assert a[1] == pytest.approx(1.5 * math.sqrt(C), rel=1e-15)
+    assert a[2] == 2.25
+    assert list(a[3:]) == [5.0, 7.0, 9.0, 11.0]
+
+    getcontext().prec = 50
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal((6, 257)) * rng.uniform(0.01, 30, (6, 1))).astype(np.float32)
+    hb = f32_bits(x)
+    a = oracle.audio_norms(hb)
+    vals = torch.from_numpy(hb.view(np.int16)).view(torch.bfloat16).float().numpy().astype(np.float64)
+    for r in range(vals.shape[0]):
+        s = sum(Fraction(float(v)) ** 2 for v in vals[r])  # bf16 values are exact dyadic rationals
+        exact = (Decimal(s.numerator) / Decimal(s.denominator)).sqrt()
+        assert abs(Decimal(a[r]) - exact) / exact < Decimal("1e-14")
+    # the batch and grid axes are kept
+    assert oracle.audio_norms(hb.reshape(2, 3, 257)).shape == (2, 3)
