@@ -25,7 +25,7 @@ EXPORTED = ("prism_plan_create", "prism_plan_bytes", "prism_plan_build", "prism_
             "prism_plan_view_get", "prism_plan_check", "prism_plan_destroy", "prism_last_error",
             "prism_plan_set_timing", "prism_plan_read_timing", "prism_timer_name", "prism_zone_shapes_noalloc",
             "prism_plan_selftest_timeout", "prism_plan_update_qkv", "prism_step_host", "prism_step_join",
-            "prism_step_wait")
+            "prism_step_wait", "prism_audio_norms")
 NUM_TIMERS = 10
 
 
@@ -82,6 +82,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.prism_step_join.restype = ctypes.c_int
     lib.prism_step_wait.argtypes = [V, ctypes.c_ulonglong]
     lib.prism_step_wait.restype = ctypes.c_int
+    lib.prism_audio_norms.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
+    lib.prism_audio_norms.restype = ctypes.c_int
     lib.prism_plan_destroy.argtypes = [V]
     lib.prism_plan_destroy.restype = None
     lib.prism_last_error.restype = ctypes.c_char_p
@@ -317,6 +319,20 @@ def prism_zone_shapes_noalloc(params: Params, V: torch.Tensor, a_norm: torch.Ten
 
 
 # Module-level names that mirror the C ABI.
+def prism_audio_norms(h: torch.Tensor, T: int, H: int, W: int, a: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """a_{t,h,w} = ||h^_{t,h,w}||_2 for h [batch, T*H*W, channels] bf16 on the current device."""
+    if h.dtype != torch.bfloat16 or not h.is_cuda or h.dim() != 3 or not h.is_contiguous():
+        raise ValueError("h must be a contiguous [batch, N, channels] bf16 CUDA tensor")
+    batch, n, ch = h.shape
+    if n != T * H * W:
+        raise ValueError("h's token axis must be T*H*W")
+    if a is None:
+        a = torch.empty((batch, T, H, W), dtype=torch.float32, device=h.device)
+    _need(a, "a", torch.float32, (batch, T, H, W))
+    _check(load_library().prism_audio_norms(_ptr(h), _ptr(a), batch, T, H, W, ch, _stream()))
+    return a
+
+
 def prism_plan_create(params: Params) -> PrismPlan:
     return PrismPlan(params)
 

@@ -358,6 +358,14 @@ prism_status prism_attn_bwd(prism_plan *plan, const void *O, const void *dO, voi
     return launch_attn_bwd(plan->pl, O, dO, dQ, dK, dV, static_cast<cudaStream_t>(stream));
 }
 
+prism_status prism_audio_norms(const void *h, float *a, int batch, int T, int H, int W, int channels, void *stream) {
+    g_last_error.clear();
+    if (!h || !a) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_audio_norms");
+    if (batch < 1 || T < 1 || H < 1 || W < 1) return fail(PRISM_ERR_INVALID_ARG, "batch, T, H, W must be >= 1");
+    if (channels < 1 || channels > (1 << 20)) return fail(PRISM_ERR_INVALID_ARG, "channels must be in [1, 2^20]");
+    return launch_audio_norms(h, a, (long long)batch * T * H * W, channels, static_cast<cudaStream_t>(stream));
+}
+
 prism_status prism_step_host(prism_plan *plan, const prism_host_io *io, void *stream, unsigned long long *ticket) {
     g_last_error.clear();
     if (!plan || !io || !ticket) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_step_host");

@@ -112,6 +112,8 @@ prism_status launch_attn_bwd_tc_main(Plan &pl, void *dK, void *dV, cudaStream_t 
 prism_status launch_attn_bwd(Plan &pl, const void *O, const void *dO, void *dQ, void *dK, void *dV,
                              cudaStream_t st);
 
+prism_status launch_audio_norms(const void *h, float *a, long long rows, int C, cudaStream_t st);
+
 // Host-buffer steps (host_pipeline.cu).
 prism_status host_step(Plan &pl, const prism_host_io &io, cudaStream_t user, unsigned long long *ticket);
 prism_status host_step_join(Plan &pl, unsigned long long ticket, cudaStream_t st);

@@ -145,6 +145,19 @@ PRISM_API prism_status prism_attn_fwd(prism_plan *plan, void *O, float *lse, voi
 PRISM_API prism_status prism_attn_bwd(prism_plan *plan, const void *O, const void *dO, void *dQ, void *dK,
                             void *dV, void *stream);
 
+/* Audio guidance for the plan: a[b][t][h][w] = || h^[b][n][:] ||_2, the L2
+ * norm over `channels` of the audio-to-video cross-attention output of video
+ * token n = (t*H + h)*W + w [Prism guide, Method section 1, the sentence
+ * before the g_d equation]; a layer computes it after its cross-attention and
+ * the next layer's prism_plan_build takes it as a_norm.  h: device, bf16
+ * [batch][T*H*W][channels], read only; a: device, fp32 [batch][T][H][W],
+ * written.  The caller owns both.  Sums of squares in fp32 (relative error
+ * of a below 1e-5 for channels <= 65536).  Enqueues one kernel on `stream`
+ * on the current device; no plan is needed.  PRISM_ERR_INVALID_ARG for NULL
+ * pointers, dimensions < 1 or channels outside [1, 2^20].                  */
+PRISM_API prism_status prism_audio_norms(const void *h, float *a, int batch, int T, int H, int W, int channels,
+                                         void *stream);
+
 /* One layer step from HOST buffers: copy the inputs to the device, build the
  * plan, run the forward and (when dO is given) the backward, and copy the
  * outputs back -- the same computation as prism_plan_build + prism_attn_fwd

@@ -84,6 +84,14 @@ def test_null_arguments_are_rejected(lib):
     lib.prism_plan_destroy(None)  # no-op
 
 
+def test_audio_norm_arguments_are_checked_on_the_host(lib):
+    assert lib.prism_audio_norms(None, None, 1, 8, 8, 8, 16, None) == 1
+    dummy = ctypes.c_void_p(16)  # never dereferenced: the sizes are rejected first
+    assert lib.prism_audio_norms(dummy, dummy, 0, 8, 8, 8, 16, None) == 1
+    assert lib.prism_audio_norms(dummy, dummy, 1, 8, 8, 8, 0, None) == 1
+    assert b"channels" in lib.prism_last_error()
+
+
 def test_host_step_arguments_are_checked_on_the_host(lib):
     from dynamic_block_sparse_zone_b200.binding import prism_host_io
     io = prism_host_io()

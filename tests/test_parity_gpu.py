@@ -530,3 +530,52 @@ def test_cuda_graph_capture_of_a_training_step():
     del graph
     plan.close()
     ref.close()
+
+
+def _audio_h(batch, N, C, seed):
+    """Synthetic cross-attention outputs: random directions with per-token scales."""
+    g = torch.Generator().manual_seed(seed)
+    dirs = torch.randn(batch, N, C, generator=g)
+    scale = torch.rand(batch, N, 1, generator=g) * 3.0 + 0.01
+    return (dirs * scale).to(torch.bfloat16)
+
+
+def test_audio_norms_against_the_oracle():
+    """prism_audio_norms vs the fp64 oracle: the 16-byte path (C = 3072), the
+    scalar path (C = 100, and C = 3072 from a misaligned base); relative
+    error <= 1e-5 (fp32 sums of exact squares)."""
+    from dynamic_block_sparse_zone_b200 import binding as B
+    _lib()
+    T, H, W = 8, 16, 32
+    for C, misalign in ((3072, False), (100, False), (3072, True)):
+        h = _audio_h(2, T * H * W, C, seed=C)
+        if misalign:
+            buf = torch.empty(h.numel() + 1, dtype=torch.bfloat16, device="cuda")
+            hd = buf[1:].view(h.shape)
+            hd.copy_(h.cuda())
+            assert hd.data_ptr() % 16 != 0
+        else:
+            hd = h.cuda()
+        a = B.prism_audio_norms(hd, T, H, W).cpu().numpy().astype(np.float64)
+        ref = oracle.audio_norms(bf16_bits(h)).reshape(2, T, H, W)
+        assert np.max(np.abs(a / ref - 1)) <= 1e-5, (C, misalign)
+
+
+def test_audio_norms_feed_the_plan():
+    """The producer's a drives prism_plan_build: the plan built on the GPU from
+    the kernel's a equals the oracle's plan from the same a."""
+    from dynamic_block_sparse_zone_b200 import binding as B
+    P = _lib()
+    w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=2, planted=2)
+    inp = make_inputs(w, 0)
+    # cross-attention outputs whose norms follow the workload's planted audio field
+    C = 3072
+    g = torch.Generator().manual_seed(7)
+    dirs = torch.randn(1, w.N, C, generator=g)
+    dirs = dirs / dirs.norm(dim=-1, keepdim=True)
+    h = (dirs * inp.a.reshape(1, w.N, 1)).to(torch.bfloat16)
+    a = B.prism_audio_norms(h.cuda(), w.T, w.H, w.W)
+    inp.a = a.cpu()
+    g_out = run_gpu(w, inp)
+    pl, _ = oracle_plan(w, inp)
+    compare_plan(w, pl, g_out["view"])
