@@ -25,7 +25,8 @@ EXPORTED = ("prism_plan_create", "prism_plan_bytes", "prism_plan_build", "prism_
             "prism_plan_view_get", "prism_plan_check", "prism_plan_destroy", "prism_last_error",
             "prism_plan_set_timing", "prism_plan_read_timing", "prism_timer_name", "prism_zone_shapes_noalloc",
             "prism_plan_selftest_timeout", "prism_plan_update_qkv", "prism_step_host", "prism_step_join",
-            "prism_step_wait", "prism_audio_norms")
+            "prism_step_wait", "prism_audio_norms", "prism_plan_build_stats", "prism_plan_stats_slice",
+            "prism_plan_build_finish")
 NUM_TIMERS = 10
 
 
@@ -39,7 +40,7 @@ class prism_params(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
                 ("heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("top_k", ctypes.c_int),
                 ("top_p", ctypes.c_float), ("max_frac", ctypes.c_float), ("fixed_shape", ctypes.c_int * 3),
-                ("eps", ctypes.c_double)]
+                ("eps", ctypes.c_double), ("heads_total", ctypes.c_int), ("head_offset", ctypes.c_int)]
 
 
 class prism_plan_view(ctypes.Structure):
@@ -82,6 +83,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.prism_step_join.restype = ctypes.c_int
     lib.prism_step_wait.argtypes = [V, ctypes.c_ulonglong]
     lib.prism_step_wait.restype = ctypes.c_int
+    lib.prism_plan_build_stats.argtypes = [V, P, P, P]
+    lib.prism_plan_build_stats.restype = ctypes.c_int
+    S = ctypes.POINTER(ctypes.c_size_t)
+    lib.prism_plan_stats_slice.argtypes = [V, ctypes.POINTER(ctypes.c_void_p), S, S, S]
+    lib.prism_plan_stats_slice.restype = ctypes.c_int
+    lib.prism_plan_build_finish.argtypes = [V, P, P, P, P]
+    lib.prism_plan_build_finish.restype = ctypes.c_int
     lib.prism_audio_norms.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
     lib.prism_audio_norms.restype = ctypes.c_int
     lib.prism_plan_destroy.argtypes = [V]
@@ -128,8 +136,13 @@ class _DevArray:
 
 
 def _dev_tensor(ptr: int, shape, dtype=torch.int32) -> torch.Tensor:
-    ts = {torch.int32: "<i4"}[dtype]
-    return torch.as_tensor(_DevArray(ptr, shape, ts), device="cuda").clone()
+    return _dev_view(ptr, shape, dtype).clone()
+
+
+def _dev_view(ptr: int, shape, dtype) -> torch.Tensor:
+    """Zero-copy tensor over device memory the plan owns (valid while the plan lives)."""
+    ts = {torch.int32: "<i4", torch.float64: "<f8"}[dtype]
+    return torch.as_tensor(_DevArray(ptr, shape, ts), device="cuda")
 
 
 @dataclass
@@ -145,11 +158,13 @@ class Params:
     max_frac: float = 0.0
     fixed_shape: Tuple[int, int, int] = (0, 0, 0)
     eps: float = 1e-6
+    heads_total: int = 0  # head sharding: this plan holds heads [head_offset, head_offset + heads)
+    head_offset: int = 0
 
     def to_c(self) -> prism_params:
         return prism_params(self.batch, self.T, self.H, self.W, self.heads, self.head_dim, self.top_k,
                             float(self.top_p), float(self.max_frac), (ctypes.c_int * 3)(*self.fixed_shape),
-                            float(self.eps))
+                            float(self.eps), int(self.heads_total), int(self.head_offset))
 
     @property
     def N(self) -> int:
@@ -197,6 +212,38 @@ class PrismPlan:
         _need(a_norm, "a_norm", torch.float32, (p.batch, p.T, p.H, p.W))
         _check(load_library().prism_plan_build(self._h, _ptr(Q), _ptr(K), _ptr(V), _ptr(a_norm), _stream()))
         return self
+
+    # -- the build in two halves (head-sharded plans) --------------------------
+    def build_stats(self, V: torch.Tensor, a_norm: torch.Tensor):
+        p = self.params
+        _need(V, "V", torch.bfloat16, self._qkv_shape())
+        _need(a_norm, "a_norm", torch.float32, (p.batch, p.T, p.H, p.W))
+        _check(load_library().prism_plan_build_stats(self._h, _ptr(V), _ptr(a_norm), _stream()))
+        return self
+
+    def stats_slice(self):
+        """(whole-layer zone-statistics buffer as a float64 device tensor, this plan's
+        slice of it as a view): the tensors alias the plan's memory."""
+        buf, off, n, tot = ctypes.c_void_p(), ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+        _check(load_library().prism_plan_stats_slice(self._h, ctypes.byref(buf), ctypes.byref(off), ctypes.byref(n),
+                                                     ctypes.byref(tot)))
+        whole = _dev_view(buf.value, (tot.value // 8,), torch.float64)
+        return whole, whole[off.value // 8:(off.value + n.value) // 8]
+
+    def build_finish(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor):
+        for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+            _need(t, n, torch.bfloat16, self._qkv_shape())
+        _check(load_library().prism_plan_build_finish(self._h, _ptr(Q), _ptr(K), _ptr(V), _stream()))
+        return self
+
+    def build_sharded(self, Q, K, V, a_norm, group=None):
+        """Head-sharded build: zone statistics of this rank's heads, one all-gather
+        of every rank's slice (torch.distributed, ranks holding equal consecutive
+        head ranges in rank order), then the rest of the plan."""
+        self.build_stats(V, a_norm)
+        whole, mine = self.stats_slice()
+        exchange_zone_stats(whole, mine, group)
+        return self.build_finish(Q, K, V)
 
     def update_qkv(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor):
         """Reuse the plan (zones, shapes, permutation, selection) for new Q, K, V."""
@@ -319,6 +366,16 @@ def prism_zone_shapes_noalloc(params: Params, V: torch.Tensor, a_norm: torch.Ten
 
 
 # Module-level names that mirror the C ABI.
+def exchange_zone_stats(whole: torch.Tensor, mine: torch.Tensor, group=None):
+    """All-gather of the ranks' zone-statistics slices into `whole` (rank order =
+    slice order).  Single process: nothing to exchange."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+        return whole
+    dist.all_gather_into_tensor(whole, mine.clone(), group=group)
+    return whole
+
+
 def prism_audio_norms(h: torch.Tensor, T: int, H: int, W: int, a: Optional[torch.Tensor] = None) -> torch.Tensor:
     """a_{t,h,w} = ||h^_{t,h,w}||_2 for h [batch, T*H*W, channels] bf16 on the current device."""
     if h.dtype != torch.bfloat16 or not h.is_cuda or h.dim() != 3 or not h.is_contiguous():

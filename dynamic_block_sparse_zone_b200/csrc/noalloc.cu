@@ -78,6 +78,11 @@ extern "C" PRISM_API prism_status prism_zone_shapes_noalloc(const prism_params *
     g.M = g.MT * g.MH * g.MW;
     g.nbmax = g.N / 64;
     g.C = p->heads * p->head_dim;
+    if (p->heads_total != 0 && p->heads_total != p->heads)
+        return fail(PRISM_ERR_UNSUPPORTED, "prism_zone_shapes_noalloc takes every head of the layer (no sharding)");
+    g.Ctot = g.C;
+    g.chunk0 = 0;
+    g.nchunk_tot = (g.C + kStatChunk - 1) / kStatChunk;
     int fixed_idx = -1;
     if (p->fixed_shape[0] || p->fixed_shape[1] || p->fixed_shape[2]) {
         int table[kNumShapes][3];

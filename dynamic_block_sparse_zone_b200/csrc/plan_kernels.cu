@@ -94,7 +94,6 @@ __global__ void __launch_bounds__(128) k_zone_stats_v(const __nv_bfloat16 *__res
     float *wpart = hpart + 8 * 8 * kStatChunk;          // [t][w][128]
     __shared__ double red[4][3];
     const int chunk = blockIdx.x, m = blockIdx.y, b = blockIdx.z;
-    const int nchunk = gridDim.x;
     const int tid = threadIdx.x, ts = tid >> 4, l = tid & 15;
     const int zt = m / (g.MH * g.MW), zh = (m / g.MW) % g.MH, zw = m % g.MW;
     const int c0 = chunk * kStatChunk + l * 8;
@@ -178,7 +177,8 @@ __global__ void __launch_bounds__(128) k_zone_stats_v(const __nv_bfloat16 *__res
     if (tid < 3) {
         double s = 0.0;
         for (int wq = 0; wq < 4; ++wq) s = __dadd_rn(s, red[wq][tid]);
-        zone_part[(((size_t)b * g.M + m) * nchunk + chunk) * 3 + tid] = s;
+        // chunk-major: a rank's heads are one contiguous slice of the layer's partials
+        zone_part[(((size_t)(g.chunk0 + chunk) * g.batch + b) * g.M + m) * 3 + tid] = s;
     }
 }
 
@@ -265,13 +265,16 @@ __device__ __forceinline__ int block_scan_excl_1024(int v, int *buf, int *total)
     return excl;
 }
 
-__device__ __forceinline__ double zone_sig(const double *zone_part, int nchunk, size_t zm, int d, int C) {
+// sigma^2_{v,d}(m): the chunk partials of zone zm (= b * M + m) summed in chunk
+// order over the whole layer's channels, divided by their count
+__device__ __forceinline__ double zone_sig(const double *zone_part, const Geo &g, size_t zm, int d) {
+    const size_t bm = (size_t)g.batch * g.M;
     double s = 0.0;
-    for (int c = 0; c < nchunk; ++c) s = __dadd_rn(s, zone_part[(zm * nchunk + c) * 3 + d]);
-    return s / (double)C;
+    for (int c = 0; c < g.nchunk_tot; ++c) s = __dadd_rn(s, zone_part[(c * bm + zm) * 3 + d]);
+    return s / (double)g.Ctot;
 }
 
-__global__ void __launch_bounds__(1024) k_zone_decide(Geo g, int nchunk, const double *__restrict__ zone_part,
+__global__ void __launch_bounds__(1024) k_zone_decide(Geo g, const double *__restrict__ zone_part,
                                                       const double *__restrict__ zone_a, double eps,
                                                       int fixed_idx, int *__restrict__ zone_B,
                                                       int *__restrict__ zone_shape, int *__restrict__ zone_blk0,
@@ -288,8 +291,8 @@ __global__ void __launch_bounds__(1024) k_zone_decide(Geo g, int nchunk, const d
     double smax = 0.0, amax = -DBL_MAX;
     for (int m = tid; m < M; m += blockDim.x) {
         size_t zm = (size_t)b * M + m;
-        double s = __dadd_rn(__dadd_rn(zone_sig(zone_part, nchunk, zm, 0, g.C), zone_sig(zone_part, nchunk, zm, 1, g.C)),
-                             zone_sig(zone_part, nchunk, zm, 2, g.C));
+        double s = __dadd_rn(__dadd_rn(zone_sig(zone_part, g, zm, 0), zone_sig(zone_part, g, zm, 1)),
+                             zone_sig(zone_part, g, zm, 2));
         smax = fmax(smax, s);
         amax = fmax(amax, zone_a[zm * 5 + 4]);
     }
@@ -324,7 +327,7 @@ __global__ void __launch_bounds__(1024) k_zone_decide(Geo g, int nchunk, const d
             size_t zm = (size_t)b * M + m;
             double sg[3], sa[3];
             for (int d = 0; d < 3; ++d) {
-                sg[d] = zone_sig(zone_part, nchunk, zm, d, g.C);
+                sg[d] = zone_sig(zone_part, g, zm, d);
                 sa[d] = zone_a[zm * 5 + d];
             }
             const double sv = __dadd_rn(__dadd_rn(sg[0], sg[1]), sg[2]);
@@ -956,11 +959,10 @@ static prism_status scan_into(const int *in, size_t n, int *out, int *tmp, cudaS
 
 size_t select_smem_bytes(const Plan &pl) { return sel_smem_layout(pl.g.D, pl.g.nbmax, pl.cap_stride).bytes; }
 
-prism_status launch_plan(Plan &pl, const void *Qv, const void *Kv, const void *Vv, const float *a,
-                         cudaStream_t st) {
+// Zone statistics of this plan's heads (their chunks of the layer's partials)
+// and of the audio guidance.
+prism_status launch_plan_stats(Plan &pl, const void *Vv, const float *a, cudaStream_t st) {
     const Geo &g = pl.g;
-    const auto *Q = static_cast<const __nv_bfloat16 *>(Qv);
-    const auto *K = static_cast<const __nv_bfloat16 *>(Kv);
     const auto *V = static_cast<const __nv_bfloat16 *>(Vv);
     const int nchunk = (g.C + kStatChunk - 1) / kStatChunk;
     const size_t smem_v = 2 * 8 * 8 * kStatChunk * sizeof(float);
@@ -968,8 +970,25 @@ prism_status launch_plan(Plan &pl, const void *Qv, const void *Kv, const void *V
     k_zone_stats_v<<<dim3(nchunk, g.M, g.batch), 128, smem_v, st>>>(V, g, pl.zone_part); }
     { TimerScope ts(pl, kTZoneA, st);
     k_zone_stats_a<<<dim3(g.M, g.batch), 512, 0, st>>>(a, g, pl.zone_a); }
+    PRISM_CUDA_OK(cudaGetLastError());
+    return PRISM_OK;
+}
+
+prism_status launch_plan(Plan &pl, const void *Qv, const void *Kv, const void *Vv, const float *a,
+                         cudaStream_t st) {
+    prism_status s = launch_plan_stats(pl, Vv, a, st);
+    return s == PRISM_OK ? launch_plan_finish(pl, Qv, Kv, Vv, st) : s;
+}
+
+// Everything after the zone statistics (which hold every chunk of the layer
+// by now): decisions, block table, permutation and pooling, selection, CSR/CSC.
+prism_status launch_plan_finish(Plan &pl, const void *Qv, const void *Kv, const void *Vv, cudaStream_t st) {
+    const Geo &g = pl.g;
+    const auto *Q = static_cast<const __nv_bfloat16 *>(Qv);
+    const auto *K = static_cast<const __nv_bfloat16 *>(Kv);
+    const auto *V = static_cast<const __nv_bfloat16 *>(Vv);
     { TimerScope ts(pl, kTDecide, st);
-    k_zone_decide<<<g.batch, 1024, 0, st>>>(g, nchunk, pl.zone_part, pl.zone_a, pl.p.eps, pl.fixed_idx,
+    k_zone_decide<<<g.batch, 1024, 0, st>>>(g, pl.zone_part, pl.zone_a, pl.p.eps, pl.fixed_idx,
                                             pl.zone_B, pl.zone_shape, pl.zone_blk0, pl.nb, pl.blk_off,
                                             pl.tile_blk, pl.zone_qt0, pl.nqt, pl.qt_row, pl.qt_blk); }
     const int pp_threads = g.C / 8 >= 384 ? 384 : ((g.C / 8 + 31) / 32) * 32;
@@ -1051,7 +1070,7 @@ prism_status launch_zone_decisions(const Geo &g, double eps, int fixed_idx, cons
     const size_t smem_v = 2 * 8 * 8 * kStatChunk * sizeof(float);
     k_zone_stats_v<<<dim3(nchunk, g.M, g.batch), 128, smem_v, st>>>(V, g, zone_part);
     k_zone_stats_a<<<dim3(g.M, g.batch), 512, 0, st>>>(a, g, zone_a);
-    k_zone_decide<<<g.batch, 1024, 0, st>>>(g, nchunk, zone_part, zone_a, eps, fixed_idx, zone_B, zone_shape,
+    k_zone_decide<<<g.batch, 1024, 0, st>>>(g, zone_part, zone_a, eps, fixed_idx, zone_B, zone_shape,
                                             zone_blk0, nb, blk_off, tile_blk, zone_qt0, nqt, qt_row, qt_blk);
     PRISM_CUDA_OK(cudaGetLastError());
     return PRISM_OK;

@@ -86,6 +86,16 @@ static prism_status check_params(const prism_params *p, Geo *g, int *fixed_idx, 
     g->M = g->MT * g->MH * g->MW;
     g->nbmax = g->N / 64;
     g->C = p->heads * p->head_dim;
+    // head sharding: this plan holds heads [head_offset, head_offset + heads) of heads_total
+    const int htot = p->heads_total ? p->heads_total : p->heads;
+    if (p->head_offset < 0 || p->head_offset + p->heads > htot)
+        return fail(PRISM_ERR_INVALID_ARG, "heads [%d, %d) do not lie within heads_total %d", p->head_offset,
+                    p->head_offset + p->heads, htot);
+    if (htot != p->heads && ((p->heads * p->head_dim) % kStatChunk || (p->head_offset * p->head_dim) % kStatChunk))
+        return fail(PRISM_ERR_UNSUPPORTED, "a head shard must cover whole %d-channel chunks", kStatChunk);
+    g->Ctot = htot * p->head_dim;
+    g->chunk0 = p->head_offset * p->head_dim / kStatChunk;
+    g->nchunk_tot = (g->Ctot + kStatChunk - 1) / kStatChunk;
     *cap_stride = cap_for(g->nbmax, p->top_k, p->max_frac);
     const long long rows = (long long)g->batch * g->heads * g->nbmax;
     if (rows * (long long)*cap_stride >= (1ll << 31))
@@ -115,7 +125,7 @@ struct Alloc {
 static size_t plan_allocs(Plan &pl, Alloc *out) {
     const Geo &g = pl.g;
     const size_t BH = (size_t)g.batch * g.heads, rows = BH * g.nbmax;
-    const int nchunk = (g.C + kStatChunk - 1) / kStatChunk;
+    const int nchunk = g.nchunk_tot;  // partials of the whole layer's channels
     const size_t nnz = rows * (size_t)pl.cap_stride;
     size_t n = 0;
     auto add = [&](void **p, size_t b) { out[n++] = Alloc{p, b}; };
@@ -315,8 +325,52 @@ prism_status prism_plan_build(prism_plan *plan, const void *Q, const void *K, co
     if (s != PRISM_OK) return s;
     const uintptr_t al = (uintptr_t)Q | (uintptr_t)K | (uintptr_t)V;
     if (al & 15) return fail(PRISM_ERR_INVALID_ARG, "Q, K, V must be 16-byte aligned");
+    if (plan->pl.g.Ctot != plan->pl.g.C)
+        return fail(PRISM_ERR_STATE, "a head-sharded plan is built with build_stats, an exchange and build_finish");
     plan->pl.have_fwd = false;
     s = launch_plan(plan->pl, Q, K, V, a_norm, static_cast<cudaStream_t>(stream));
+    if (s == PRISM_OK) plan->pl.built = true;
+    return s;
+}
+
+prism_status prism_plan_build_stats(prism_plan *plan, const void *V, const float *a_norm, void *stream) {
+    g_last_error.clear();
+    if (!plan || !V || !a_norm) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_plan_build_stats");
+    prism_status s = device_guard(plan->pl);
+    if (s != PRISM_OK) return s;
+    if ((uintptr_t)V & 15) return fail(PRISM_ERR_INVALID_ARG, "V must be 16-byte aligned");
+    plan->pl.have_fwd = false;
+    plan->pl.built = false;
+    s = launch_plan_stats(plan->pl, V, a_norm, static_cast<cudaStream_t>(stream));
+    plan->pl.have_stats = s == PRISM_OK;
+    return s;
+}
+
+prism_status prism_plan_stats_slice(prism_plan *plan, void **buf, size_t *slice_offset, size_t *slice_bytes,
+                                    size_t *total_bytes) {
+    g_last_error.clear();
+    if (!plan || !buf || !slice_offset || !slice_bytes || !total_bytes)
+        return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_plan_stats_slice");
+    const Geo &g = plan->pl.g;
+    const size_t per_chunk = (size_t)g.batch * g.M * 3 * sizeof(double);
+    *buf = plan->pl.zone_part;
+    *slice_offset = (size_t)g.chunk0 * per_chunk;
+    *slice_bytes = (size_t)((g.C + kStatChunk - 1) / kStatChunk) * per_chunk;
+    *total_bytes = (size_t)g.nchunk_tot * per_chunk;
+    return PRISM_OK;
+}
+
+prism_status prism_plan_build_finish(prism_plan *plan, const void *Q, const void *K, const void *V, void *stream) {
+    g_last_error.clear();
+    if (!plan || !Q || !K || !V) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_plan_build_finish");
+    prism_status s = device_guard(plan->pl);
+    if (s != PRISM_OK) return s;
+    const uintptr_t al = (uintptr_t)Q | (uintptr_t)K | (uintptr_t)V;
+    if (al & 15) return fail(PRISM_ERR_INVALID_ARG, "Q, K, V must be 16-byte aligned");
+    if (!plan->pl.have_stats) return fail(PRISM_ERR_STATE, "prism_plan_build_finish needs prism_plan_build_stats first");
+    plan->pl.have_fwd = false;
+    plan->pl.have_stats = false;
+    s = launch_plan_finish(plan->pl, Q, K, V, static_cast<cudaStream_t>(stream));
     if (s == PRISM_OK) plan->pl.built = true;
     return s;
 }
@@ -373,6 +427,8 @@ prism_status prism_step_host(prism_plan *plan, const prism_host_io *io, void *st
         return fail(PRISM_ERR_INVALID_ARG, "prism_step_host needs Q, K, V, a_norm and O");
     if (io->dO && (!io->dQ || !io->dK || !io->dV))
         return fail(PRISM_ERR_INVALID_ARG, "prism_step_host with dO needs dQ, dK and dV");
+    if (plan->pl.g.Ctot != plan->pl.g.C)
+        return fail(PRISM_ERR_STATE, "prism_step_host runs unsharded plans only");
     prism_status s = device_guard(plan->pl);
     if (s != PRISM_OK) return s;
     return host_step(plan->pl, *io, static_cast<cudaStream_t>(stream), ticket);

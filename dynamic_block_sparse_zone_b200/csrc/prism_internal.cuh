@@ -30,7 +30,11 @@ struct HostPipe;    // host-buffer step pipeline, defined in host_pipeline.cu
 // Per-launch problem geometry, passed by value to kernels.
 struct Geo {
     int batch, T, H, W, heads, D;
-    int N, M, MT, MH, MW, nbmax, C;
+    int N, M, MT, MH, MW, nbmax, C;  // C = heads * D: the channels this plan holds
+    // Zone statistics are kept per 128-channel chunk of the whole layer
+    // (heads_total * D channels, Ctot); this plan's heads are chunks
+    // [chunk0, chunk0 + C / 128) of nchunk_tot.  Unsharded: Ctot = C, chunk0 = 0.
+    int Ctot, chunk0, nchunk_tot;
 };
 
 // Everything a plan owns (device pointers unless noted).
@@ -42,8 +46,9 @@ struct Plan {
     int device;
     bool have_fwd;
     bool built;
+    bool have_stats;        // zone statistics computed since the last finished build
     // zone statistics and decisions
-    double *zone_part;      // [batch][M][nchunk][3]  sum_c of directional variances
+    double *zone_part;      // [nchunk_tot][batch][M][3] per 128-channel chunk: sum_c of directional variances
     double *zone_a;         // [batch][M][5]  sigma2_a T,H,W, mean a, max a
     int *zone_B;            // [batch][M]
     int *zone_shape;        // [batch][M]
@@ -105,6 +110,8 @@ prism_status fail_cuda(cudaError_t e, const char *what, const char *file, int li
 // Launchers (each returns PRISM_OK or an error after checking the launch).
 prism_status launch_plan(Plan &pl, const void *Q, const void *K, const void *V, const float *a,
                          cudaStream_t st);
+prism_status launch_plan_stats(Plan &pl, const void *V, const float *a, cudaStream_t st);
+prism_status launch_plan_finish(Plan &pl, const void *Q, const void *K, const void *V, cudaStream_t st);
 prism_status launch_attn_fwd_tc(Plan &pl, void *O, float *lse, cudaStream_t st);
 prism_status launch_regather(Plan &pl, const void *Q, const void *K, const void *V, cudaStream_t st);
 prism_status make_tensor_maps(Plan &pl);

@@ -66,7 +66,14 @@ typedef enum prism_status {
  * fixed_shape: {0,0,0} selects the dynamic shape of every zone
  *   [Prism guide, Method sections 1-2]; otherwise every zone uses this edge
  *   triple, which must be one of the 16 candidates (edges in {2,4,8}).
- * eps: the epsilon of the indicator g_d (1e-6 when <= 0 is given).        */
+ * eps: the epsilon of the indicator g_d (1e-6 when <= 0 is given).
+ * heads_total, head_offset: head sharding.  0, 0 (or heads_total == heads)
+ *   = the plan holds every head of the layer.  Otherwise the plan holds
+ *   heads [head_offset, head_offset + heads) of heads_total, Q/K/V carry only
+ *   those heads, and the plan is built in two halves around one exchange of
+ *   zone statistics between the ranks (prism_plan_build_stats,
+ *   prism_plan_stats_slice, prism_plan_build_finish); heads * head_dim and
+ *   head_offset * head_dim must be multiples of 128.                       */
 typedef struct prism_params {
     int batch, T, H, W, heads, head_dim;
     int top_k;
@@ -74,6 +81,7 @@ typedef struct prism_params {
     float max_frac;
     int fixed_shape[3];
     double eps;
+    int heads_total, head_offset;
 } prism_params;
 
 typedef struct prism_plan prism_plan;
@@ -117,6 +125,31 @@ PRISM_API size_t prism_plan_bytes(const prism_params *params);
  * transpose.  Q, K, V, a_norm: device, layouts above; read only.            */
 PRISM_API prism_status prism_plan_build(prism_plan *plan, const void *Q, const void *K, const void *V,
                               const float *a_norm, void *stream);
+
+/* The plan build in two halves, for head-sharded plans (one rank per GPU,
+ * each holding some heads of the layer).  The zone decisions need the
+ * statistics of every channel of the layer; after the decisions the heads are
+ * independent [Prism guide, Method sections 1-3].
+ *   prism_plan_build_stats: zone statistics of this plan's heads (V, device,
+ *     [batch][N][heads][head_dim]) and of a_norm.
+ *   prism_plan_stats_slice: the plan's device buffer of per-chunk zone
+ *     statistics of the whole layer (*buf, *total_bytes) and this plan's
+ *     slice of it (*slice_offset bytes in, *slice_bytes long).  Slices are
+ *     contiguous and ordered by head, so with ranks holding equal consecutive
+ *     head ranges one all-gather (each rank sending its slice, receiving the
+ *     whole buffer in rank order) gives every rank the layer's statistics.
+ *     The buffer belongs to the plan.
+ *   prism_plan_build_finish: decisions, permutation and pooling, selection,
+ *     CSR / CSC from the (complete) statistics, Q, K, V of this plan's heads.
+ * Every rank computes the same zone shapes and permutation, bit for bit the
+ * ones an unsharded plan of the whole layer computes.  prism_plan_build is
+ * build_stats followed by build_finish and is refused (PRISM_ERR_STATE) for a
+ * sharded plan, as is prism_step_host.                                     */
+PRISM_API prism_status prism_plan_build_stats(prism_plan *plan, const void *V, const float *a_norm, void *stream);
+PRISM_API prism_status prism_plan_stats_slice(prism_plan *plan, void **buf, size_t *slice_offset, size_t *slice_bytes,
+                                              size_t *total_bytes);
+PRISM_API prism_status prism_plan_build_finish(prism_plan *plan, const void *Q, const void *K, const void *V,
+                                               void *stream);
 
 /* Plan reuse: gathers new Q, K, V (device, layouts above) into the plan's
  * block-contiguous copies using the plan's existing zone shapes, permutation

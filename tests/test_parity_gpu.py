@@ -579,3 +579,63 @@ def test_audio_norms_feed_the_plan():
     g_out = run_gpu(w, inp)
     pl, _ = oracle_plan(w, inp)
     compare_plan(w, pl, g_out["view"])
+
+
+def test_head_sharded_plan_equals_the_whole_layer():
+    """A layer's heads split over two ranks (emulated in one process, the
+    all-gather done by copies): every rank's zone shapes, permutation and block
+    table equal those of an unsharded plan of the whole layer bit for bit, its
+    heads' selections equal the whole plan's rows for them, and its forward
+    outputs equal the whole plan's for its heads."""
+    P = _lib()
+    w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=4, planted=2)
+    inp = make_inputs(w, 0)
+    Q, K, V, a = (x.cuda() for x in (inp.Q, inp.K, inp.V, inp.a))
+    whole = P.PrismPlan(P.params_for(w))
+    whole.build(Q, K, V, a)
+    O_all, lse_all = whole.fwd()
+    v_all = whole.view()
+    torch.cuda.synchronize()
+
+    hs = 2
+    ranks = []
+    for r in range(2):
+        prm = P.params_for(w)
+        prm.heads, prm.heads_total, prm.head_offset = hs, w.heads, r * hs
+        plan = P.PrismPlan(prm)
+        sl = slice(r * hs, (r + 1) * hs)
+        Qr, Kr, Vr = (x[:, :, sl].contiguous() for x in (Q, K, V))
+        with pytest.raises(P.PrismError):
+            plan.build(Qr, Kr, Vr, a)  # a sharded plan needs the exchange
+        with pytest.raises(P.PrismError):
+            plan.build_finish(Qr, Kr, Vr)  # statistics first
+        plan.build_stats(Vr, a)
+        ranks.append((plan, Qr, Kr, Vr))
+    slices = [p.stats_slice() for p, *_ in ranks]
+    for r in range(2):  # the all-gather: every rank receives the other's slice
+        for s in range(2):
+            if s != r:
+                lo = slices[s][1].data_ptr() - slices[s][0].data_ptr()
+                slices[r][0][lo // 8: lo // 8 + slices[s][1].numel()].copy_(slices[s][1])
+    for r, (plan, Qr, Kr, Vr) in enumerate(ranks):
+        plan.build_finish(Qr, Kr, Vr)
+        O_r, lse_r = plan.fwd()
+        torch.cuda.synchronize()
+        plan.check()
+        v = plan.view()
+        for key in ("zone_B", "zone_shape", "perm"):
+            assert torch.equal(v[key], v_all[key]), key
+        nb = int(v["n_blocks"][0])
+        assert nb == int(v_all["n_blocks"][0])
+        assert torch.equal(v["blk_off"][:, :nb + 1], v_all["blk_off"][:, :nb + 1])
+        rp, rp_all = v["row_ptr"].cpu().numpy(), v_all["row_ptr"].cpu().numpy()
+        col, col_all = v["col_idx"].cpu().numpy(), v_all["col_idx"].cpu().numpy()
+        nbmax = v["nbmax"]
+        for hh in range(hs):
+            for i in range(nb):
+                ra, rb = hh * nbmax + i, (r * hs + hh) * nbmax + i
+                assert np.array_equal(col[rp[ra]:rp[ra + 1]], col_all[rp_all[rb]:rp_all[rb + 1]])
+        assert torch.equal(O_r, O_all[:, :, r * hs:(r + 1) * hs])
+        assert torch.equal(lse_r, lse_all[:, r * hs:(r + 1) * hs])
+        plan.close()
+    whole.close()
