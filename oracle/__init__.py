@@ -63,6 +63,8 @@ def _load():
             "orc_select": (None, [_P, _P, _I, _I, _I, _I, _D, _D, _I, _P, _P, _P]),
             "orc_attn_fwd_rows": (None, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _I,
                                          _I, _P, _P, _P, _P]),
+            "orc_attn_fwd_taylor_rows": (None, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _I,
+                                                _I, _P, _P, _P, _P]),
             "orc_attn_bwd_dq_rows": (None, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P,
                                             _I, _I, _P, _P, _P]),
             "orc_attn_bwd_dkv_rows": (None, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P,
@@ -285,6 +287,21 @@ def attn_fwd_rows(pl: OraclePlan, Q_bits, K_bits, V_bits, req_h, req_tok):
     _load().orc_attn_fwd_rows(_ptr(Qb), _ptr(Kb), _ptr(Vb), pl.T, pl.H, pl.W, pl.heads, pl.D, pl.nb,
                               _ptr(box), _ptr(cnt), _ptr(cols), stride, n, _ptr(req_h),
                               _ptr(req_tok), _ptr(O), _ptr(lse))
+    return O, lse
+
+
+def attn_fwd_taylor_rows(pl: OraclePlan, Q_bits, K_bits, V_bits, req_h, req_tok):
+    """O [n, D] and LSE [n] with the blocks outside each S_i added through a
+    zeroth-order Taylor term (pooled key, mean value, weight |B_j|)
+    [In-Context Sparse Attention article, grouped computation]."""
+    box, cnt, cols, stride = _attn_args(pl)
+    req_h = _c(req_h, np.int32); req_tok = _c(req_tok, np.int32)
+    n = req_h.shape[0]
+    O = np.zeros((n, pl.D)); lse = np.zeros(n)
+    Qb = _c(Q_bits, np.uint16); Kb = _c(K_bits, np.uint16); Vb = _c(V_bits, np.uint16)
+    _load().orc_attn_fwd_taylor_rows(_ptr(Qb), _ptr(Kb), _ptr(Vb), pl.T, pl.H, pl.W, pl.heads, pl.D,
+                                     pl.nb, _ptr(box), _ptr(cnt), _ptr(cols), stride, n, _ptr(req_h),
+                                     _ptr(req_tok), _ptr(O), _ptr(lse))
     return O, lse
 
 

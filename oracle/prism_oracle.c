@@ -42,6 +42,11 @@
  *   orc_attn_*                                     pinned (dense reduction vs
  *                                                  library SDPA, masked dense,
  *                                                  finite differences)
+ *   orc_attn_fwd_taylor_rows                       pinned (exact when every block
+ *                                                  is constant; uniform scores give
+ *                                                  the global mean of V; error of
+ *                                                  second order in a zero-mean key
+ *                                                  perturbation)
  *   orc_audio_norms                                pinned (closed forms: constant
  *                                                  rows, one-hot rows, integer
  *                                                  norms; an exact rational sum
@@ -577,6 +582,99 @@ void orc_attn_fwd_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
         free(toks);
         free(s);
     }
+    free(cx.tok2blk);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Forward with a zeroth-order Taylor term for the key blocks outside S_i.   */
+/* [In-Context Sparse Attention article, the grouped-computation paragraphs: */
+/* the flat path replaces the tokens of a key block by the block's mean and  */
+/* keeps only the zeroth-order term of the exponential's expansion.]         */
+/* Reading, for the blocks Prism's selection leaves out: for a token t of a  */
+/* key block j not in S_i, exp(q.k_t/sqrt(D)) is expanded around the block's */
+/* mean key kbar_j (mean of its bf16 keys, fp64) and cut after the constant  */
+/* term, exp(q.kbar_j/sqrt(D)).  Summed over the |B_j| tokens of the block:  */
+/*   normaliser  += |B_j| exp(q.kbar_j/sqrt(D))                              */
+/*   numerator   += exp(q.kbar_j/sqrt(D)) sum_t v_t                          */
+/*                = |B_j| exp(q.kbar_j/sqrt(D)) vbar_j.                      */
+/* The tokens of the blocks in S_i enter exactly, as in orc_attn_fwd_rows;   */
+/* one softmax normalises both parts.  LSE is log of the whole normaliser.  */
+/* ------------------------------------------------------------------------ */
+void orc_attn_fwd_taylor_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                              int T, int H, int W, int heads, int D, int nb, const int *box,
+                              const int *cnt, const int *cols, int stride,
+                              int nreq, const int *req_h, const int *req_tok,
+                              double *O /* [nreq][D] */, double *lse /* [nreq] */)
+{
+    attn_ctx cx = {Q, K, V, NULL, H, W, heads, D, nb, stride, box, cnt, cols, NULL};
+    ctx_init(&cx, T, H, W, nb, box);
+    size_t N = (size_t)T * H * W;
+    double *Kbar = (double *)malloc(sizeof(double) * (size_t)heads * nb * D);
+    double *Vbar = (double *)malloc(sizeof(double) * (size_t)heads * nb * D);
+    orc_pool(K, T, H, W, heads, D, nb, box, Kbar);
+    orc_pool(V, T, H, W, heads, D, nb, box, Vbar);
+    double sq = sqrt((double)D);
+#pragma omp parallel
+    {
+        int *toks = (int *)malloc(sizeof(int) * N);
+        double *s = (double *)malloc(sizeof(double) * N);
+        double *z = (double *)malloc(sizeof(double) * nb);
+        char *in_s = (char *)malloc((size_t)nb);
+#pragma omp for schedule(dynamic, 4)
+        for (int r = 0; r < nreq; ++r) {
+            int hd = req_h[r], q = req_tok[r];
+            int i = cx.tok2blk[q];
+            size_t row = (size_t)hd * nb + i;
+            memset(in_s, 0, (size_t)nb);
+            for (int u = 0; u < cnt[row]; ++u)
+                in_s[cols[row * stride + u]] = 1;
+            /* exact part: every token of the selected blocks */
+            int n = row_scores(&cx, hd, q, toks, s);
+            /* Taylor part: one pooled term per block outside S_i */
+            double mx = -INFINITY;
+            for (int u = 0; u < n; ++u)
+                if (s[u] > mx)
+                    mx = s[u];
+            for (int j = 0; j < nb; ++j) {
+                if (in_s[j])
+                    continue;
+                double dot = 0.0;
+                for (int c = 0; c < D; ++c)
+                    dot += widen_bf16(Q[((size_t)q * heads + hd) * D + c]) * Kbar[((size_t)hd * nb + j) * D + c];
+                z[j] = dot / sq;
+                if (z[j] > mx)
+                    mx = z[j];
+            }
+            double l = 0.0;
+            for (int u = 0; u < n; ++u)
+                l += exp(s[u] - mx);
+            for (int j = 0; j < nb; ++j)
+                if (!in_s[j])
+                    l += (double)(box[6 * j + 3] * box[6 * j + 4] * box[6 * j + 5]) * exp(z[j] - mx);
+            double L = mx + log(l);
+            for (int c = 0; c < D; ++c)
+                O[(size_t)r * D + c] = 0.0;
+            for (int u = 0; u < n; ++u) {
+                double pr = exp(s[u] - L);
+                for (int c = 0; c < D; ++c)
+                    O[(size_t)r * D + c] += pr * widen_bf16(V[((size_t)toks[u] * heads + hd) * D + c]);
+            }
+            for (int j = 0; j < nb; ++j) {
+                if (in_s[j])
+                    continue;
+                double wt = (double)(box[6 * j + 3] * box[6 * j + 4] * box[6 * j + 5]) * exp(z[j] - L);
+                for (int c = 0; c < D; ++c)
+                    O[(size_t)r * D + c] += wt * Vbar[((size_t)hd * nb + j) * D + c];
+            }
+            lse[r] = L;
+        }
+        free(toks);
+        free(s);
+        free(z);
+        free(in_s);
+    }
+    free(Kbar);
+    free(Vbar);
     free(cx.tok2blk);
 }
 

@@ -396,6 +396,147 @@ def test_sparse_attention_equals_masked_dense_fwd_bwd(name):
 
 
 # ---------------------------------------------------------------------------
+# Taylor term for the blocks outside S_i [In-Context Sparse Attention article,
+# grouped computation]: block j outside S_i enters as |B_j| exp(q.kbar_j/sqrt D)
+# with value vbar_j
+# ---------------------------------------------------------------------------
+def _mixed_blocks(T=8, H=16, W=16):
+    """A block partition with volumes 64, 128 and 256 (one zone shape each,
+    round robin over the zones) and its token -> block map."""
+    table = oracle.shape_table()
+    by_vol = {v: [i for i, e in enumerate(table) if int(e.sum()) == v] for v in (6, 7, 8)}
+    M = (T // 8) * (H // 8) * (W // 8)
+    zs = np.array([by_vol[(6, 7, 8)[m % 3]][m % len(by_vol[(6, 7, 8)[m % 3]])] for m in range(M)], np.int32)
+    box = oracle.blocks(T, H, W, zs)
+    tok_blk = np.zeros(T * H * W, np.int64)
+    for j, b in enumerate(box):
+        t, h, w_ = np.meshgrid(np.arange(b[0], b[0] + b[3]), np.arange(b[1], b[1] + b[4]),
+                               np.arange(b[2], b[2] + b[5]), indexing="ij")
+        tok_blk[((t * H + h) * W + w_).ravel()] = j
+    return box, tok_blk
+
+
+def _random_selection(rs, heads, nb):
+    stride = nb
+    cnt = np.zeros((heads, nb), np.int32)
+    cols = np.full((heads, nb, stride), -1, np.int32)
+    for h in range(heads):
+        for i in range(nb):
+            n = int(rs.integers(1, max(2, nb // 3)))
+            sel = np.sort(rs.choice(nb, size=n, replace=False))
+            cnt[h, i] = n
+            cols[h, i, :n] = sel
+    return cnt, cols
+
+
+def _taylor_plan(T, H, W, heads, D, box, cnt, cols):
+    from types import SimpleNamespace
+    return SimpleNamespace(T=T, H=H, W=W, heads=heads, D=D, nb=len(box), box=box, cnt=cnt, cols=cols)
+
+
+def _dense(Qb, Kb, Vb, h):
+    q, k, v = (_to64(x)[:, h, :].numpy() for x in (Qb, Kb, Vb))
+    s = q @ k.T / math.sqrt(q.shape[1])
+    mx = s.max(axis=1, keepdims=True)
+    e = np.exp(s - mx)
+    return (e @ v) / e.sum(axis=1, keepdims=True), (mx[:, 0] + np.log(e.sum(axis=1)))
+
+
+def test_taylor_is_exact_for_blockwise_constant_keys_and_values():
+    """With every key block's keys equal and its values equal, the zeroth-order
+    term is the whole sum over the block: the output is dense attention over all
+    tokens, whatever the selection (block volumes 64, 128 and 256 mixed)."""
+    T, H, W, heads, D = 8, 16, 16, 2, 32
+    rs = np.random.default_rng(5)
+    box, tok_blk = _mixed_blocks(T, H, W)
+    nb, N = len(box), T * H * W
+    assert set((box[:, 3] * box[:, 4] * box[:, 5]).tolist()) == {64, 128, 256}
+    kb = rs.normal(0, 1.0, (nb, heads, D)).astype(np.float32)
+    vb = rs.normal(0, 1.0, (nb, heads, D)).astype(np.float32)
+    Qb = f32_bits(rs.normal(0, 1.0, (N, heads, D)))
+    Kb = f32_bits(kb[tok_blk])
+    Vb = f32_bits(vb[tok_blk])
+    cnt, cols = _random_selection(rs, heads, nb)
+    pl = _taylor_plan(T, H, W, heads, D, box, cnt, cols)
+    for h in range(heads):
+        ref_o, ref_lse = _dense(Qb, Kb, Vb, h)
+        O, lse = oracle.attn_fwd_taylor_rows(pl, Qb, Kb, Vb, np.full(N, h, np.int32), np.arange(N, dtype=np.int32))
+        np.testing.assert_allclose(O, ref_o, atol=1e-12, rtol=1e-10)
+        np.testing.assert_allclose(lse, ref_lse, rtol=1e-12)
+    # the sparse output alone misses the blocks outside S_i: the test can tell
+    O_s, _ = oracle.attn_fwd_rows(pl, Qb, Kb, Vb, np.zeros(N, np.int32), np.arange(N, dtype=np.int32))
+    assert np.max(np.abs(O_s - _dense(Qb, Kb, Vb, 0)[0])) > 1e-2
+
+
+def test_taylor_with_zero_queries_is_the_mean_of_all_values():
+    """q = 0 makes every score 0: exact and pooled terms alike weigh each token
+    equally, so O is the mean of V over all N tokens and LSE = log N."""
+    T, H, W, heads, D = 8, 16, 16, 2, 16
+    rs = np.random.default_rng(6)
+    box, _ = _mixed_blocks(T, H, W)
+    nb, N = len(box), T * H * W
+    Qb = f32_bits(np.zeros((N, heads, D)))
+    Kb = f32_bits(rs.normal(0, 1.0, (N, heads, D)))
+    Vb = f32_bits(rs.normal(0, 1.0, (N, heads, D)))
+    cnt, cols = _random_selection(rs, heads, nb)
+    pl = _taylor_plan(T, H, W, heads, D, box, cnt, cols)
+    req_t = rs.integers(0, N, 64).astype(np.int32)
+    for h in range(heads):
+        O, lse = oracle.attn_fwd_taylor_rows(pl, Qb, Kb, Vb, np.full(64, h, np.int32), req_t)
+        mean = _to64(Vb)[:, h, :].numpy().mean(axis=0)
+        np.testing.assert_allclose(O, np.broadcast_to(mean, O.shape), atol=1e-13)
+        np.testing.assert_allclose(lse, math.log(N), rtol=1e-14)
+
+
+def test_taylor_error_is_second_order_around_the_block_mean():
+    """Keys k_t = kbar_j + eps * delta_t with delta summing to zero over each
+    block (tokens paired with opposite signs) and values constant per block:
+    the first-order term of the expansion around the mean cancels, so the error
+    against dense attention shrinks 4x when eps halves (2x would mean the
+    expansion point is not the mean)."""
+    T, H, W, heads, D = 8, 16, 16, 1, 16
+    rs = np.random.default_rng(7)
+    box, tok_blk = _mixed_blocks(T, H, W)
+    nb, N = len(box), T * H * W
+    base = rs.integers(-2, 3, (nb, heads, D)).astype(np.float32) * 0.5
+    vb = rs.normal(0, 1.0, (nb, heads, D)).astype(np.float32)
+    sign = rs.choice([-1.0, 1.0], (N, heads, D)).astype(np.float32)
+    for j in range(nb):  # pair consecutive tokens of the block with opposite signs
+        toks = np.nonzero(tok_blk == j)[0]
+        sign[toks[1::2]] = -sign[toks[0::2]]
+    Qb = f32_bits(rs.normal(0, 1.0, (N, heads, D)))
+    Vb = f32_bits(vb[tok_blk])
+    cnt, cols = _random_selection(rs, heads, nb)
+    pl = _taylor_plan(T, H, W, heads, D, box, cnt, cols)
+    req_t = np.arange(0, N, 5, dtype=np.int32)
+    errs = []
+    for k in (5, 6, 7):
+        eps = 2.0 ** -k
+        kk = base[tok_blk] + eps * sign
+        Kb = f32_bits(kk)
+        np.testing.assert_array_equal(_to64(Kb).numpy(), kk)  # exact in bf16
+        O, _ = oracle.attn_fwd_taylor_rows(pl, Qb, Kb, Vb, np.zeros(len(req_t), np.int32), req_t)
+        errs.append(np.max(np.abs(O - _dense(Qb, Kb, Vb, 0)[0][req_t])))
+    assert errs[0] > 1e-6
+    for a, b in zip(errs, errs[1:]):
+        assert 3.8 < a / b < 4.2, errs
+
+
+def test_taylor_with_every_block_selected_is_the_sparse_forward():
+    """No block outside S_i: nothing to approximate."""
+    w = WORKLOADS["tiny_8x16x16"]
+    inp, Qb, Kb, Vb = _tiny_case(w, 2)
+    pl = oracle.plan(Qb, Kb, Vb, inp.a[0].numpy(), w.T, w.H, w.W, w.heads, w.head_dim, 10 ** 6, 1.0)
+    assert np.all(pl.cnt == pl.nb)
+    rt = np.arange(0, w.N, 3, dtype=np.int32)
+    rh = (rt % w.heads).astype(np.int32)
+    O_t, l_t = oracle.attn_fwd_taylor_rows(pl, Qb, Kb, Vb, rh, rt)
+    O_s, l_s = oracle.attn_fwd_rows(pl, Qb, Kb, Vb, rh, rt)
+    np.testing.assert_array_equal(O_t, O_s)
+    np.testing.assert_array_equal(l_t, l_s)
+
+
+# ---------------------------------------------------------------------------
 # Generator: planted zones stand out along their axis
 # ---------------------------------------------------------------------------
 def test_planted_zones_raise_directional_variation():
