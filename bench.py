@@ -115,6 +115,25 @@ def selected_pairs(view, D):
     return int((si * sj).sum().item())
 
 
+def pooled_pairs(view):
+    """sum over rows of |B_i| * (N_b - |S_i|): (query token, pooled key block)
+    pairs of the Taylor term, per sample."""
+    import torch
+    blk = view["blk_off"].long()
+    nbmax = view["nbmax"]
+    rp = view["row_ptr"].long()
+    B = blk.shape[0]
+    nbs = torch.as_tensor([int(x) for x in view["n_blocks"]], device=rp.device)
+    rows = torch.arange(rp.numel() - 1, device=rp.device)
+    counts = rp[1:] - rp[:-1]
+    sample = rows // (rows.numel() // B)
+    i = rows % nbmax
+    valid = i < nbs[sample]
+    sizes = blk[:, 1:] - blk[:, :-1]
+    si = torch.where(valid, sizes[sample, i.clamp(max=nbmax - 1)], torch.zeros_like(i))
+    return int((si * (nbs[sample] - counts) * valid).sum().item())
+
+
 def kernel_bytes(name, w, nb, pairs_unused):
     """Algorithmic HBM bytes of one launch of the plan kernels (one sample)."""
     N, C, D, h = w.N, w.heads * w.head_dim, w.head_dim, w.heads
@@ -126,6 +145,8 @@ def kernel_bytes(name, w, nb, pairs_unused):
         return 2 * N * C * 2 + N * C * 2 + h * N * 4
     if name == "dq_finalize":
         return h * N * D * 4 + N * C * 2
+    if name == "taylor_pool":  # read V (permuted) and the fp64 pooled keys, write two bf16 pooled copies
+        return N * C * 2 + h * nb * D * 8 + 2 * h * nb * D * 2
     return None
 
 
@@ -178,7 +199,7 @@ def run_ours(args, rank, world, dev):
 
     def step(Q, K, V, a, dO):
         plan.build(Q, K, V, a)
-        plan.fwd(O, lse)
+        plan.fwd(O, lse, taylor=args.taylor)
         if not args.fwd_only:
             plan.bwd(O, dO, dQ, dK, dV)
 
@@ -189,7 +210,8 @@ def run_ours(args, rank, world, dev):
     view = plan.view()
     pairs = selected_pairs(view, w.head_dim)
     nb = view["n_blocks"][0]
-    flops_fwd = 4.0 * w.head_dim * pairs
+    tpairs = pooled_pairs(view) if args.taylor else 0
+    flops_fwd = 4.0 * w.head_dim * (pairs + tpairs)
     flops_bwd = 10.0 * w.head_dim * pairs
     flops_step = flops_fwd + (0.0 if args.fwd_only else flops_bwd)
 
@@ -270,7 +292,7 @@ def run_ours(args, rank, world, dev):
     # plan and the attention kernels, and copies its outputs back; the plan
     # overlaps one step's copies with its neighbours' kernels on three streams.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.taylor:
         host_in = [x.cpu().pin_memory() for x in (inp.Q, inp.K, inp.V, inp.a)]
         host_dO = None if args.fwd_only else inp.dO.cpu().pin_memory()
         host_out = [torch.empty(shp, dtype=torch.bfloat16).pin_memory() for _ in range(1 if args.fwd_only else 4)]
@@ -315,7 +337,7 @@ def run_ours(args, rank, world, dev):
         if name == "select":
             rec["fp64_tflops"] = round(2.0 * w.head_dim * nb * nb * w.heads * w.batch * steps_or_1(args) /
                                        (tms * 1e-3) / 1e12, 3)
-        if name == "attn_fwd":
+        if name in ("attn_fwd", "attn_fwd_taylor"):
             rec["tflops"] = round(flops_fwd / (avg * 1e-3) / 1e12, 2)
         elif name == "attn_bwd":
             rec["tflops"] = round(flops_bwd / (avg * 1e-3) / 1e12, 2)
@@ -352,7 +374,10 @@ def run_ours(args, rank, world, dev):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "pass": "forward" if args.fwd_only else "forward+backward",
+        "config": {"workload": w.name,
+                   "pass": ("forward with the Taylor term for unselected blocks" if args.taylor else
+                            "forward" if args.fwd_only else "forward+backward"),
+                   "taylor_pooled_pairs": tpairs if args.taylor else None,
                    "grid": [w.T, w.H, w.W], "tokens": w.N, "heads": w.heads,
                    "head_dim": w.head_dim, "top_k": w.top_k, "top_p": w.top_p, "max_frac": w.max_frac,
                    "n_blocks": nb, "selected_token_pairs": pairs, "flops_per_step": flops_step,
@@ -411,8 +436,9 @@ def oracle_setup(w, dev):
     return pl, hb, plan_s
 
 
-def oracle_sample(pl, hb, w, rows, seed):
-    """fwd + dQ of `rows` query tokens of one head; returns (seconds, flops)."""
+def oracle_sample(pl, hb, w, rows, seed, taylor=False):
+    """fwd + dQ of `rows` query tokens of one head (taylor: the forward with the
+    Taylor term alone); returns (seconds, flops)."""
     import numpy as np
     import oracle
     rs = np.random.default_rng(seed)
@@ -427,6 +453,11 @@ def oracle_sample(pl, hb, w, rows, seed):
     for t in req_t:
         i = tok2blk[t]
         keys += int(sizes[pl.cols[0, i, :pl.cnt[0, i]]].sum())
+    if taylor:
+        pooled = int(sum(pl.nb - pl.cnt[0, tok2blk[t]] for t in req_t))
+        t0 = time.time()
+        oracle.attn_fwd_taylor_rows(pl, hb[0], hb[1], hb[2], req_h, req_t)
+        return time.time() - t0, 4.0 * w.head_dim * (keys + pooled)
     t0 = time.time()
     oracle.attn_fwd_rows(pl, hb[0], hb[1], hb[2], req_h, req_t)
     oracle.attn_bwd_dq_rows(pl, hb[0], hb[1], hb[2], hb[3], req_h, req_t)
@@ -435,12 +466,13 @@ def oracle_sample(pl, hb, w, rows, seed):
     return dt, 10.0 * w.head_dim * keys
 
 
-def cpu_baseline(w, dev, rows):
+def cpu_baseline(w, dev, rows, taylor=False):
     import oracle
     pl, hb, plan_s = oracle_setup(w, dev)
-    dt, fl = oracle_sample(pl, hb, w, rows, 123)
+    dt, fl = oracle_sample(pl, hb, w, rows, 123, taylor)
+    what = "forward with the Taylor term" if taylor else "forward + dQ"
     return {"value": round(fl / dt / 1e12, 8), "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"fp64 oracle forward + dQ of {rows} random query tokens of head 0 on the same "
+            "sample": f"fp64 oracle {what} of {rows} random query tokens of head 0 on the same "
                       f"workload ({dt:.1f} s); oracle plan with 1-head selection took {plan_s:.1f} s, not counted"}
 
 
@@ -480,10 +512,14 @@ def main():
     ap.add_argument("--fwd-only", action="store_true", help="step = plan + forward (forward-only workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true", help="time replays of the step captured in a CUDA graph")
+    ap.add_argument("--taylor", action="store_true",
+                    help="forward with the zeroth-order Taylor term for the unselected blocks (implies --fwd-only)")
     ap.add_argument("--heads", type=int, default=0, help="override the workload's head count (profiling)")
     ap.add_argument("--cpu-rows", type=int, default=6000)
     ap.add_argument("--ref-rows", type=int, default=1500)
     args = ap.parse_args()
+    if args.taylor:
+        args.fwd_only = True
     if args.warmup < 3:
         args.warmup = 3
 
@@ -509,7 +545,7 @@ def main():
         if world == 1 and not args.no_cpu_baseline:
             torch.cuda.empty_cache()
             from dynamic_block_sparse_zone_b200.synth import WORKLOADS
-            res["cpu_baseline"] = cpu_baseline(workload_of(args), dev, args.cpu_rows)
+            res["cpu_baseline"] = cpu_baseline(workload_of(args), dev, args.cpu_rows, args.taylor)
         print(json.dumps(res), flush=True)
     if world > 1:
         import torch.distributed as dist

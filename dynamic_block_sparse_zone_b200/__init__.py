@@ -4,9 +4,9 @@ The computation lives in libprism.so (CUDA, C ABI in include/prism.h);
 ``binding`` marshals torch tensors into it.  ``synth`` draws seeded inputs.
 """
 from .binding import (PrismError, PrismPlan, Params, load_library, params_for, prism_attn_bwd,
-                      prism_attn_fwd, prism_plan_build, prism_plan_bytes, prism_plan_create,
+                      prism_attn_fwd, prism_attn_fwd_taylor, prism_plan_build, prism_plan_bytes, prism_plan_create,
                       prism_plan_destroy)
 
 __all__ = ["PrismError", "PrismPlan", "Params", "load_library", "params_for", "prism_attn_bwd",
-           "prism_attn_fwd", "prism_plan_build", "prism_plan_bytes", "prism_plan_create",
+           "prism_attn_fwd", "prism_attn_fwd_taylor", "prism_plan_build", "prism_plan_bytes", "prism_plan_create",
            "prism_plan_destroy"]

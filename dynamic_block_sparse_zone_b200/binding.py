@@ -26,8 +26,8 @@ EXPORTED = ("prism_plan_create", "prism_plan_bytes", "prism_plan_build", "prism_
             "prism_plan_set_timing", "prism_plan_read_timing", "prism_timer_name", "prism_zone_shapes_noalloc",
             "prism_plan_selftest_timeout", "prism_plan_update_qkv", "prism_step_host", "prism_step_join",
             "prism_step_wait", "prism_audio_norms", "prism_plan_build_stats", "prism_plan_stats_slice",
-            "prism_plan_build_finish")
-NUM_TIMERS = 10
+            "prism_plan_build_finish", "prism_attn_fwd_taylor")
+NUM_TIMERS = 12
 
 
 class PrismError(RuntimeError):
@@ -70,6 +70,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.prism_plan_bytes.restype = ctypes.c_size_t
     lib.prism_plan_build.argtypes = [V, P, P, P, P, P]
     lib.prism_attn_fwd.argtypes = [V, P, P, P]
+    lib.prism_attn_fwd_taylor.argtypes = [V, P, P, P]
+    lib.prism_attn_fwd_taylor.restype = ctypes.c_int
     lib.prism_plan_update_qkv.argtypes = [V, P, P, P, P]
     lib.prism_plan_update_qkv.restype = ctypes.c_int
     lib.prism_attn_bwd.argtypes = [V, P, P, P, P, P, P]
@@ -252,7 +254,10 @@ class PrismPlan:
         _check(load_library().prism_plan_update_qkv(self._h, _ptr(Q), _ptr(K), _ptr(V), _stream()))
         return self
 
-    def fwd(self, O: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, want_lse: bool = True):
+    def fwd(self, O: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+            taylor: bool = False):
+        """Sparse forward over S_i; with taylor=True the blocks outside S_i are
+        added through their pooled keys and mean values (prism_attn_fwd_taylor)."""
         p = self.params
         if O is None:
             O = torch.empty(self._qkv_shape(), dtype=torch.bfloat16, device="cuda")
@@ -261,7 +266,8 @@ class PrismPlan:
             lse = torch.empty((p.batch, p.heads, p.N), dtype=torch.float32, device="cuda")
         if lse is not None:
             _need(lse, "lse", torch.float32, (p.batch, p.heads, p.N))
-        _check(load_library().prism_attn_fwd(self._h, _ptr(O), _ptr(lse), _stream()))
+        fn = load_library().prism_attn_fwd_taylor if taylor else load_library().prism_attn_fwd
+        _check(fn(self._h, _ptr(O), _ptr(lse), _stream()))
         return O, lse
 
     def bwd(self, O: torch.Tensor, dO: torch.Tensor, dQ=None, dK=None, dV=None):
@@ -400,6 +406,10 @@ def prism_plan_build(plan: PrismPlan, Q, K, V, a_norm) -> PrismPlan:
 
 def prism_attn_fwd(plan: PrismPlan, O=None, lse=None):
     return plan.fwd(O, lse)
+
+
+def prism_attn_fwd_taylor(plan: PrismPlan, O=None, lse=None):
+    return plan.fwd(O, lse, taylor=True)
 
 
 def prism_attn_bwd(plan: PrismPlan, O, dO, dQ=None, dK=None, dV=None):

@@ -26,6 +26,16 @@
 //                than 2^8 (it is current then: S_c was issued after PV_{c-1}).
 //                Epilogue: O / l to the user layout, log-sum-exp.
 // TMEM columns: S / P [0,128), O [128, 128+D).
+//
+// Taylor variant (kTaylor) [In-Context Sparse Attention article, grouped
+// computation: the flat path scores block-mean keys and keeps the zeroth-order
+// term of the exponential]: after the selected blocks, the same pipeline
+// streams the head's pooled keys kbar_j and mean values vbar_j (bf16, 128 per
+// chunk).  Block j then adds |B_j| exp2(x) with x its scaled pooled score: its
+// softmax column gets the bias log2 |B_j|, or -inf when j is in S_i (those
+// blocks are already exact) or past the last block.  Each softmax warp writes
+// the 128 biases of a chunk into its own shared buffer from a bitmask of S_i
+// that the CTA builds once; one online softmax covers both parts.
 #include <cuda.h>
 
 #include "tc_common.cuh"
@@ -52,15 +62,21 @@ struct Layout {
     static constexpr uint32_t kNumBars = 9;
     static constexpr uint32_t kBytes = kBars + kNumBars * 8 + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;  // slack to align the base to 1024
+    // Taylor variant: per-softmax-warp bias of a chunk, then the S_i bitmask
+    static constexpr uint32_t kBias = (kBytes + 15) & ~15u;
+    static constexpr uint32_t kMask = kBias + 4 * 128 * 4;
+    static uint32_t taylor_alloc(int nbmax) { return kMask + (((nbmax + 31) / 32 * 4 + 15) & ~15u) + 1024; }
 };
 
 // Site codes recorded with a timeout.
 enum { kSiteQ = 1, kSiteK, kSiteV, kSiteKEmpty, kSiteVEmpty, kSiteS, kSiteP, kSiteO };
 
-template <int D>
+template <int D, bool kTaylor>
 __global__ void __launch_bounds__(kThreads, 2)
     k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, Geo g, const int *__restrict__ nqt,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
+                  const __grid_constant__ CUtensorMap tmVb, const int *__restrict__ nbv, Geo g,
+                  const int *__restrict__ nqt,
                   const int *__restrict__ qt_row, const int *__restrict__ qt_blk, const int *__restrict__ blk_off,
                   const int *__restrict__ row_ptr, const int *__restrict__ col, const int *__restrict__ perm,
                   __nv_bfloat16 *__restrict__ O, float *__restrict__ lse_user, float *__restrict__ nlse_p,
@@ -90,6 +106,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) nseg += __shfl_xor_sync(0xffffffffu, nseg, o);
     const int nchunk = (nseg + 1) >> 1;
+    // Taylor variant: pooled chunks follow the selected ones
+    const int nbb = kTaylor ? nbv[b] : 0;
+    const int nseg_t = (nbb + 63) >> 6;
+    const int nchunk_all = nchunk + ((nseg_t + 1) >> 1);
+    auto chunk_full = [&](int c) { return c < nchunk ? (2 * c + 1) < nseg : (2 * (c - nchunk) + 1) < nseg_t; };
+    uint32_t *mask = reinterpret_cast<uint32_t *>(smem + L::kMask);
+    if constexpr (kTaylor)
+        for (int w = threadIdx.x; w < (nbb + 31) >> 5; w += kThreads) mask[w] = 0u;
 
     const uint32_t bar_q = sbase + L::kBars;
     const uint32_t bar_kf = bar_q + 8, bar_ke = bar_q + 16, bar_vf = bar_q + 24, bar_ve = bar_q + 32;
@@ -122,6 +146,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if constexpr (kTaylor) {  // S_i as a bitmask over the key blocks
+        for (int u = c_begin + threadIdx.x; u < c_end; u += kThreads) {
+            const int j = col[u];
+            atomicOr(&mask[j >> 5], 1u << (j & 31));
+        }
+        __syncthreads();
+    }
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS = tmem, tO = tmem + 128;
 
@@ -140,16 +171,22 @@ __global__ void __launch_bounds__(kThreads, 2)
                 r_end = bo[col[u] + 1];
             }
             int kissued = 0, vissued = 0;
-            for (int c = 0; c < nchunk; ++c) {
-                const int nsg = min(2, nseg - 2 * c);
+            for (int c = 0; c < nchunk_all; ++c) {
+                const bool pooled = kTaylor && c >= nchunk;
+                const int nsg = pooled ? min(2, nseg_t - 2 * (c - nchunk)) : min(2, nseg - 2 * c);
                 const uint32_t bytes = nsg * 64 * D * 2;
+                const CUtensorMap *mK = pooled ? &tmKb : &tmK, *mV = pooled ? &tmVb : &tmV;
                 int rows[2];
-                for (int gsg = 0; gsg < nsg; ++gsg) {
-                    rows[gsg] = r;
-                    r += 64;
-                    if (r >= r_end && ++u < c_end) {
-                        r = bo[col[u]];
-                        r_end = bo[col[u] + 1];
+                if (pooled) {  // rows of the pooled [batch*heads][nbmax][D] copies
+                    for (int gsg = 0; gsg < nsg; ++gsg) rows[gsg] = bh * g.nbmax + 128 * (c - nchunk) + 64 * gsg;
+                } else {
+                    for (int gsg = 0; gsg < nsg; ++gsg) {
+                        rows[gsg] = rowbase + r;
+                        r += 64;
+                        if (r >= r_end && ++u < c_end) {
+                            r = bo[col[u]];
+                            r_end = bo[col[u] + 1];
+                        }
                     }
                 }
                 // K_c once S_{c-1} has consumed the K buffer
@@ -157,16 +194,16 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mbar_expect_tx(bar_kf, bytes);
                 for (int gsg = 0; gsg < nsg; ++gsg)
                     for (int hf = 0; hf < L::kHalves; ++hf)
-                        tma_load_2d(sbase + L::kK + hf * L::kTileBytes + gsg * 8192, &tmK, bar_kf, hf * 64,
-                                    rowbase + rows[gsg]);
+                        tma_load_2d(sbase + L::kK + hf * L::kTileBytes + gsg * 8192, mK, bar_kf, hf * 64,
+                                    rows[gsg]);
                 kissued = c + 1;
                 // V_c once P_{c-1} V_{c-1} has consumed the V buffer
                 if (c > 0 && !mbar_wait(bar_ve, (c - 1) & 1, status, kSiteVEmpty, abort_flag)) break;
                 mbar_expect_tx(bar_vf, bytes);
                 for (int gsg = 0; gsg < nsg; ++gsg)
                     for (int hf = 0; hf < L::kHalves; ++hf)
-                        tma_load_2d(sbase + L::kV + hf * L::kTileBytes + gsg * 8192, &tmV, bar_vf, hf * 64,
-                                    rowbase + rows[gsg]);
+                        tma_load_2d(sbase + L::kV + hf * L::kTileBytes + gsg * 8192, mV, bar_vf, hf * 64,
+                                    rows[gsg]);
                 vissued = c + 1;
             }
             // drain: every issued load must land before the CTA may exit
@@ -180,8 +217,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             constexpr uint32_t idS128 = idesc_bf16(128, 128, false), idS64 = idesc_bf16(128, 64, false);
             constexpr uint32_t idPV = idesc_bf16(128, D, true);
             bool ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, status, kSiteQ, abort_flag));
-            for (int c = 0; ok && c < nchunk; ++c) {
-                const bool full = (2 * c + 1) < nseg;
+            for (int c = 0; ok && c < nchunk_all; ++c) {
+                const bool full = chunk_full(c);
                 if (!__all_sync(0xffffffffu, mbar_wait(bar_kf, c & 1, status, kSiteK, abort_flag))) break;
                 tc_fence_after();
                 // k-step kk: 32 B along a 128-B row, the second 64 columns a tile further
@@ -215,11 +252,26 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         float m = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int c = 0; c < nchunk; ++c) {
+        const uint32_t bias_s = sbase + L::kBias + quad * 512;  // this warp's 128 column biases
+        for (int c = 0; c < nchunk_all; ++c) {
+            const bool pooled = kTaylor && c >= nchunk;
+            if (pooled) {  // biases of this chunk's pooled keys, before S lands
+                float *bias = reinterpret_cast<float *>(smem + L::kBias + quad * 512);
+                __syncwarp();  // the warp has read the previous chunk's biases
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 128 * (c - nchunk) + 32 * e + lane;
+                    float bv = -INFINITY;
+                    // block volumes are powers of two: log2 |B_j| is exact
+                    if (j < nbb && !((mask[j >> 5] >> (j & 31)) & 1u)) bv = (float)(31 - __clz(bo[j + 1] - bo[j]));
+                    bias[32 * e + lane] = bv;
+                }
+                __syncwarp();
+            }
             ok = __all_sync(0xffffffffu, mbar_wait(bar_s, c & 1, status, kSiteS, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            const int nq = ((2 * c + 1) < nseg) ? 4 : 2;  // 32-column groups of S in this chunk
+            const int nq = chunk_full(c) ? 4 : 2;  // 32-column groups of S in this chunk
             const uint32_t tSr = tS + lane_off;
             // the whole S row into registers: one TMEM round trip for both passes
             uint32_t sr[128];
@@ -227,22 +279,51 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int q = 0; q < 4; ++q)
                 if (q < nq) tmem_ld32(tSr + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * q]));
             tmem_wait_ld();
-            // pass 1: row max (three-input max, four independent chains)
+            // pass 1: row max (three-input max, four independent chains).  Pooled
+            // chunks first turn S into x = S*scale*log2e + bias in place.
             float mxa = -INFINITY, mxb = -INFINITY, mxc = -INFINITY, mxd = -INFINITY;
+            if (pooled) {
+                const uint64_t s2 = splat2(scale_log2);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                if (q < nq) {
+                for (int q = 0; q < 4; ++q)
+                    if (q < nq) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        const float *v = reinterpret_cast<const float *>(&sr[32 * q + e]);
-                        mxa = fmax3(mxa, v[0], v[1]);
-                        mxb = fmax3(mxb, v[2], v[3]);
-                        mxc = fmax3(mxc, v[4], v[5]);
-                        mxd = fmax3(mxd, v[6], v[7]);
+                        for (int e = 0; e < 32; e += 4) {
+                            const float4 bb = lds_f4(bias_s + (32 * q + e) * 4);
+                            float x0, x1, x2, x3;
+                            fma2(__uint_as_float(sr[32 * q + e]), __uint_as_float(sr[32 * q + e + 1]), s2,
+                                 pair2(bb.x, bb.y), x0, x1);
+                            fma2(__uint_as_float(sr[32 * q + e + 2]), __uint_as_float(sr[32 * q + e + 3]), s2,
+                                 pair2(bb.z, bb.w), x2, x3);
+                            sr[32 * q + e] = __float_as_uint(x0);
+                            sr[32 * q + e + 1] = __float_as_uint(x1);
+                            sr[32 * q + e + 2] = __float_as_uint(x2);
+                            sr[32 * q + e + 3] = __float_as_uint(x3);
+                            if (e & 4) {
+                                mxc = fmax3(mxc, x0, x1);
+                                mxd = fmax3(mxd, x2, x3);
+                            } else {
+                                mxa = fmax3(mxa, x0, x1);
+                                mxb = fmax3(mxb, x2, x3);
+                            }
+                        }
                     }
-                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (q < nq) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 8) {
+                            const float *v = reinterpret_cast<const float *>(&sr[32 * q + e]);
+                            mxa = fmax3(mxa, v[0], v[1]);
+                            mxb = fmax3(mxb, v[2], v[3]);
+                            mxc = fmax3(mxc, v[4], v[5]);
+                            mxd = fmax3(mxd, v[6], v[7]);
+                        }
+                    }
+            }
             const float mx = fmaxf(fmaxf(mxa, mxb), fmaxf(mxc, mxd));
-            const float mx2 = mx * scale_log2;
+            const float mx2 = pooled ? mx : mx * scale_log2;
             const bool need = (c > 0) && (mx2 > m + kRescaleThreshold);
             if (c == 0) m = mx2;
             // TMEM loads / stores are warp-collective: the whole warp rescales when
@@ -265,8 +346,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             // pass 2: P = exp2(S*scale*log2e - m), bf16 pairs written over S
             // (group q packs into columns [16q, 16q+16); all of S is in registers).
-            // (scale, -m) and the running sum as packed fp32 pairs
-            const uint64_t s2 = splat2(scale_log2), c2 = splat2(-m);
+            // (scale, -m) and the running sum as packed fp32 pairs; a pooled
+            // chunk's registers already hold the scaled, biased x.
+            const uint64_t s2 = splat2(pooled ? 1.0f : scale_log2), c2 = splat2(-m);
             uint64_t acc2 = 0;
 #pragma unroll
             for (int q = 0; q < 4; ++q)
@@ -295,8 +377,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_arrive(bar_p2);
         }
         // epilogue: the last product P V must have landed
-        if (ok && nchunk > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (nchunk - 1) & 1, status, kSiteO, abort_flag));
-        if (ok && nchunk > 0) {
+        if (ok && nchunk_all > 0)
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (nchunk_all - 1) & 1, status, kSiteO, abort_flag));
+        if (ok && nchunk_all > 0) {
             tc_fence_after();
             const float inv = 1.f / l;
             const int n = q0 + rowid;
@@ -321,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             if (write) {
                 const float lse2 = m + __log2f(l);
-                nlse_p[(size_t)bh * g.N + n] = -lse2;  // negated, log2 units: the backward's exp2 addend
+                if (!kTaylor) nlse_p[(size_t)bh * g.N + n] = -lse2;  // negated, log2 units: the backward's exp2 addend
                 if (lse_user) lse_user[(size_t)bh * g.N + tok] = lse2 * 0.69314718055994531f;
             }
         }
@@ -409,7 +492,10 @@ static prism_status make_map_f32_rows(CUtensorMap *m, const void *base, uint64_t
 
 prism_status make_tensor_maps(Plan &pl) {
     const uint64_t rows = (uint64_t)pl.g.batch * pl.g.heads * pl.g.N;
+    const uint64_t prow = (uint64_t)pl.g.batch * pl.g.heads * pl.g.nbmax;
     prism_status s = make_map(&pl.tmQ, pl.Qp, rows, pl.g.D);
+    if (s == PRISM_OK) s = make_map(&pl.tmKb, pl.Kb, prow, pl.g.D);
+    if (s == PRISM_OK) s = make_map(&pl.tmVb, pl.Vb, prow, pl.g.D);
     if (s == PRISM_OK) s = make_map(&pl.tmK, pl.Kp, rows, pl.g.D);
     if (s == PRISM_OK) s = make_map(&pl.tmV, pl.Vp, rows, pl.g.D);
     if (s == PRISM_OK) s = make_map(&pl.tmdO, pl.dOp, rows, pl.g.D);
@@ -417,28 +503,92 @@ prism_status make_tensor_maps(Plan &pl) {
     return s;
 }
 
-template <int D>
+template <int D, bool kTaylor>
 static prism_status fwd_tc_impl(Plan &pl, void *O, float *lse, cudaStream_t st) {
     const Geo &g = pl.g;
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
-    TimerScope ts(pl, kTAttnFwd, st);
-    fwdtc::k_attn_fwd_tc<D><<<dim3(g.nbmax, g.batch * g.heads), fwdtc::kThreads, fwdtc::Layout<D>::kAlloc, st>>>(
-        pl.tmQ, pl.tmK, pl.tmV, g, pl.nqt, pl.qt_row, pl.qt_blk, pl.blk_off, pl.row_ptr, pl.col, pl.perm,
-        static_cast<__nv_bfloat16 *>(O), lse, pl.nlse_p, scale_log2, pl.status);
+    const uint32_t smem = kTaylor ? fwdtc::Layout<D>::taylor_alloc(g.nbmax) : fwdtc::Layout<D>::kAlloc;
+    TimerScope ts(pl, kTaylor ? kTAttnFwdTaylor : kTAttnFwd, st);
+    fwdtc::k_attn_fwd_tc<D, kTaylor><<<dim3(g.nbmax, g.batch * g.heads), fwdtc::kThreads, smem, st>>>(
+        pl.tmQ, pl.tmK, pl.tmV, pl.tmKb, pl.tmVb, pl.nb, g, pl.nqt, pl.qt_row, pl.qt_blk, pl.blk_off, pl.row_ptr,
+        pl.col, pl.perm, static_cast<__nv_bfloat16 *>(O), lse, pl.nlse_p, scale_log2, pl.status);
     PRISM_CUDA_OK(cudaGetLastError());
     return PRISM_OK;
 }
 
+// Largest dynamic shared memory of a CTA on sm_100 (227 KB).
+constexpr int kMaxDynSmem = 232448;
+
 prism_status configure_attn_tc_kernels() {
-    PRISM_CUDA_OK(cudaFuncSetAttribute(fwdtc::k_attn_fwd_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    PRISM_CUDA_OK(cudaFuncSetAttribute(fwdtc::k_attn_fwd_tc<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)fwdtc::Layout<64>::kAlloc));
-    PRISM_CUDA_OK(cudaFuncSetAttribute(fwdtc::k_attn_fwd_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    PRISM_CUDA_OK(cudaFuncSetAttribute(fwdtc::k_attn_fwd_tc<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)fwdtc::Layout<128>::kAlloc));
+    PRISM_CUDA_OK(cudaFuncSetAttribute(fwdtc::k_attn_fwd_tc<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kMaxDynSmem));
+    PRISM_CUDA_OK(cudaFuncSetAttribute(fwdtc::k_attn_fwd_tc<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kMaxDynSmem));
     return PRISM_OK;
 }
 
 prism_status launch_attn_fwd_tc(Plan &pl, void *O, float *lse, cudaStream_t st) {
-    return pl.g.D == 64 ? fwd_tc_impl<64>(pl, O, lse, st) : fwd_tc_impl<128>(pl, O, lse, st);
+    return pl.g.D == 64 ? fwd_tc_impl<64, false>(pl, O, lse, st) : fwd_tc_impl<128, false>(pl, O, lse, st);
+}
+
+bool taylor_fits(const Geo &g) {
+    const uint32_t need = g.D == 64 ? fwdtc::Layout<64>::taylor_alloc(g.nbmax) : fwdtc::Layout<128>::taylor_alloc(g.nbmax);
+    return need <= (uint32_t)kMaxDynSmem;
+}
+
+// Pooled bf16 copies for the Taylor term, one CTA per (block j, sample*head):
+// Kb_j = bf16(kbar_j) from the plan's fp64 pooled keys; Vb_j = bf16(mean of
+// the block's rows of the permuted V), summed in fp32.
+__global__ void __launch_bounds__(256) k_taylor_pool(Geo g, const int *__restrict__ nbv,
+                                                     const int *__restrict__ blk_off,
+                                                     const double *__restrict__ Kbar,
+                                                     const __nv_bfloat16 *__restrict__ Vp,
+                                                     __nv_bfloat16 *__restrict__ Kb, __nv_bfloat16 *__restrict__ Vb) {
+    __shared__ float part[256 * 8];
+    const int j = blockIdx.x, bh = blockIdx.y, b = bh / g.heads;
+    if (j >= nbv[b]) return;
+    const int *bo = blk_off + (size_t)b * (g.nbmax + 1);
+    const int r0 = bo[j], r1 = bo[j + 1];
+    const size_t prow = (size_t)bh * g.nbmax + j;
+    for (int d = threadIdx.x; d < g.D; d += blockDim.x) Kb[prow * g.D + d] = __double2bfloat16(Kbar[prow * g.D + d]);
+    const int lpr = g.D / 8, groups = 256 / lpr;  // 16-byte lanes per row, rows in flight
+    const int ln = threadIdx.x % lpr, grp = threadIdx.x / lpr;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const __nv_bfloat16 *src = Vp + ((size_t)bh * g.N) * g.D + ln * 8;
+    for (int r = r0 + grp; r < r1; r += groups) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(src + (size_t)r * g.D));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            acc[2 * k] += __uint_as_float(w[k] << 16);
+            acc[2 * k + 1] += __uint_as_float(w[k] & 0xFFFF0000u);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) part[threadIdx.x * 8 + k] = acc[k];
+    __syncthreads();
+    const float inv = 1.0f / (float)(r1 - r0);  // a power of two: exact
+    for (int d = threadIdx.x; d < g.D; d += blockDim.x) {
+        const int l = d / 8, k = d % 8;
+        float sum = 0.f;
+        for (int q = 0; q < groups; ++q) sum += part[(q * lpr + l) * 8 + k];
+        Vb[prow * g.D + d] = __float2bfloat16_rn(sum * inv);
+    }
+}
+
+prism_status launch_attn_fwd_taylor(Plan &pl, void *O, float *lse, cudaStream_t st) {
+    const Geo &g = pl.g;
+    {
+        TimerScope ts(pl, kTTaylorPool, st);
+        k_taylor_pool<<<dim3(g.nbmax, g.batch * g.heads), 256, 0, st>>>(g, pl.nb, pl.blk_off, pl.Kbar, pl.Vp,
+                                                                        pl.Kb, pl.Vb);
+        PRISM_CUDA_OK(cudaGetLastError());
+    }
+    return g.D == 64 ? fwd_tc_impl<64, true>(pl, O, lse, st) : fwd_tc_impl<128, true>(pl, O, lse, st);
 }
 
 }  // namespace prism

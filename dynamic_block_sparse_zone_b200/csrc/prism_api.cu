@@ -147,6 +147,8 @@ static size_t plan_allocs(Plan &pl, Alloc *out) {
     add((void **)&pl.Vp, BH * g.N * g.D * 2);
     add((void **)&pl.Qbar, rows * g.D * sizeof(double));
     add((void **)&pl.Kbar, rows * g.D * sizeof(double));
+    add((void **)&pl.Kb, rows * g.D * 2);
+    add((void **)&pl.Vb, rows * g.D * 2);
     add((void **)&pl.score_keys, (size_t)pl.score_group * g.nbmax * g.nbmax * sizeof(unsigned long long));
     add((void **)&pl.cnt, rows * sizeof(int));
     add((void **)&pl.cols_pad, nnz * sizeof(int));
@@ -284,6 +286,8 @@ prism_status prism_plan_create(const prism_params *params, prism_plan **out) {
     }
     e = cudaMallocHost((void **)&pl.host_nb, 64 * sizeof(int));
     if (e == cudaSuccess) e = cudaMemset(pl.status, 0, 16 * sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(pl.Kb, 0, (size_t)pl.g.batch * pl.g.heads * pl.g.nbmax * pl.g.D * 2);
+    if (e == cudaSuccess) e = cudaMemset(pl.Vb, 0, (size_t)pl.g.batch * pl.g.heads * pl.g.nbmax * pl.g.D * 2);
     if (e != cudaSuccess) {
         release_buffers(pl);
         delete h;
@@ -399,6 +403,18 @@ prism_status prism_attn_fwd(prism_plan *plan, void *O, float *lse, void *stream)
     return s;
 }
 
+prism_status prism_attn_fwd_taylor(prism_plan *plan, void *O, float *lse, void *stream) {
+    g_last_error.clear();
+    if (!plan || !O) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_attn_fwd_taylor");
+    prism_status s = device_guard(plan->pl);
+    if (s != PRISM_OK) return s;
+    if (!plan->pl.built) return fail(PRISM_ERR_STATE, "prism_attn_fwd_taylor needs a built plan");
+    if ((uintptr_t)O & 15) return fail(PRISM_ERR_INVALID_ARG, "O must be 16-byte aligned");
+    if (!taylor_fits(plan->pl.g))
+        return fail(PRISM_ERR_UNSUPPORTED, "too many blocks for the Taylor forward's shared-memory bitmask");
+    return launch_attn_fwd_taylor(plan->pl, O, lse, static_cast<cudaStream_t>(stream));
+}
+
 prism_status prism_attn_bwd(prism_plan *plan, const void *O, const void *dO, void *dQ, void *dK, void *dV,
                             void *stream) {
     g_last_error.clear();
@@ -477,7 +493,7 @@ prism_status prism_plan_view_get(prism_plan *plan, prism_plan_view *view, void *
 
 static const char *const kTimerNames[kTCount] = {"zone_stats_v", "zone_stats_a", "zone_decide", "permute_pool",
                                                   "select", "csr_csc", "attn_fwd", "attn_bwd_pre", "attn_bwd",
-                                                  "dq_finalize"};
+                                                  "dq_finalize", "taylor_pool", "attn_fwd_taylor"};
 
 const char *prism_timer_name(int id) { return (id >= 0 && id < kTCount) ? kTimerNames[id] : ""; }
 

@@ -20,7 +20,7 @@ constexpr int kNumShapes = 16;
 
 enum TimerId {
     kTZoneV = 0, kTZoneA, kTDecide, kTPermutePool, kTSelect, kTCsr, kTAttnFwd, kTBwdPre, kTAttnBwd, kTDqFinal,
-    kTCount
+    kTTaylorPool, kTAttnFwdTaylor, kTCount
 };
 static_assert(kTCount == PRISM_NUM_TIMERS, "timer count");
 
@@ -64,6 +64,8 @@ struct Plan {
     // permuted head-major inputs and pooled blocks
     __nv_bfloat16 *Qp, *Kp, *Vp;   // [batch*heads][N][D]
     double *Qbar, *Kbar;           // [batch*heads][nbmax][D]
+    __nv_bfloat16 *Kb, *Vb;        // [batch*heads][nbmax][D] bf16 pooled keys / mean values (Taylor term),
+                                   // zeroed at creation so rows past a build's last block stay finite
     // selection
     unsigned long long *score_keys;  // [score_group][nbmax][nbmax] order-preserving score keys
     int score_group;        // heads scored per pass
@@ -86,6 +88,7 @@ struct Plan {
     HostPipe *pipe;         // NULL until the first host-buffer step
     // TMA descriptors of the permuted copies, viewed as [batch*heads*N][D] bf16
     CUtensorMap tmQ, tmK, tmV, tmdO;
+    CUtensorMap tmKb, tmVb;  // the pooled bf16 copies, viewed as [batch*heads*nbmax][D]
     CUtensorMap tmdQ;       // fp32 [batch*heads*N][D], 64-row boxes, reduce-add target
 };
 
@@ -113,6 +116,8 @@ prism_status launch_plan(Plan &pl, const void *Q, const void *K, const void *V, 
 prism_status launch_plan_stats(Plan &pl, const void *V, const float *a, cudaStream_t st);
 prism_status launch_plan_finish(Plan &pl, const void *Q, const void *K, const void *V, cudaStream_t st);
 prism_status launch_attn_fwd_tc(Plan &pl, void *O, float *lse, cudaStream_t st);
+prism_status launch_attn_fwd_taylor(Plan &pl, void *O, float *lse, cudaStream_t st);
+bool taylor_fits(const Geo &g);  // the Taylor forward's shared memory fits one CTA
 prism_status launch_regather(Plan &pl, const void *Q, const void *K, const void *V, cudaStream_t st);
 prism_status make_tensor_maps(Plan &pl);
 prism_status launch_attn_bwd_tc_main(Plan &pl, void *dK, void *dV, cudaStream_t st);

@@ -170,6 +170,24 @@ PRISM_API prism_status prism_plan_update_qkv(prism_plan *plan, const void *Q, co
  * plan keeps its own copy of the statistics for prism_attn_bwd.           */
 PRISM_API prism_status prism_attn_fwd(prism_plan *plan, void *O, float *lse, void *stream);
 
+/* Forward with a zeroth-order Taylor term for the key blocks outside S_i
+ * [In-Context Sparse Attention article, grouped computation: the flat path
+ * scores block-mean keys and keeps the zeroth-order term of the
+ * exponential].  The blocks of S_i enter exactly, as in prism_attn_fwd; each
+ * other key block j enters once, through its mean key kbar_j and mean value
+ * vbar_j (both rounded to bf16), as if all |B_j| of its tokens scored
+ * q.kbar_j / sqrt(D):
+ *   O_q = (sum_{t in S_i} e^{s_qt} v_t + sum_{j not in S_i} |B_j| e^{q.kbar_j/sqrt D} vbar_j)
+ *         / (the same sums without v).
+ * Same arguments, layouts and errors as prism_attn_fwd; lse (optional) is
+ * the log of the whole denominator.  Reads the plan's pooled keys and its
+ * permuted V of the last build or update; enqueues a pooling kernel and the
+ * attention kernel.  It leaves the statistics that prism_attn_bwd uses
+ * untouched: the backward differentiates the sparse forward only.
+ * PRISM_ERR_UNSUPPORTED when the bitmask of S_i (one bit per key block)
+ * does not fit a CTA's shared memory (more than about 1.6 million blocks). */
+PRISM_API prism_status prism_attn_fwd_taylor(prism_plan *plan, void *O, float *lse, void *stream);
+
 /* Gradient of sum(O * dO) with respect to Q, K, V through the same sparse
  * attention (the plan and the forward's statistics are reused).  O is the
  * forward's output and dO the incoming gradient (device, bf16, user layout);
@@ -254,7 +272,7 @@ PRISM_API prism_status prism_plan_selftest_timeout(prism_plan *plan, void *strea
  * for each timer id the summed milliseconds and the number of launches since
  * the previous read (arrays of PRISM_NUM_TIMERS host entries), and resets.
  * Timer ids and names: prism_timer_name(id).                               */
-#define PRISM_NUM_TIMERS 10
+#define PRISM_NUM_TIMERS 12
 PRISM_API prism_status prism_plan_set_timing(prism_plan *plan, int enable);
 PRISM_API prism_status prism_plan_read_timing(prism_plan *plan, float *total_ms, int *launches);
 PRISM_API const char *prism_timer_name(int id);

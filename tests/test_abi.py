@@ -79,6 +79,7 @@ def test_null_arguments_are_rejected(lib):
     assert lib.prism_plan_create(None, None) == 1
     assert lib.prism_plan_build(None, None, None, None, None, None) == 1
     assert lib.prism_attn_fwd(None, None, None, None) == 1
+    assert lib.prism_attn_fwd_taylor(None, None, None, None) == 1
     assert lib.prism_attn_bwd(None, None, None, None, None, None, None) == 1
     assert lib.prism_plan_build_stats(None, None, None, None) == 1
     assert lib.prism_plan_build_finish(None, None, None, None, None) == 1

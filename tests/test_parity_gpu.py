@@ -139,6 +139,23 @@ def check_forward(w, inp, g, pl, bits, nrows, heads=None, b=0):
     return req_h, req_t
 
 
+def check_forward_taylor(w, plan, pl, bits, nrows, heads=None, b=0, out=None):
+    """prism_attn_fwd_taylor against the oracle's forward with the zeroth-order
+    Taylor term for the blocks outside S_i, on sampled rows (out: the (O, lse)
+    of an earlier call)."""
+    O, lse = plan.fwd(taylor=True) if out is None else out
+    torch.cuda.synchronize()
+    plan.check()
+    rs = np.random.default_rng(12)
+    req_h, req_t = sample_rows(rs, w, nrows, heads)
+    ho = req_h if heads is None else np.searchsorted(np.asarray(heads), req_h).astype(np.int32)
+    pl_h = pl if heads is None else _heads_view(pl, heads)
+    O_ref, lse_ref = oracle.attn_fwd_taylor_rows(pl_h, *_head_slice(bits, heads), ho, req_t)
+    res = assert_close("O(taylor)", O[b].float().cpu().numpy()[req_t, req_h], O_ref)
+    assert np.max(np.abs(lse[b].cpu().numpy()[req_h, req_t] - lse_ref)) < 2e-3
+    return res
+
+
 def _heads_view(pl, heads):
     import copy
     p2 = copy.copy(pl)
@@ -302,6 +319,7 @@ def test_latent720p_full_size():
     pl, bits = oracle_plan(w, inp, heads=heads)
     ties = compare_plan(w, pl, g["view"], heads=heads)
     check_forward(w, inp, g, pl, bits, 256, heads=heads)
+    check_forward_taylor(w, g["plan"], pl, bits, 128, heads=heads)
     print("720p near-ties", ties, "blocks", pl.nb)
 
 
@@ -330,6 +348,7 @@ def test_latent2k_train_full_size_sampled():
     assert_close("dK", g["dK"][0].float().cpu().numpy()[req_t, heads[0]], dK_ref)
     assert_close("dV", g["dV"][0].float().cpu().numpy()[req_t, heads[0]], dV_ref)
     check_gradient_sums(g, inp)
+    check_forward_taylor(w, g["plan"], pl, bits, 64, heads=heads)
     print("2K near-ties", ties, "blocks", pl.nb)
 
 
@@ -428,6 +447,8 @@ def test_plan_reuse_with_new_inputs():
     assert_close("O", O[0].float().cpu().numpy()[req_t, req_h], O_ref)
     dQ_ref = oracle.attn_bwd_dq_rows(pl, *bits2, bf16_bits(second.dO[0]), req_h[:128], req_t[:128])
     assert_close("dQ", dQ[0].float().cpu().numpy()[req_t[:128], req_h[:128]], dQ_ref)
+    # the Taylor term pools the second inputs' keys and values under the first plan
+    check_forward_taylor(w, plan, pl, bits2, 512)
 
 
 def test_host_steps_match_the_device_path():
@@ -639,3 +660,72 @@ def test_head_sharded_plan_equals_the_whole_layer():
         assert torch.equal(lse_r, lse_all[:, r * hs:(r + 1) * hs])
         plan.close()
     whole.close()
+
+
+# ---------------------------------------------------------------------------
+# Zeroth-order Taylor term for the key blocks outside S_i
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("name", ["tiny_8x16x16", "dynamic_16x32x32", "dynamic_small_d64", "batch2"])
+def test_taylor_forward_parity(name):
+    if name == "dynamic_small_d64":
+        w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=3, head_dim=64, planted=2)
+    elif name == "batch2":  # two samples with their own block counts
+        w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=2, planted=2, batch=2)
+    else:
+        w = WORKLOADS[name]
+    inp = make_inputs(w, 13)
+    g = run_gpu(w, inp)
+    out = g["plan"].fwd(taylor=True)
+    for b in range(w.batch):
+        pl, bits = oracle_plan(w, inp, b=b)
+        compare_plan(w, pl, g["view"], b=b)
+        assert 0 < pl.cnt.min() and pl.cnt.max() < pl.nb  # blocks outside S_i exist
+        mx, rel = check_forward_taylor(w, g["plan"], pl, bits, 4096 if w.N <= 4096 else 1024, b=b, out=out)
+        # the acceptance bounds tell the Taylor output from the sparse one
+        z, r = np.zeros(512, np.int32), np.arange(512, dtype=np.int32)
+        O_s, _ = oracle.attn_fwd_rows(pl, *bits, z, r)
+        mx_s, rel_s = _err(out[0][b].float().cpu().numpy()[r, z], O_s)
+        assert mx_s > ATOL or rel_s > RTOL_L2, (mx_s, rel_s)
+        print(name, b, "taylor max-abs", mx, "rel-L2", rel)
+
+
+def test_taylor_with_every_block_selected_is_the_sparse_forward():
+    """No block outside S_i: every pooled column is masked, so the Taylor
+    forward is the sparse forward bit for bit (two samples)."""
+    w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=24, heads=2, top_k=10 ** 6, planted=1, batch=2)
+    inp = make_inputs(w, 14)
+    P = _lib()
+    plan = P.PrismPlan(P.params_for(w))
+    plan.build(*(x.cuda() for x in (inp.Q, inp.K, inp.V, inp.a)))
+    O_s, l_s = plan.fwd()
+    O_t, l_t = plan.fwd(taylor=True)
+    torch.cuda.synchronize()
+    plan.check()
+    assert torch.equal(O_s.view(torch.int16), O_t.view(torch.int16))
+    assert torch.equal(l_s, l_t)
+
+
+def test_taylor_leaves_the_backward_statistics_alone():
+    """prism_attn_fwd_taylor does not touch what prism_attn_bwd reads: the
+    gradients after fwd, fwd_taylor, bwd equal those after fwd, bwd (dK and
+    dV bit for bit; dQ, whose fp32 partial sums land in any order, in at least
+    nine elements of ten and within relative L2 2e-3 -- a Taylor LSE in place
+    of the sparse one would move nearly every element)."""
+    w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=16, heads=2, planted=1, backward=True)
+    inp = make_inputs(w, 15)
+    P = _lib()
+    plan = P.PrismPlan(P.params_for(w))
+    plan.build(*(x.cuda() for x in (inp.Q, inp.K, inp.V, inp.a)))
+    dO = inp.dO.cuda()
+    O, _ = plan.fwd()
+    ref = [t.clone() for t in plan.bwd(O, dO)]
+    plan.fwd(taylor=True)
+    got = plan.bwd(O, dO)
+    torch.cuda.synchronize()
+    plan.check()
+    for a, b in zip(ref[1:], got[1:]):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    same = (ref[0].view(torch.int16) == got[0].view(torch.int16)).double().mean().item()
+    dq0, dq1 = ref[0].double(), got[0].double()
+    rel = ((dq0 - dq1).norm() / dq0.norm()).item()
+    assert same >= 0.9 and rel <= 2e-3, (same, rel)
