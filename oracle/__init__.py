@@ -61,14 +61,18 @@ def _load():
             "orc_select_row": (_I, [_P, _I, _I, _D, _I, _P, _P]),
             "orc_cap": (_I, [_I, _I, _D]),
             "orc_select": (None, [_P, _P, _I, _I, _I, _I, _D, _D, _I, _P, _P, _P]),
-            "orc_attn_fwd_rows": (None, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _I,
+            "orc_attn_fwd_rows": (None, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I,
                                          _I, _P, _P, _P, _P]),
-            "orc_attn_fwd_taylor_rows": (None, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _I,
+            "orc_attn_fwd_taylor_rows": (None, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I,
                                                 _I, _P, _P, _P, _P]),
-            "orc_attn_bwd_dq_rows": (None, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P,
+            "orc_attn_bwd_dq_rows": (None, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P,
                                             _I, _I, _P, _P, _P]),
-            "orc_attn_bwd_dkv_rows": (None, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P,
+            "orc_attn_bwd_dkv_rows": (None, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P,
                                              _I, _I, _P, _P, _P, _P]),
+            "orc_pool_blocks": (None, [_P, _I, _I, _I, _P, _P, _P]),
+            "orc_hilbert_index": (ctypes.c_uint64, [_I, _I, _I, _I]),
+            "orc_hilbert_indices": (None, [_P, ctypes.c_longlong, _I, _P]),
+            "orc_hilbert_perm": (None, [_I, _I, _I, _P]),
             "orc_audio_norms": (None, [_P, _P, ctypes.c_longlong, _I]),
             "orc_num_threads": (_I, []),
         }
@@ -256,6 +260,78 @@ def plan(Q_bits, K_bits, V_bits, a, T, H, W, heads, D, k, p, max_frac=0.0,
                       Qb, Kb, cnt, cols, diag)
 
 
+def pool_blocks(X_bits: np.ndarray, heads: int, D: int, perm, blk_off) -> np.ndarray:
+    """fp64 means of blocks given as perm runs: [heads, nb, D]."""
+    X_bits = _c(X_bits, np.uint16)
+    perm = _c(perm, np.int32)
+    off = _c(blk_off, np.int32)
+    nb = off.shape[0] - 1
+    out = np.zeros((heads, nb, D))
+    _load().orc_pool_blocks(_ptr(X_bits), heads, D, nb, _ptr(perm), _ptr(off), _ptr(out))
+    return out
+
+
+def hilbert_indices(pts, k: int) -> np.ndarray:
+    """Hilbert index of each point (t, h, w) of the 2^k cube ([n, 3] ints)."""
+    pts = _c(pts, np.int32).reshape(-1, 3)
+    out = np.zeros(pts.shape[0], np.uint64)
+    _load().orc_hilbert_indices(_ptr(pts), ctypes.c_longlong(pts.shape[0]), k, _ptr(out))
+    return out
+
+
+def hilbert_perm(T: int, H: int, W: int) -> np.ndarray:
+    """Raster indices of the grid's tokens in the order of the Hilbert curve of
+    the smallest enclosing 2^k cube [DFSAttn page, first component]."""
+    p = np.zeros(T * H * W, np.int32)
+    _load().orc_hilbert_perm(T, H, W, _ptr(p))
+    return p
+
+
+@dataclass
+class HilbertPlan:
+    """Hilbert-order fixed-block plan: blocks are runs of `bsize` tokens of the
+    curve's order; pooling, selection and attention as in Prism's plan."""
+    T: int
+    H: int
+    W: int
+    heads: int
+    D: int
+    bsize: int
+    perm: np.ndarray
+    Qbar: np.ndarray
+    Kbar: np.ndarray
+    cnt: np.ndarray
+    cols: np.ndarray
+    diag: np.ndarray
+
+    @property
+    def nb(self) -> int:
+        return self.T * self.H * self.W // self.bsize
+
+    def blk_off(self) -> np.ndarray:
+        return np.arange(0, self.T * self.H * self.W + 1, self.bsize, dtype=np.int64)
+
+    def row_sets(self, h: int):
+        return [self.cols[h, i, : self.cnt[h, i]] for i in range(self.nb)]
+
+
+def plan_hilbert(Q_bits, K_bits, V_bits, T, H, W, heads, D, bsize, k, p, max_frac=0.0,
+                 with_select=True) -> HilbertPlan:
+    """Hilbert-order fixed-block plan for one sample (V is not needed: there are
+    no zone statistics).  *_bits: [N, heads, D] uint16 (bf16)."""
+    N = T * H * W
+    assert N % bsize == 0
+    pm = hilbert_perm(T, H, W)
+    off = np.arange(0, N + 1, bsize)
+    Qb = pool_blocks(Q_bits.reshape(N, heads, D), heads, D, pm, off)
+    Kb = pool_blocks(K_bits.reshape(N, heads, D), heads, D, pm, off)
+    if with_select:
+        cnt, cols, diag = select(Qb, Kb, k, p, max_frac)
+    else:
+        cnt = cols = diag = None
+    return HilbertPlan(T, H, W, heads, D, bsize, pm, Qb, Kb, cnt, cols, diag)
+
+
 def audio_norms(h_bits: np.ndarray) -> np.ndarray:
     """a_{t,h,w} = ||h^_{t,h,w}||_2 over the last axis of bf16 bits h_bits [..., C]
     (fp64, channel order) [Prism guide, Method section 1]."""
@@ -270,22 +346,25 @@ def audio_norms(h_bits: np.ndarray) -> np.ndarray:
 # --------------------------------------------------------------------------
 # Attention on requested outputs
 # --------------------------------------------------------------------------
-def _attn_args(pl: OraclePlan):
-    box = _c(pl.box, np.int32)
+def _attn_args(pl):
+    """Blocks as perm / blk_off runs, and the selection arrays, of a plan
+    (OraclePlan, HilbertPlan or any object with the same fields)."""
+    perm = _c(pl.perm, np.int32)
+    off = _c(pl.blk_off(), np.int32)
     cnt = _c(pl.cnt, np.int32)
     cols = _c(np.where(pl.cols < 0, 0, pl.cols), np.int32)
-    return box, cnt, cols, cols.shape[-1]
+    return perm, off, cnt, cols, cols.shape[-1]
 
 
 def attn_fwd_rows(pl: OraclePlan, Q_bits, K_bits, V_bits, req_h, req_tok):
     """O [n, D] and LSE [n] of query tokens req_tok (raster index) of heads req_h."""
-    box, cnt, cols, stride = _attn_args(pl)
+    perm, off, cnt, cols, stride = _attn_args(pl)
     req_h = _c(req_h, np.int32); req_tok = _c(req_tok, np.int32)
     n = req_h.shape[0]
     O = np.zeros((n, pl.D)); lse = np.zeros(n)
     Qb = _c(Q_bits, np.uint16); Kb = _c(K_bits, np.uint16); Vb = _c(V_bits, np.uint16)
     _load().orc_attn_fwd_rows(_ptr(Qb), _ptr(Kb), _ptr(Vb), pl.T, pl.H, pl.W, pl.heads, pl.D, pl.nb,
-                              _ptr(box), _ptr(cnt), _ptr(cols), stride, n, _ptr(req_h),
+                              _ptr(perm), _ptr(off), _ptr(cnt), _ptr(cols), stride, n, _ptr(req_h),
                               _ptr(req_tok), _ptr(O), _ptr(lse))
     return O, lse
 
@@ -294,36 +373,36 @@ def attn_fwd_taylor_rows(pl: OraclePlan, Q_bits, K_bits, V_bits, req_h, req_tok)
     """O [n, D] and LSE [n] with the blocks outside each S_i added through a
     zeroth-order Taylor term (pooled key, mean value, weight |B_j|)
     [In-Context Sparse Attention article, grouped computation]."""
-    box, cnt, cols, stride = _attn_args(pl)
+    perm, off, cnt, cols, stride = _attn_args(pl)
     req_h = _c(req_h, np.int32); req_tok = _c(req_tok, np.int32)
     n = req_h.shape[0]
     O = np.zeros((n, pl.D)); lse = np.zeros(n)
     Qb = _c(Q_bits, np.uint16); Kb = _c(K_bits, np.uint16); Vb = _c(V_bits, np.uint16)
     _load().orc_attn_fwd_taylor_rows(_ptr(Qb), _ptr(Kb), _ptr(Vb), pl.T, pl.H, pl.W, pl.heads, pl.D,
-                                     pl.nb, _ptr(box), _ptr(cnt), _ptr(cols), stride, n, _ptr(req_h),
+                                     pl.nb, _ptr(perm), _ptr(off), _ptr(cnt), _ptr(cols), stride, n, _ptr(req_h),
                                      _ptr(req_tok), _ptr(O), _ptr(lse))
     return O, lse
 
 
 def attn_bwd_dq_rows(pl: OraclePlan, Q_bits, K_bits, V_bits, dO_bits, req_h, req_tok):
-    box, cnt, cols, stride = _attn_args(pl)
+    perm, off, cnt, cols, stride = _attn_args(pl)
     req_h = _c(req_h, np.int32); req_tok = _c(req_tok, np.int32)
     n = req_h.shape[0]
     dQ = np.zeros((n, pl.D))
     arrs = [_c(x, np.uint16) for x in (Q_bits, K_bits, V_bits, dO_bits)]
     _load().orc_attn_bwd_dq_rows(*[_ptr(x) for x in arrs], pl.T, pl.H, pl.W, pl.heads, pl.D, pl.nb,
-                                 _ptr(box), _ptr(cnt), _ptr(cols), stride, n, _ptr(req_h),
+                                 _ptr(perm), _ptr(off), _ptr(cnt), _ptr(cols), stride, n, _ptr(req_h),
                                  _ptr(req_tok), _ptr(dQ))
     return dQ
 
 
 def attn_bwd_dkv_rows(pl: OraclePlan, Q_bits, K_bits, V_bits, dO_bits, req_h, req_tok):
-    box, cnt, cols, stride = _attn_args(pl)
+    perm, off, cnt, cols, stride = _attn_args(pl)
     req_h = _c(req_h, np.int32); req_tok = _c(req_tok, np.int32)
     n = req_h.shape[0]
     dK = np.zeros((n, pl.D)); dV = np.zeros((n, pl.D))
     arrs = [_c(x, np.uint16) for x in (Q_bits, K_bits, V_bits, dO_bits)]
     _load().orc_attn_bwd_dkv_rows(*[_ptr(x) for x in arrs], pl.T, pl.H, pl.W, pl.heads, pl.D, pl.nb,
-                                  _ptr(box), _ptr(cnt), _ptr(cols), stride, n, _ptr(req_h),
+                                  _ptr(perm), _ptr(off), _ptr(cnt), _ptr(cols), stride, n, _ptr(req_h),
                                   _ptr(req_tok), _ptr(dK), _ptr(dV))
     return dK, dV

@@ -47,6 +47,13 @@
  *                                                  the global mean of V; error of
  *                                                  second order in a zero-mean key
  *                                                  perturbation)
+ *   orc_hilbert_index, orc_hilbert_perm            pinned (a bijection of the cube
+ *                                                  whose consecutive points are unit
+ *                                                  steps and whose aligned sub-cubes
+ *                                                  are index intervals; the grid's
+ *                                                  order is by increasing index)
+ *   orc_pool_blocks                                pinned (block constants, index
+ *                                                  means, equal to orc_pool on boxes)
  *   orc_audio_norms                                pinned (closed forms: constant
  *                                                  rows, one-hot rows, integer
  *                                                  norms; an exact rational sum
@@ -356,6 +363,116 @@ void orc_pool(const uint16_t *X, int T, int H, int W, int heads, int D, int nb,
     }
 }
 
+/* Block means over blocks given as runs of a permutation: block j holds
+ * the tokens perm[blk_off[j]] ... perm[blk_off[j+1]-1].  X is [N][heads][D]
+ * bf16 bits; Xbar is [heads][nb][D].  The sum runs in block order. */
+void orc_pool_blocks(const uint16_t *X, int heads, int D, int nb, const int *perm,
+                     const int *blk_off, double *Xbar)
+{
+#pragma omp parallel for schedule(dynamic)
+    for (int j = 0; j < nb; ++j) {
+        double cnt = (double)(blk_off[j + 1] - blk_off[j]);
+        for (int hd = 0; hd < heads; ++hd)
+            for (int c = 0; c < D; ++c) {
+                double s = 0.0;
+                for (int m = blk_off[j]; m < blk_off[j + 1]; ++m)
+                    s += widen_bf16(X[((size_t)perm[m] * heads + hd) * D + c]);
+                Xbar[((size_t)hd * nb + j) * D + c] = s / cnt;
+            }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Hilbert-order fixed blocks [DFSAttn page, first component: tokens are     */
+/* reordered along a 3D Hilbert curve, so that tokens next to each other in  */
+/* the order are neighbours in space and time, and grouped into blocks].     */
+/*                                                                           */
+/* The curve is the one of the 2^k cube, k the smallest with 2^k >= T, H, W, */
+/* with the index of Skilling's method ("Programming the Hilbert curve",     */
+/* AIP Conf. Proc. 707, 2004): the coordinates (x0, x1, x2) = (t, h, w) go   */
+/* through the method's two passes -- for each bit level from the top, the   */
+/* lower bits of x0 are inverted (where x_i has that bit) or exchanged with  */
+/* those of x_i (where it does not); then a Gray encoding across the three   */
+/* coordinates -- and the index is read off the transformed coordinates bit  */
+/* level by bit level from the top, x0's bit first.  Reading: a grid that is */
+/* not a cube takes the cube's curve restricted to its tokens (the pages do  */
+/* not say how the curve meets a non-cube grid).                             */
+/* ------------------------------------------------------------------------ */
+uint64_t orc_hilbert_index(int t, int h, int w, int k)
+{
+    unsigned x[3] = {(unsigned)t, (unsigned)h, (unsigned)w};
+    if (k < 1)
+        return 0;
+    unsigned top = 1u << (k - 1);
+    /* pass 1: from the top bit level down to level 1 */
+    for (unsigned q = top; q > 1; q >>= 1) {
+        unsigned low = q - 1;
+        for (int i = 0; i < 3; ++i) {
+            if (x[i] & q) {
+                x[0] ^= low;
+            } else {
+                unsigned diff = (x[0] ^ x[i]) & low;
+                x[0] ^= diff;
+                x[i] ^= diff;
+            }
+        }
+    }
+    /* pass 2: Gray encoding */
+    x[1] ^= x[0];
+    x[2] ^= x[1];
+    unsigned flip = 0;
+    for (unsigned q = top; q > 1; q >>= 1)
+        if (x[2] & q)
+            flip ^= q - 1;
+    for (int i = 0; i < 3; ++i)
+        x[i] ^= flip;
+    /* interleave: bit levels from the top, x0 before x1 before x2 */
+    uint64_t idx = 0;
+    for (int b = k - 1; b >= 0; --b)
+        for (int i = 0; i < 3; ++i)
+            idx = (idx << 1) | ((x[i] >> b) & 1u);
+    return idx;
+}
+
+void orc_hilbert_indices(const int *pts /* [n][3] (t,h,w) */, long long n, int k, uint64_t *out)
+{
+#pragma omp parallel for schedule(static)
+    for (long long r = 0; r < n; ++r)
+        out[r] = orc_hilbert_index(pts[3 * r], pts[3 * r + 1], pts[3 * r + 2], k);
+}
+
+typedef struct {
+    uint64_t key;
+    int tok;
+} hkey_t;
+
+static int cmp_hkey(const void *pa, const void *pb)
+{
+    const hkey_t *a = (const hkey_t *)pa, *b = (const hkey_t *)pb;
+    return (a->key > b->key) - (a->key < b->key);
+}
+
+/* perm[n] = raster index of the n-th grid token along the curve. */
+void orc_hilbert_perm(int T, int H, int W, int *perm)
+{
+    int k = 0;
+    while ((1 << k) < T || (1 << k) < H || (1 << k) < W)
+        ++k;
+    size_t N = (size_t)T * H * W;
+    hkey_t *a = (hkey_t *)malloc(sizeof(hkey_t) * N);
+    for (int t = 0; t < T; ++t)
+        for (int h = 0; h < H; ++h)
+            for (int w = 0; w < W; ++w) {
+                size_t n = ((size_t)t * H + h) * W + w;
+                a[n].key = orc_hilbert_index(t, h, w, k);
+                a[n].tok = (int)n;
+            }
+    qsort(a, N, sizeof(hkey_t), cmp_hkey);
+    for (size_t n = 0; n < N; ++n)
+        perm[n] = a[n].tok;
+    free(a);
+}
+
 /* ------------------------------------------------------------------------ */
 /* Hybrid selection for one query block [Prism guide, Method section 3]:    */
 /*   P = softmax_j(z_j);  S = Top-k(P,k) U Top-p(P,p).                       */
@@ -489,32 +606,30 @@ void orc_select(const double *Qbar, const double *Kbar, int heads, int nb, int D
 /*   dQ_q = sum_t dS_qt k_t / sqrt(D),  dK_t = sum_q dS_qt q_q / sqrt(D),    */
 /*   dV_t = sum_q P_qt dO_q.                                                 */
 /* Tokens are raster indices; Q,K,V,dO are [N][heads][D] bf16 bits.  The    */
-/* selection is (cnt, cols, stride) as written by orc_select; box and nb    */
-/* describe the blocks.  Only requested outputs are computed.               */
+/* selection is (cnt, cols, stride) as written by orc_select; the blocks    */
+/* are given as perm / blk_off: block j holds the tokens perm[blk_off[j]],  */
+/* ..., perm[blk_off[j+1]-1], in that order (for zone blocks, raster order  */
+/* inside the box).  Only requested outputs are computed.                   */
 /* ------------------------------------------------------------------------ */
 typedef struct {
     const uint16_t *Q, *K, *V, *dO;
-    int H, W, heads, D, nb, stride;
-    const int *box, *cnt, *cols;
+    int heads, D, nb, stride;
+    const int *perm, *blk_off, *cnt, *cols;
     int *tok2blk;
 } attn_ctx;
 
-static void ctx_init(attn_ctx *cx, int T, int H, int W, int nb, const int *box)
+static void ctx_init(attn_ctx *cx, int T, int H, int W)
 {
     size_t N = (size_t)T * H * W;
     cx->tok2blk = (int *)malloc(sizeof(int) * N);
-    for (int j = 0; j < nb; ++j) {
-        const int *b = &box[6 * j];
-        for (int t = b[0]; t < b[0] + b[3]; ++t)
-            for (int h = b[1]; h < b[1] + b[4]; ++h)
-                for (int w = b[2]; w < b[2] + b[5]; ++w)
-                    cx->tok2blk[((size_t)t * H + h) * W + w] = j;
-    }
+    for (int j = 0; j < cx->nb; ++j)
+        for (int n = cx->blk_off[j]; n < cx->blk_off[j + 1]; ++n)
+            cx->tok2blk[cx->perm[n]] = j;
 }
 
 /* Scores of query token q (head hd) against every selected key token, in
- * the order: selected blocks ascending, tokens of a block raster.  Returns
- * the count; toks/s receive the key tokens and their scores. */
+ * the order: selected blocks ascending, tokens of a block in block order.
+ * Returns the count; toks/s receive the key tokens and their scores. */
 static int row_scores(const attn_ctx *cx, int hd, int q, int *toks, double *s)
 {
     int i = cx->tok2blk[q];
@@ -523,19 +638,16 @@ static int row_scores(const attn_ctx *cx, int hd, int q, int *toks, double *s)
     double sq = sqrt((double)cx->D);
     int n = 0;
     for (int u = 0; u < cx->cnt[r]; ++u) {
-        const int *b = &cx->box[6 * cl[u]];
-        for (int t = b[0]; t < b[0] + b[3]; ++t)
-            for (int h = b[1]; h < b[1] + b[4]; ++h)
-                for (int w = b[2]; w < b[2] + b[5]; ++w) {
-                    int kt = (t * cx->H + h) * cx->W + w;
-                    double dot = 0.0;
-                    for (int c = 0; c < cx->D; ++c)
-                        dot += widen_bf16(cx->Q[((size_t)q * cx->heads + hd) * cx->D + c]) *
-                               widen_bf16(cx->K[((size_t)kt * cx->heads + hd) * cx->D + c]);
-                    toks[n] = kt;
-                    s[n] = dot / sq;
-                    ++n;
-                }
+        for (int m = cx->blk_off[cl[u]]; m < cx->blk_off[cl[u] + 1]; ++m) {
+            int kt = cx->perm[m];
+            double dot = 0.0;
+            for (int c = 0; c < cx->D; ++c)
+                dot += widen_bf16(cx->Q[((size_t)q * cx->heads + hd) * cx->D + c]) *
+                       widen_bf16(cx->K[((size_t)kt * cx->heads + hd) * cx->D + c]);
+            toks[n] = kt;
+            s[n] = dot / sq;
+            ++n;
+        }
     }
     return n;
 }
@@ -553,13 +665,13 @@ static double row_lse(const double *s, int n)
 }
 
 void orc_attn_fwd_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
-                       int T, int H, int W, int heads, int D, int nb, const int *box,
-                       const int *cnt, const int *cols, int stride,
+                       int T, int H, int W, int heads, int D, int nb, const int *perm,
+                       const int *blk_off, const int *cnt, const int *cols, int stride,
                        int nreq, const int *req_h, const int *req_tok,
                        double *O /* [nreq][D] */, double *lse /* [nreq] */)
 {
-    attn_ctx cx = {Q, K, V, NULL, H, W, heads, D, nb, stride, box, cnt, cols, NULL};
-    ctx_init(&cx, T, H, W, nb, box);
+    attn_ctx cx = {Q, K, V, NULL, heads, D, nb, stride, perm, blk_off, cnt, cols, NULL};
+    ctx_init(&cx, T, H, W);
     size_t N = (size_t)T * H * W;
 #pragma omp parallel
     {
@@ -601,18 +713,18 @@ void orc_attn_fwd_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
 /* one softmax normalises both parts.  LSE is log of the whole normaliser.  */
 /* ------------------------------------------------------------------------ */
 void orc_attn_fwd_taylor_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
-                              int T, int H, int W, int heads, int D, int nb, const int *box,
-                              const int *cnt, const int *cols, int stride,
+                              int T, int H, int W, int heads, int D, int nb, const int *perm,
+                              const int *blk_off, const int *cnt, const int *cols, int stride,
                               int nreq, const int *req_h, const int *req_tok,
                               double *O /* [nreq][D] */, double *lse /* [nreq] */)
 {
-    attn_ctx cx = {Q, K, V, NULL, H, W, heads, D, nb, stride, box, cnt, cols, NULL};
-    ctx_init(&cx, T, H, W, nb, box);
+    attn_ctx cx = {Q, K, V, NULL, heads, D, nb, stride, perm, blk_off, cnt, cols, NULL};
+    ctx_init(&cx, T, H, W);
     size_t N = (size_t)T * H * W;
     double *Kbar = (double *)malloc(sizeof(double) * (size_t)heads * nb * D);
     double *Vbar = (double *)malloc(sizeof(double) * (size_t)heads * nb * D);
-    orc_pool(K, T, H, W, heads, D, nb, box, Kbar);
-    orc_pool(V, T, H, W, heads, D, nb, box, Vbar);
+    orc_pool_blocks(K, heads, D, nb, perm, blk_off, Kbar);
+    orc_pool_blocks(V, heads, D, nb, perm, blk_off, Vbar);
     double sq = sqrt((double)D);
 #pragma omp parallel
     {
@@ -650,7 +762,7 @@ void orc_attn_fwd_taylor_rows(const uint16_t *Q, const uint16_t *K, const uint16
                 l += exp(s[u] - mx);
             for (int j = 0; j < nb; ++j)
                 if (!in_s[j])
-                    l += (double)(box[6 * j + 3] * box[6 * j + 4] * box[6 * j + 5]) * exp(z[j] - mx);
+                    l += (double)(blk_off[j + 1] - blk_off[j]) * exp(z[j] - mx);
             double L = mx + log(l);
             for (int c = 0; c < D; ++c)
                 O[(size_t)r * D + c] = 0.0;
@@ -662,7 +774,7 @@ void orc_attn_fwd_taylor_rows(const uint16_t *Q, const uint16_t *K, const uint16
             for (int j = 0; j < nb; ++j) {
                 if (in_s[j])
                     continue;
-                double wt = (double)(box[6 * j + 3] * box[6 * j + 4] * box[6 * j + 5]) * exp(z[j] - L);
+                double wt = (double)(blk_off[j + 1] - blk_off[j]) * exp(z[j] - L);
                 for (int c = 0; c < D; ++c)
                     O[(size_t)r * D + c] += wt * Vbar[((size_t)hd * nb + j) * D + c];
             }
@@ -680,12 +792,12 @@ void orc_attn_fwd_taylor_rows(const uint16_t *Q, const uint16_t *K, const uint16
 
 void orc_attn_bwd_dq_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                           const uint16_t *dO, int T, int H, int W, int heads, int D, int nb,
-                          const int *box, const int *cnt, const int *cols, int stride,
+                          const int *perm, const int *blk_off, const int *cnt, const int *cols, int stride,
                           int nreq, const int *req_h, const int *req_tok,
                           double *dQ /* [nreq][D] */)
 {
-    attn_ctx cx = {Q, K, V, dO, H, W, heads, D, nb, stride, box, cnt, cols, NULL};
-    ctx_init(&cx, T, H, W, nb, box);
+    attn_ctx cx = {Q, K, V, dO, heads, D, nb, stride, perm, blk_off, cnt, cols, NULL};
+    ctx_init(&cx, T, H, W);
     size_t N = (size_t)T * H * W;
     double sq = sqrt((double)D);
 #pragma omp parallel
@@ -739,12 +851,12 @@ static int row_has(const int *cl, int n, int j)
 
 void orc_attn_bwd_dkv_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                            const uint16_t *dO, int T, int H, int W, int heads, int D, int nb,
-                           const int *box, const int *cnt, const int *cols, int stride,
+                           const int *perm, const int *blk_off, const int *cnt, const int *cols, int stride,
                            int nreq, const int *req_h, const int *req_tok,
                            double *dK /* [nreq][D] */, double *dV /* [nreq][D] */)
 {
-    attn_ctx cx = {Q, K, V, dO, H, W, heads, D, nb, stride, box, cnt, cols, NULL};
-    ctx_init(&cx, T, H, W, nb, box);
+    attn_ctx cx = {Q, K, V, dO, heads, D, nb, stride, perm, blk_off, cnt, cols, NULL};
+    ctx_init(&cx, T, H, W);
     size_t N = (size_t)T * H * W;
     double sq = sqrt((double)D);
     /* Query blocks whose selection holds a requested key token's block. */
@@ -796,25 +908,22 @@ void orc_attn_bwd_dkv_rows(const uint16_t *Q, const uint16_t *K, const uint16_t 
             size_t row = (size_t)hd * nb + i;
             if (!row_has(&cols[row * stride], cnt[row], j))
                 continue;
-            const int *b = &box[6 * i];
-            for (int t = b[0]; t < b[0] + b[3]; ++t)
-                for (int h = b[1]; h < b[1] + b[4]; ++h)
-                    for (int w = b[2]; w < b[2] + b[5]; ++w) {
-                        int q = (t * H + h) * W + w;
-                        double dot = 0.0, dpq = 0.0;
-                        for (int c = 0; c < D; ++c) {
-                            dot += widen_bf16(Q[((size_t)q * heads + hd) * D + c]) *
-                                   widen_bf16(K[((size_t)kt * heads + hd) * D + c]);
-                            dpq += widen_bf16(dO[((size_t)q * heads + hd) * D + c]) *
-                                   widen_bf16(V[((size_t)kt * heads + hd) * D + c]);
-                        }
-                        double pr = exp(dot / sq - L[(size_t)hd * N + q]);
-                        double ds = pr * (dpq - Dl[(size_t)hd * N + q]);
-                        for (int c = 0; c < D; ++c) {
-                            dv[c] += pr * widen_bf16(dO[((size_t)q * heads + hd) * D + c]);
-                            dk[c] += ds * widen_bf16(Q[((size_t)q * heads + hd) * D + c]) / sq;
-                        }
-                    }
+            for (int m = blk_off[i]; m < blk_off[i + 1]; ++m) {
+                int q = perm[m];
+                double dot = 0.0, dpq = 0.0;
+                for (int c = 0; c < D; ++c) {
+                    dot += widen_bf16(Q[((size_t)q * heads + hd) * D + c]) *
+                           widen_bf16(K[((size_t)kt * heads + hd) * D + c]);
+                    dpq += widen_bf16(dO[((size_t)q * heads + hd) * D + c]) *
+                           widen_bf16(V[((size_t)kt * heads + hd) * D + c]);
+                }
+                double pr = exp(dot / sq - L[(size_t)hd * N + q]);
+                double ds = pr * (dpq - Dl[(size_t)hd * N + q]);
+                for (int c = 0; c < D; ++c) {
+                    dv[c] += pr * widen_bf16(dO[((size_t)q * heads + hd) * D + c]);
+                    dk[c] += ds * widen_bf16(Q[((size_t)q * heads + hd) * D + c]) / sq;
+                }
+            }
         }
     }
     free(need);

@@ -431,7 +431,10 @@ def _random_selection(rs, heads, nb):
 
 def _taylor_plan(T, H, W, heads, D, box, cnt, cols):
     from types import SimpleNamespace
-    return SimpleNamespace(T=T, H=H, W=W, heads=heads, D=D, nb=len(box), box=box, cnt=cnt, cols=cols)
+    sizes = box[:, 3] * box[:, 4] * box[:, 5]
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+    return SimpleNamespace(T=T, H=H, W=W, heads=heads, D=D, nb=len(box), box=box, cnt=cnt, cols=cols,
+                           perm=oracle.perm(T, H, W, box), blk_off=lambda: off)
 
 
 def _dense(Qb, Kb, Vb, h):
@@ -534,6 +537,95 @@ def test_taylor_with_every_block_selected_is_the_sparse_forward():
     O_s, l_s = oracle.attn_fwd_rows(pl, Qb, Kb, Vb, rh, rt)
     np.testing.assert_array_equal(O_t, O_s)
     np.testing.assert_array_equal(l_t, l_s)
+
+
+# ---------------------------------------------------------------------------
+# Hilbert-order fixed blocks [DFSAttn page, first component]
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("k", [1, 2, 3, 4])
+def test_hilbert_index_is_a_hilbert_curve(k):
+    """On the 2^k cube the index is a bijection onto [0, 8^k), it starts at the
+    origin, consecutive points are one unit step apart (a Hamiltonian path of
+    the lattice), and every aligned 2^j sub-cube fills one interval of 8^j
+    consecutive indices (the recursive structure of the Hilbert curve)."""
+    S = 1 << k
+    pts = np.stack(np.meshgrid(np.arange(S), np.arange(S), np.arange(S), indexing="ij"), -1).reshape(-1, 3)
+    idx = oracle.hilbert_indices(pts, k).astype(np.int64)
+    assert np.array_equal(np.sort(idx), np.arange(S ** 3))
+    order = pts[np.argsort(idx)]
+    assert np.array_equal(order[0], [0, 0, 0])
+    steps = np.abs(np.diff(order, axis=0)).sum(axis=1)
+    assert np.all(steps == 1)
+    for j in range(1, k):
+        cube = (pts >> j)
+        cid = (cube[:, 0] * (S >> j) + cube[:, 1]) * (S >> j) + cube[:, 2]
+        for c in np.unique(cid):
+            sub = np.sort(idx[cid == c])
+            assert sub[-1] - sub[0] == 8 ** j - 1 and sub[0] % 8 ** j == 0
+
+
+def test_hilbert_perm_orders_the_grid_by_curve_index():
+    """A non-cube grid takes the enclosing cube's curve: perm is a bijection of
+    the tokens and their curve indices increase along it."""
+    T, H, W = 8, 16, 24
+    pm = oracle.hilbert_perm(T, H, W)
+    assert np.array_equal(np.sort(pm), np.arange(T * H * W))
+    t, h, w = pm // (H * W), (pm // W) % H, pm % W
+    idx = oracle.hilbert_indices(np.stack([t, h, w], -1), 5).astype(np.int64)
+    assert np.all(np.diff(idx) > 0)
+    # within the cube's first 8x16x16 octant pair the grid is whole: unit steps there
+    steps = np.abs(np.diff(np.stack([t, h, w], -1), axis=0)).sum(axis=1)
+    assert np.mean(steps == 1) > 0.95
+
+
+def test_pool_blocks_closed_forms():
+    """Means over perm runs: a field constant on each block gives the constant;
+    the field x = raster index gives the mean of the block's indices; on box
+    blocks it equals the box pooling."""
+    T, H, W, heads, D = 8, 16, 16, 2, 8
+    N = T * H * W
+    pm = oracle.hilbert_perm(T, H, W)
+    off = np.arange(0, N + 1, 128)
+    const = np.repeat(np.arange(N // 128, dtype=np.float32) * 0.5, 128)
+    X = np.zeros((N, heads, D), np.float32)
+    X[pm] = const[:, None, None]
+    got = oracle.pool_blocks(f32_bits(X), heads, D, pm, off)
+    np.testing.assert_array_equal(got, np.broadcast_to(const[::128][None, :, None], got.shape))
+    Xi = np.broadcast_to(np.arange(N, dtype=np.float32)[:, None, None], (N, heads, D)).copy()
+    Xi = Xi % 256  # exact in bf16
+    got = oracle.pool_blocks(f32_bits(Xi), heads, D, pm, off)
+    want = (pm % 256).reshape(-1, 128).mean(axis=1)
+    np.testing.assert_allclose(got[0, :, 0], want, rtol=0, atol=1e-12)
+    box, _ = _mixed_blocks(T, H, W)
+    pb = oracle.perm(T, H, W, box)
+    sizes = box[:, 3] * box[:, 4] * box[:, 5]
+    offb = np.concatenate([[0], np.cumsum(sizes)])
+    Xr = f32_bits(np.random.default_rng(3).normal(0, 1, (N, heads, D)))
+    np.testing.assert_array_equal(oracle.pool_blocks(Xr, heads, D, pb, offb),
+                                  oracle.pool(Xr, T, H, W, heads, D, box))
+
+
+def test_hilbert_plan_attention_equals_masked_dense():
+    """Selection and attention on Hilbert blocks: the sparse forward and its
+    gradients equal dense SDPA under the plan's token mask (fp64)."""
+    T, H, W, heads, D = 8, 16, 16, 2, 32
+    w = scaled(WORKLOADS["tiny_8x16x16"], heads=heads, head_dim=D)
+    inp = make_inputs(w, 4, with_grad_output=True)
+    Qb, Kb, Vb, dOb = (bf16_bits(x[0]) for x in (inp.Q, inp.K, inp.V, inp.dO))
+    pl = oracle.plan_hilbert(Qb, Kb, Vb, T, H, W, heads, D, 128, 2, 0.9)
+    assert pl.nb == 16 and 0 < pl.cnt.min() and pl.cnt.max() < pl.nb
+    N = T * H * W
+    for h in range(heads):
+        ref_o, ref_dq, ref_dk, ref_dv = _masked_dense(Qb, Kb, Vb, dOb, pl, h)
+        rh, rt = np.full(N, h, np.int32), np.arange(N, dtype=np.int32)
+        O, _ = oracle.attn_fwd_rows(pl, Qb, Kb, Vb, rh, rt)
+        np.testing.assert_allclose(O, ref_o, atol=1e-12, rtol=1e-9)
+        dQ = oracle.attn_bwd_dq_rows(pl, Qb, Kb, Vb, dOb, rh, rt)
+        np.testing.assert_allclose(dQ, ref_dq, atol=1e-11, rtol=1e-8)
+        sample = np.arange(0, N, 11, dtype=np.int32)
+        dK, dV = oracle.attn_bwd_dkv_rows(pl, Qb, Kb, Vb, dOb, np.full(len(sample), h, np.int32), sample)
+        np.testing.assert_allclose(dK, ref_dk[sample], atol=1e-11, rtol=1e-8)
+        np.testing.assert_allclose(dV, ref_dv[sample], atol=1e-11, rtol=1e-8)
 
 
 # ---------------------------------------------------------------------------
