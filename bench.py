@@ -191,7 +191,7 @@ def run_ours(args, rank, world, dev):
     w = workload_of(args)
     P.load_library()
     inp = make_inputs(w, seed=0, device=dev, with_grad_output=True)
-    plan = P.PrismPlan(P.params_for(w))
+    plan = P.PrismPlan(P.params_for(w, hilbert_block=args.hilbert))
     shp = inp.Q.shape
     O = torch.empty(shp, dtype=torch.bfloat16, device=dev)
     lse = torch.empty((w.batch, w.heads, w.N), dtype=torch.float32, device=dev)
@@ -375,6 +375,8 @@ def run_ours(args, rank, world, dev):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": w.name,
+                   "plan": (f"Hilbert order, fixed {args.hilbert}-token blocks" if args.hilbert else
+                            "Prism zones (dynamic volume and shape)"),
                    "pass": ("forward with the Taylor term for unselected blocks" if args.taylor else
                             "forward" if args.fwd_only else "forward+backward"),
                    "taylor_pooled_pairs": tpairs if args.taylor else None,
@@ -415,7 +417,7 @@ def traffic_for(kernel):
 # --------------------------------------------------------------------------
 # CPU oracle (baseline and reference arm)
 # --------------------------------------------------------------------------
-def oracle_setup(w, dev):
+def oracle_setup(w, dev, hilbert=0):
     import numpy as np
     import oracle
     from dynamic_block_sparse_zone_b200.synth import bf16_bits, make_inputs
@@ -424,8 +426,12 @@ def oracle_setup(w, dev):
     a = inp.a[0].cpu().numpy()
     del inp
     t0 = time.time()
-    pl = oracle.plan(bits[0], bits[1], bits[2], a, w.T, w.H, w.W, w.heads, w.head_dim, w.top_k,
-                     float(np.float32(w.top_p)), float(np.float32(w.max_frac)), with_select=False)
+    if hilbert:
+        pl = oracle.plan_hilbert(bits[0], bits[1], bits[2], w.T, w.H, w.W, w.heads, w.head_dim, hilbert, w.top_k,
+                                 float(np.float32(w.top_p)), float(np.float32(w.max_frac)), with_select=False)
+    else:
+        pl = oracle.plan(bits[0], bits[1], bits[2], a, w.T, w.H, w.W, w.heads, w.head_dim, w.top_k,
+                         float(np.float32(w.top_p)), float(np.float32(w.max_frac)), with_select=False)
     head = [0]
     cnt, cols, diag = oracle.select(pl.Qbar[head], pl.Kbar[head], w.top_k, float(np.float32(w.top_p)),
                                     float(np.float32(w.max_frac)))
@@ -444,9 +450,9 @@ def oracle_sample(pl, hb, w, rows, seed, taylor=False):
     rs = np.random.default_rng(seed)
     req_t = rs.integers(0, w.N, size=rows).astype(np.int32)
     req_h = np.zeros(rows, np.int32)
-    sizes = pl.box[:, 3] * pl.box[:, 4] * pl.box[:, 5]
-    tok2blk = np.empty(w.N, np.int64)
     off = pl.blk_off()
+    sizes = np.diff(off)
+    tok2blk = np.empty(w.N, np.int64)
     for j in range(pl.nb):
         tok2blk[pl.perm[off[j]:off[j + 1]]] = j
     keys = 0
@@ -466,9 +472,9 @@ def oracle_sample(pl, hb, w, rows, seed, taylor=False):
     return dt, 10.0 * w.head_dim * keys
 
 
-def cpu_baseline(w, dev, rows, taylor=False):
+def cpu_baseline(w, dev, rows, taylor=False, hilbert=0):
     import oracle
-    pl, hb, plan_s = oracle_setup(w, dev)
+    pl, hb, plan_s = oracle_setup(w, dev, hilbert)
     dt, fl = oracle_sample(pl, hb, w, rows, 123, taylor)
     what = "forward with the Taylor term" if taylor else "forward + dQ"
     return {"value": round(fl / dt / 1e12, 8), "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
@@ -480,7 +486,7 @@ def run_reference(args, dev):
     import oracle
     from dynamic_block_sparse_zone_b200.synth import WORKLOADS
     w = workload_of(args)
-    pl, hb, plan_s = oracle_setup(w, dev)
+    pl, hb, plan_s = oracle_setup(w, dev, args.hilbert)
     rows = args.ref_rows
     for s in range(args.warmup):
         oracle_sample(pl, hb, w, rows, 1000 + s)
@@ -512,6 +518,8 @@ def main():
     ap.add_argument("--fwd-only", action="store_true", help="step = plan + forward (forward-only workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true", help="time replays of the step captured in a CUDA graph")
+    ap.add_argument("--hilbert", type=int, default=0, choices=[0, 64, 128, 256],
+                    help="Hilbert-order plan with fixed blocks of this many tokens (the DFSAttn-style baseline)")
     ap.add_argument("--taylor", action="store_true",
                     help="forward with the zeroth-order Taylor term for the unselected blocks (implies --fwd-only)")
     ap.add_argument("--heads", type=int, default=0, help="override the workload's head count (profiling)")
@@ -545,7 +553,7 @@ def main():
         if world == 1 and not args.no_cpu_baseline:
             torch.cuda.empty_cache()
             from dynamic_block_sparse_zone_b200.synth import WORKLOADS
-            res["cpu_baseline"] = cpu_baseline(workload_of(args), dev, args.cpu_rows, args.taylor)
+            res["cpu_baseline"] = cpu_baseline(workload_of(args), dev, args.cpu_rows, args.taylor, args.hilbert)
         print(json.dumps(res), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -40,7 +40,8 @@ class prism_params(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
                 ("heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("top_k", ctypes.c_int),
                 ("top_p", ctypes.c_float), ("max_frac", ctypes.c_float), ("fixed_shape", ctypes.c_int * 3),
-                ("eps", ctypes.c_double), ("heads_total", ctypes.c_int), ("head_offset", ctypes.c_int)]
+                ("eps", ctypes.c_double), ("heads_total", ctypes.c_int), ("head_offset", ctypes.c_int),
+                ("hilbert_block", ctypes.c_int)]
 
 
 class prism_plan_view(ctypes.Structure):
@@ -162,11 +163,13 @@ class Params:
     eps: float = 1e-6
     heads_total: int = 0  # head sharding: this plan holds heads [head_offset, head_offset + heads)
     head_offset: int = 0
+    hilbert_block: int = 0  # 64/128/256: Hilbert-order fixed-block plan (DFSAttn-style baseline)
 
     def to_c(self) -> prism_params:
         return prism_params(self.batch, self.T, self.H, self.W, self.heads, self.head_dim, self.top_k,
                             float(self.top_p), float(self.max_frac), (ctypes.c_int * 3)(*self.fixed_shape),
-                            float(self.eps), int(self.heads_total), int(self.head_offset))
+                            float(self.eps), int(self.heads_total), int(self.head_offset),
+                            int(self.hilbert_block))
 
     @property
     def N(self) -> int:
@@ -207,11 +210,13 @@ class PrismPlan:
         return (p.batch, p.N, p.heads, p.head_dim)
 
     # -- the three hot-path calls ---------------------------------------------
-    def build(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, a_norm: torch.Tensor):
+    def build(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, a_norm: Optional[torch.Tensor]):
+        """a_norm may be None for a Hilbert-order plan (no zone statistics)."""
         p = self.params
         for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
             _need(t, n, torch.bfloat16, self._qkv_shape())
-        _need(a_norm, "a_norm", torch.float32, (p.batch, p.T, p.H, p.W))
+        if a_norm is not None or not p.hilbert_block:
+            _need(a_norm, "a_norm", torch.float32, (p.batch, p.T, p.H, p.W))
         _check(load_library().prism_plan_build(self._h, _ptr(Q), _ptr(K), _ptr(V), _ptr(a_norm), _stream()))
         return self
 
@@ -289,7 +294,9 @@ class PrismPlan:
         p = self.params
         shp = self._qkv_shape()
         host = [(Q, "Q", torch.bfloat16, shp), (K, "K", torch.bfloat16, shp), (V, "V", torch.bfloat16, shp),
-                (a_norm, "a_norm", torch.float32, (p.batch, p.T, p.H, p.W)), (O, "O", torch.bfloat16, shp)]
+                (O, "O", torch.bfloat16, shp)]
+        if a_norm is not None or not p.hilbert_block:  # a Hilbert-order plan does not read a_norm
+            host.append((a_norm, "a_norm", torch.float32, (p.batch, p.T, p.H, p.W)))
         if lse is not None:
             host.append((lse, "lse", torch.float32, (p.batch, p.heads, p.N)))
         if dO is not None:
@@ -420,7 +427,9 @@ def prism_plan_destroy(plan: PrismPlan):
     plan.close()
 
 
-def params_for(w, batch: Optional[int] = None) -> Params:
-    """Params of a synth.Workload."""
+def params_for(w, batch: Optional[int] = None, hilbert_block: int = 0) -> Params:
+    """Params of a synth.Workload (hilbert_block: the Hilbert-order fixed-block
+    plan with blocks of that many tokens instead of Prism's zone plan)."""
     return Params(batch=batch or w.batch, T=w.T, H=w.H, W=w.W, heads=w.heads, head_dim=w.head_dim,
-                  top_k=w.top_k, top_p=w.top_p, max_frac=w.max_frac, fixed_shape=tuple(w.fixed_shape))
+                  top_k=w.top_k, top_p=w.top_p, max_frac=w.max_frac,
+                  fixed_shape=(0, 0, 0) if hilbert_block else tuple(w.fixed_shape), hilbert_block=hilbert_block)

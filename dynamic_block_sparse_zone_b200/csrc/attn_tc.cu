@@ -33,9 +33,10 @@
 // streams the head's pooled keys kbar_j and mean values vbar_j (bf16, 128 per
 // chunk).  Block j then adds |B_j| exp2(x) with x its scaled pooled score: its
 // softmax column gets the bias log2 |B_j|, or -inf when j is in S_i (those
-// blocks are already exact) or past the last block.  Each softmax warp writes
-// the 128 biases of a chunk into its own shared buffer from a bitmask of S_i
-// that the CTA builds once; one online softmax covers both parts.
+// blocks are already exact) or past the last block.  The CTA first tabulates
+// log2 |B_j| of every key block in shared memory (one byte each, -1 for the
+// blocks of S_i); each softmax warp then turns a chunk's 128 entries into
+// float biases in its own buffer.  One online softmax covers both parts.
 #include <cuda.h>
 
 #include "tc_common.cuh"
@@ -62,10 +63,11 @@ struct Layout {
     static constexpr uint32_t kNumBars = 9;
     static constexpr uint32_t kBytes = kBars + kNumBars * 8 + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;  // slack to align the base to 1024
-    // Taylor variant: per-softmax-warp bias of a chunk, then the S_i bitmask
+    // Taylor variant: per-softmax-warp bias of a chunk, then the log2 |B_j|
+    // table (int8, -1 for the blocks of S_i)
     static constexpr uint32_t kBias = (kBytes + 15) & ~15u;
-    static constexpr uint32_t kMask = kBias + 4 * 128 * 4;
-    static uint32_t taylor_alloc(int nbmax) { return kMask + (((nbmax + 31) / 32 * 4 + 15) & ~15u) + 1024; }
+    static constexpr uint32_t kLg = kBias + 4 * 128 * 4;
+    static uint32_t taylor_alloc(int nbmax) { return kLg + ((nbmax + 15) & ~15u) + 1024; }
 };
 
 // Site codes recorded with a timeout.
@@ -111,9 +113,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int nseg_t = (nbb + 63) >> 6;
     const int nchunk_all = nchunk + ((nseg_t + 1) >> 1);
     auto chunk_full = [&](int c) { return c < nchunk ? (2 * c + 1) < nseg : (2 * (c - nchunk) + 1) < nseg_t; };
-    uint32_t *mask = reinterpret_cast<uint32_t *>(smem + L::kMask);
-    if constexpr (kTaylor)
-        for (int w = threadIdx.x; w < (nbb + 31) >> 5; w += kThreads) mask[w] = 0u;
+    int8_t *lg = reinterpret_cast<int8_t *>(smem + L::kLg);
+    if constexpr (kTaylor)  // block volumes are powers of two: log2 |B_j| is exact
+        for (int j = threadIdx.x; j < nbb; j += kThreads) lg[j] = (int8_t)(31 - __clz(bo[j + 1] - bo[j]));
 
     const uint32_t bar_q = sbase + L::kBars;
     const uint32_t bar_kf = bar_q + 8, bar_ke = bar_q + 16, bar_vf = bar_q + 24, bar_ve = bar_q + 32;
@@ -146,11 +148,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if constexpr (kTaylor) {  // S_i as a bitmask over the key blocks
-        for (int u = c_begin + threadIdx.x; u < c_end; u += kThreads) {
-            const int j = col[u];
-            atomicOr(&mask[j >> 5], 1u << (j & 31));
-        }
+    if constexpr (kTaylor) {  // the blocks of S_i are exact: no pooled term
+        for (int u = c_begin + threadIdx.x; u < c_end; u += kThreads) lg[col[u]] = -1;
         __syncthreads();
     }
     const uint32_t tmem = *tmem_slot;
@@ -261,10 +260,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int j = 128 * (c - nchunk) + 32 * e + lane;
-                    float bv = -INFINITY;
-                    // block volumes are powers of two: log2 |B_j| is exact
-                    if (j < nbb && !((mask[j >> 5] >> (j & 31)) & 1u)) bv = (float)(31 - __clz(bo[j + 1] - bo[j]));
-                    bias[32 * e + lane] = bv;
+                    const int v = j < nbb ? lg[j] : -1;
+                    bias[32 * e + lane] = v < 0 ? -INFINITY : (float)v;
                 }
                 __syncwarp();
             }

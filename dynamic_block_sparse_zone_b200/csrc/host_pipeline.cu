@@ -130,7 +130,8 @@ prism_status host_step(Plan &pl, const prism_host_io &io, cudaStream_t user, uns
     PRISM_CUDA_OK(cudaMemcpyAsync(hp.in[s][kQ], io.Q, qkv, cudaMemcpyHostToDevice, hp.h2d));
     PRISM_CUDA_OK(cudaMemcpyAsync(hp.in[s][kK], io.K, qkv, cudaMemcpyHostToDevice, hp.h2d));
     PRISM_CUDA_OK(cudaMemcpyAsync(hp.in[s][kV], io.V, qkv, cudaMemcpyHostToDevice, hp.h2d));
-    PRISM_CUDA_OK(cudaMemcpyAsync(hp.in[s][kA], io.a_norm, abytes, cudaMemcpyHostToDevice, hp.h2d));
+    if (io.a_norm)  // a Hilbert-order plan has no use for it
+        PRISM_CUDA_OK(cudaMemcpyAsync(hp.in[s][kA], io.a_norm, abytes, cudaMemcpyHostToDevice, hp.h2d));
     PRISM_CUDA_OK(cudaEventRecord(hp.in_ready[s], hp.h2d));
     if (bwd) {
         PRISM_CUDA_OK(cudaMemcpyAsync(hp.in[s][kdO], io.dO, qkv, cudaMemcpyHostToDevice, hp.h2d));

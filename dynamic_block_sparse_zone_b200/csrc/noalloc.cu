@@ -62,6 +62,7 @@ extern "C" PRISM_API prism_status prism_zone_shapes_noalloc(const prism_params *
     if (p->head_dim != 64 && p->head_dim != 128)
         return fail(PRISM_ERR_UNSUPPORTED, "head_dim %d unsupported (64 or 128)", p->head_dim);
     if ((uintptr_t)V & 15) return fail(PRISM_ERR_INVALID_ARG, "V must be 16-byte aligned");
+    if (p->hilbert_block) return fail(PRISM_ERR_UNSUPPORTED, "a Hilbert-order plan has no zone shapes");
     Geo g;
     g.batch = p->batch;
     g.T = p->T;

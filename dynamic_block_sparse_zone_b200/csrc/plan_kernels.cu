@@ -443,6 +443,9 @@ __device__ __forceinline__ int block_token(const Geo &g, const BlockGeom &bg, in
     return ((bg.t0 + tt) * g.H + (bg.h0 + hh)) * g.W + (bg.w0 + ww);
 }
 
+// kPerm: the blocks are runs of an existing permutation (Hilbert-order plans),
+// which is read instead of derived from the zone shapes and written.
+template <bool kPerm>
 __global__ void __launch_bounds__(384) k_permute_pool(const __nv_bfloat16 *__restrict__ Q,
                                                       const __nv_bfloat16 *__restrict__ K,
                                                       const __nv_bfloat16 *__restrict__ V, Geo g,
@@ -453,9 +456,17 @@ __global__ void __launch_bounds__(384) k_permute_pool(const __nv_bfloat16 *__res
                                                       double *__restrict__ Kbar) {
     const int j = blockIdx.x, b = blockIdx.y;
     if (j >= nb[b]) return;
-    const BlockGeom bg = block_geom(g, blk_off + (size_t)b * (g.nbmax + 1), zone_shape + (size_t)b * g.M, j);
-    for (int r = threadIdx.x; r < bg.B; r += blockDim.x)
-        perm[(size_t)b * g.N + bg.off + r] = block_token(g, bg, r);
+    BlockGeom bg;
+    if constexpr (kPerm) {
+        const int *bo = blk_off + (size_t)b * (g.nbmax + 1);
+        bg.off = bo[j];
+        bg.B = bo[j + 1] - bo[j];
+    } else {
+        bg = block_geom(g, blk_off + (size_t)b * (g.nbmax + 1), zone_shape + (size_t)b * g.M, j);
+        for (int r = threadIdx.x; r < bg.B; r += blockDim.x)
+            perm[(size_t)b * g.N + bg.off + r] = block_token(g, bg, r);
+    }
+    const int *pb = perm + (size_t)b * g.N + bg.off;
     const int G = g.C / 8;
     const double inv = 1.0 / (double)bg.B;  // B is a power of two: exact
     for (int grp = threadIdx.x; grp < G; grp += blockDim.x) {
@@ -470,7 +481,7 @@ __global__ void __launch_bounds__(384) k_permute_pool(const __nv_bfloat16 *__res
         const size_t dst0 = (bh * g.N + bg.off) * g.D + d0;
 #pragma unroll 4
         for (int r = 0; r < bg.B; ++r) {
-            const size_t tok = (size_t)block_token(g, bg, r);
+            const size_t tok = kPerm ? (size_t)pb[r] : (size_t)block_token(g, bg, r);
             const uint4 q = ld_stream(srcQ + tok * g.C);
             const uint4 k = ld_stream(srcK + tok * g.C);
             const uint4 v = ld_stream(srcV + tok * g.C);
@@ -948,7 +959,7 @@ __global__ void __launch_bounds__(256) k_csc_sort(size_t ncols, const int *__res
 // ---------------------------------------------------------------------------
 // host: launch the whole planner
 // ---------------------------------------------------------------------------
-static prism_status scan_into(const int *in, size_t n, int *out, int *tmp, cudaStream_t st) {
+prism_status scan_ints(const int *in, size_t n, int *out, int *tmp, cudaStream_t st) {
     const int nchunks = (int)((n + 1023) / 1024);
     k_scan_chunks<<<nchunks, 1024, 0, st>>>(in, (int)n, out, tmp);
     k_scan_totals<<<1, 1024, 0, st>>>(tmp, nchunks, out, (int)n);
@@ -974,8 +985,14 @@ prism_status launch_plan_stats(Plan &pl, const void *Vv, const float *a, cudaStr
     return PRISM_OK;
 }
 
+static prism_status launch_gather_select(Plan &pl, const __nv_bfloat16 *Q, const __nv_bfloat16 *K,
+                                        const __nv_bfloat16 *V, cudaStream_t st);
+
 prism_status launch_plan(Plan &pl, const void *Qv, const void *Kv, const void *Vv, const float *a,
                          cudaStream_t st) {
+    if (pl.p.hilbert_block)  // fixed order and blocks: gather, pool, select
+        return launch_gather_select(pl, static_cast<const __nv_bfloat16 *>(Qv),
+                                    static_cast<const __nv_bfloat16 *>(Kv), static_cast<const __nv_bfloat16 *>(Vv), st);
     prism_status s = launch_plan_stats(pl, Vv, a, st);
     return s == PRISM_OK ? launch_plan_finish(pl, Qv, Kv, Vv, st) : s;
 }
@@ -991,10 +1008,29 @@ prism_status launch_plan_finish(Plan &pl, const void *Qv, const void *Kv, const 
     k_zone_decide<<<g.batch, 1024, 0, st>>>(g, pl.zone_part, pl.zone_a, pl.p.eps, pl.fixed_idx,
                                             pl.zone_B, pl.zone_shape, pl.zone_blk0, pl.nb, pl.blk_off,
                                             pl.tile_blk, pl.zone_qt0, pl.nqt, pl.qt_row, pl.qt_blk); }
-    const int pp_threads = g.C / 8 >= 384 ? 384 : ((g.C / 8 + 31) / 32) * 32;
-    { TimerScope ts(pl, kTPermutePool, st);
-    k_permute_pool<<<dim3(g.nbmax, g.batch), pp_threads, 0, st>>>(Q, K, V, g, pl.nb, pl.blk_off, pl.zone_shape,
-                                                                   pl.perm, pl.Qp, pl.Kp, pl.Vp, pl.Qbar, pl.Kbar); }
+    return launch_gather_select(pl, Q, K, V, st);
+}
+
+static int permute_pool_threads(const Geo &g) { return g.C / 8 >= 384 ? 384 : ((g.C / 8 + 31) / 32) * 32; }
+
+static void launch_permute_pool(Plan &pl, const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
+                                cudaStream_t st) {
+    const Geo &g = pl.g;
+    TimerScope ts(pl, kTPermutePool, st);
+    if (pl.p.hilbert_block)
+        k_permute_pool<true><<<dim3(g.nbmax, g.batch), permute_pool_threads(g), 0, st>>>(
+            Q, K, V, g, pl.nb, pl.blk_off, pl.zone_shape, pl.perm, pl.Qp, pl.Kp, pl.Vp, pl.Qbar, pl.Kbar);
+    else
+        k_permute_pool<false><<<dim3(g.nbmax, g.batch), permute_pool_threads(g), 0, st>>>(
+            Q, K, V, g, pl.nb, pl.blk_off, pl.zone_shape, pl.perm, pl.Qp, pl.Kp, pl.Vp, pl.Qbar, pl.Kbar);
+}
+
+// The block-contiguous copies and pooled means, then scores, selection and
+// the CSR / CSC (the block table is in place).
+static prism_status launch_gather_select(Plan &pl, const __nv_bfloat16 *Q, const __nv_bfloat16 *K,
+                                        const __nv_bfloat16 *V, cudaStream_t st) {
+    const Geo &g = pl.g;
+    launch_permute_pool(pl, Q, K, V, st);
     PRISM_CUDA_OK(cudaGetLastError());
     const size_t rows = (size_t)g.batch * g.heads * g.nbmax;
     {
@@ -1018,12 +1054,12 @@ prism_status launch_plan_finish(Plan &pl, const void *Qv, const void *Kv, const 
     }
     PRISM_CUDA_OK(cudaGetLastError());
     TimerScope ts_csr(pl, kTCsr, st);
-    prism_status s = scan_into(pl.cnt, rows, pl.row_ptr, pl.scan_tmp, st);
+    prism_status s = scan_ints(pl.cnt, rows, pl.row_ptr, pl.scan_tmp, st);
     if (s != PRISM_OK) return s;
     PRISM_CUDA_OK(cudaMemsetAsync(pl.colT_cursor, 0, rows * sizeof(int), st));
     k_csr_compact<<<1184, 256, 0, st>>>(g, pl.cap_stride, pl.cnt, pl.cols_pad, pl.row_ptr, pl.col, pl.colT_cursor);
     PRISM_CUDA_OK(cudaGetLastError());
-    s = scan_into(pl.colT_cursor, rows, pl.colT_ptr, pl.scan_tmp, st);
+    s = scan_ints(pl.colT_cursor, rows, pl.colT_ptr, pl.scan_tmp, st);
     if (s != PRISM_OK) return s;
     PRISM_CUDA_OK(cudaMemsetAsync(pl.colT_cursor, 0, rows * sizeof(int), st));
     k_csc_fill<<<1184, 256, 0, st>>>(g, pl.row_ptr, pl.col, pl.colT_ptr, pl.colT_cursor, pl.rowT);
@@ -1045,16 +1081,11 @@ prism_status configure_plan_kernels(const Plan &pl) {
 }
 
 // Re-gathers new Q, K, V into the plan's block-contiguous copies with the
-// plan's existing block table (the selection is kept; the pooled means are
-// refreshed by the same kernel but not used again).
+// plan's existing block table (the selection is kept; the refreshed pooled
+// keys feed only the Taylor forward).
 prism_status launch_regather(Plan &pl, const void *Qv, const void *Kv, const void *Vv, cudaStream_t st) {
-    const Geo &g = pl.g;
-    const int pp_threads = g.C / 8 >= 384 ? 384 : ((g.C / 8 + 31) / 32) * 32;
-    TimerScope ts(pl, kTPermutePool, st);
-    k_permute_pool<<<dim3(g.nbmax, g.batch), pp_threads, 0, st>>>(
-        static_cast<const __nv_bfloat16 *>(Qv), static_cast<const __nv_bfloat16 *>(Kv),
-        static_cast<const __nv_bfloat16 *>(Vv), g, pl.nb, pl.blk_off, pl.zone_shape, pl.perm, pl.Qp, pl.Kp, pl.Vp,
-        pl.Qbar, pl.Kbar);
+    launch_permute_pool(pl, static_cast<const __nv_bfloat16 *>(Qv), static_cast<const __nv_bfloat16 *>(Kv),
+                        static_cast<const __nv_bfloat16 *>(Vv), st);
     PRISM_CUDA_OK(cudaGetLastError());
     return PRISM_OK;
 }

@@ -102,6 +102,13 @@ static prism_status check_params(const prism_params *p, Geo *g, int *fixed_idx, 
         return fail(PRISM_ERR_UNSUPPORTED, "selection too large for 32-bit CSR offsets (%lld x %d)", rows, *cap_stride);
     if ((long long)g->batch * g->heads * g->N * g->D >= (1ll << 40))
         return fail(PRISM_ERR_UNSUPPORTED, "tensors too large");
+    if (p->hilbert_block) {
+        if (p->hilbert_block != 64 && p->hilbert_block != 128 && p->hilbert_block != 256)
+            return fail(PRISM_ERR_INVALID_ARG, "hilbert_block must be 0, 64, 128 or 256");
+        if (fs[0] || fs[1] || fs[2]) return fail(PRISM_ERR_INVALID_ARG, "hilbert_block and fixed_shape exclude each other");
+        if (hilbert_level(*g) > 9)
+            return fail(PRISM_ERR_UNSUPPORTED, "Hilbert order: grid side above 512 (the cube's flags would exceed 2^27)");
+    }
     const double head_scores = (double)g->nbmax * g->nbmax * 8.0;  // bytes of one head's block scores
     if (head_scores > 2.0 * (1ull << 30))
         return fail(PRISM_ERR_UNSUPPORTED, "too many blocks for the score scratch (%d blocks per sample)", g->nbmax);
@@ -297,6 +304,7 @@ prism_status prism_plan_create(const prism_params *params, prism_plan **out) {
     if (s == PRISM_OK) s = configure_attn_tc_kernels();
     if (s == PRISM_OK) s = configure_attn_bwd_tc_kernels();
     if (s == PRISM_OK) s = make_tensor_maps(pl);
+    if (s == PRISM_OK && pl.p.hilbert_block) s = setup_hilbert_plan(pl);
 
     if (s != PRISM_OK) {
         release_buffers(pl);
@@ -324,12 +332,13 @@ static prism_status device_guard(const Plan &pl) {
 prism_status prism_plan_build(prism_plan *plan, const void *Q, const void *K, const void *V, const float *a_norm,
                               void *stream) {
     g_last_error.clear();
-    if (!plan || !Q || !K || !V || !a_norm) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_plan_build");
+    if (!plan || !Q || !K || !V || (!a_norm && !plan->pl.p.hilbert_block))
+        return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_plan_build");
     prism_status s = device_guard(plan->pl);
     if (s != PRISM_OK) return s;
     const uintptr_t al = (uintptr_t)Q | (uintptr_t)K | (uintptr_t)V;
     if (al & 15) return fail(PRISM_ERR_INVALID_ARG, "Q, K, V must be 16-byte aligned");
-    if (plan->pl.g.Ctot != plan->pl.g.C)
+    if (plan->pl.g.Ctot != plan->pl.g.C && !plan->pl.p.hilbert_block)
         return fail(PRISM_ERR_STATE, "a head-sharded plan is built with build_stats, an exchange and build_finish");
     plan->pl.have_fwd = false;
     s = launch_plan(plan->pl, Q, K, V, a_norm, static_cast<cudaStream_t>(stream));
@@ -343,6 +352,8 @@ prism_status prism_plan_build_stats(prism_plan *plan, const void *V, const float
     prism_status s = device_guard(plan->pl);
     if (s != PRISM_OK) return s;
     if ((uintptr_t)V & 15) return fail(PRISM_ERR_INVALID_ARG, "V must be 16-byte aligned");
+    if (plan->pl.p.hilbert_block)
+        return fail(PRISM_ERR_STATE, "a Hilbert-order plan has no zone statistics: build it with prism_plan_build");
     plan->pl.have_fwd = false;
     plan->pl.built = false;
     s = launch_plan_stats(plan->pl, V, a_norm, static_cast<cudaStream_t>(stream));
@@ -411,7 +422,7 @@ prism_status prism_attn_fwd_taylor(prism_plan *plan, void *O, float *lse, void *
     if (!plan->pl.built) return fail(PRISM_ERR_STATE, "prism_attn_fwd_taylor needs a built plan");
     if ((uintptr_t)O & 15) return fail(PRISM_ERR_INVALID_ARG, "O must be 16-byte aligned");
     if (!taylor_fits(plan->pl.g))
-        return fail(PRISM_ERR_UNSUPPORTED, "too many blocks for the Taylor forward's shared-memory bitmask");
+        return fail(PRISM_ERR_UNSUPPORTED, "too many key blocks for the Taylor forward's shared-memory table");
     return launch_attn_fwd_taylor(plan->pl, O, lse, static_cast<cudaStream_t>(stream));
 }
 
@@ -439,12 +450,12 @@ prism_status prism_audio_norms(const void *h, float *a, int batch, int T, int H,
 prism_status prism_step_host(prism_plan *plan, const prism_host_io *io, void *stream, unsigned long long *ticket) {
     g_last_error.clear();
     if (!plan || !io || !ticket) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_step_host");
-    if (!io->Q || !io->K || !io->V || !io->a_norm || !io->O)
+    if (!io->Q || !io->K || !io->V || (!io->a_norm && !plan->pl.p.hilbert_block) || !io->O)
         return fail(PRISM_ERR_INVALID_ARG, "prism_step_host needs Q, K, V, a_norm and O");
     if (io->dO && (!io->dQ || !io->dK || !io->dV))
         return fail(PRISM_ERR_INVALID_ARG, "prism_step_host with dO needs dQ, dK and dV");
-    if (plan->pl.g.Ctot != plan->pl.g.C)
-        return fail(PRISM_ERR_STATE, "prism_step_host runs unsharded plans only");
+    if (plan->pl.g.Ctot != plan->pl.g.C && !plan->pl.p.hilbert_block)
+        return fail(PRISM_ERR_STATE, "prism_step_host runs unsharded zone plans only");
     prism_status s = device_guard(plan->pl);
     if (s != PRISM_OK) return s;
     return host_step(plan->pl, *io, static_cast<cudaStream_t>(stream), ticket);

@@ -126,6 +126,15 @@ prism_status launch_attn_bwd(Plan &pl, const void *O, const void *dO, void *dQ, 
 
 prism_status launch_audio_norms(const void *h, float *a, long long rows, int C, cudaStream_t st);
 
+// Exclusive scan of n ints into out[0..n] (out[n] = total); tmp holds
+// (n + 1023) / 1024 + 1 ints.
+prism_status scan_ints(const int *in, size_t n, int *out, int *tmp, cudaStream_t st);
+
+// Hilbert-order fixed-block plans (hilbert_plan.cu): the curve's level k
+// (2^k >= T, H, W) and the one-time order and block tables of a new plan.
+int hilbert_level(const Geo &g);
+prism_status setup_hilbert_plan(Plan &pl);
+
 // Host-buffer steps (host_pipeline.cu).
 prism_status host_step(Plan &pl, const prism_host_io &io, cudaStream_t user, unsigned long long *ticket);
 prism_status host_step_join(Plan &pl, unsigned long long ticket, cudaStream_t st);

@@ -73,7 +73,17 @@ typedef enum prism_status {
  *   those heads, and the plan is built in two halves around one exchange of
  *   zone statistics between the ranks (prism_plan_build_stats,
  *   prism_plan_stats_slice, prism_plan_build_finish); heads * head_dim and
- *   head_offset * head_dim must be multiples of 128.                       */
+ *   head_offset * head_dim must be multiples of 128.  (A Hilbert-order plan
+ *   needs no exchange: it is built with prism_plan_build on any shard.)
+ * hilbert_block: 0 = Prism's zone plan.  64, 128 or 256 = the comparison
+ *   baseline of the DFSAttn page's first component: tokens ordered along
+ *   the 3D Hilbert curve of the smallest 2^k cube holding the grid (Skilling's
+ *   index, t before h before w; the grid's tokens in the cube's curve order),
+ *   blocks of hilbert_block consecutive tokens of that order, then Prism's
+ *   pooled scoring, selection and attention.  No zone statistics: a_norm and
+ *   fixed_shape are unused (fixed_shape must be {0,0,0}); the grid's longest
+ *   side must be at most 512.  The order is computed once by
+ *   prism_plan_create (which then synchronises the device).                */
 typedef struct prism_params {
     int batch, T, H, W, heads, head_dim;
     int top_k;
@@ -82,6 +92,7 @@ typedef struct prism_params {
     int fixed_shape[3];
     double eps;
     int heads_total, head_offset;
+    int hilbert_block;
 } prism_params;
 
 typedef struct prism_plan prism_plan;
@@ -91,7 +102,9 @@ typedef struct prism_plan prism_plan;
  * NBMAX = N/64 is the most blocks a sample can have; every per-block array is
  * sized for it, entries past a sample's n_blocks are unspecified.
  *   zone_B      int [batch][N/512]      block volume B(m) in {64,128,256}
- *   zone_shape  int [batch][N/512]      index into the 16-entry candidate
+ *                                       (0 in a Hilbert-order plan)
+ *   zone_shape  int [batch][N/512]      (-1 in a Hilbert-order plan)
+ *                                       index into the 16-entry candidate
  *                                       table (volume 64: 0-6, 128: 7-12,
  *                                       256: 13-15; lexicographic (bT,bH,bW))
  *   perm        int [batch][N]          perm[n_new] = raster index of the
@@ -184,8 +197,9 @@ PRISM_API prism_status prism_attn_fwd(prism_plan *plan, void *O, float *lse, voi
  * permuted V of the last build or update; enqueues a pooling kernel and the
  * attention kernel.  It leaves the statistics that prism_attn_bwd uses
  * untouched: the backward differentiates the sparse forward only.
- * PRISM_ERR_UNSUPPORTED when the bitmask of S_i (one bit per key block)
- * does not fit a CTA's shared memory (more than about 1.6 million blocks). */
+ * PRISM_ERR_UNSUPPORTED when the per-CTA table of key blocks (one byte
+ * each) does not fit a CTA's shared memory (more than about 128 thousand
+ * blocks, i.e. over 8 million tokens per sample).                          */
 PRISM_API prism_status prism_attn_fwd_taylor(prism_plan *plan, void *O, float *lse, void *stream);
 
 /* Gradient of sum(O * dO) with respect to Q, K, V through the same sparse

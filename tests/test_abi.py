@@ -62,6 +62,10 @@ def test_plan_bytes_and_validation(lib):
     assert prism_plan_bytes(_params(top_p=1.5)) == 0
     assert prism_plan_bytes(_params(fixed_shape=(4, 4, 2))) == 0   # volume 32: not a candidate
     assert prism_plan_bytes(_params(fixed_shape=(4, 4, 4))) > 0
+    assert prism_plan_bytes(_params(hilbert_block=128)) > 0          # Hilbert-order baseline
+    assert prism_plan_bytes(_params(hilbert_block=96)) == 0          # not 64 / 128 / 256
+    assert prism_plan_bytes(_params(hilbert_block=64, fixed_shape=(4, 4, 4))) == 0
+    assert prism_plan_bytes(_params(T=8, H=8, W=1024, hilbert_block=64)) == 0   # cube side 1024 > 512
 
 
 def test_create_rejects_bad_params_before_touching_the_device(lib):

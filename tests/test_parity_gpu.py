@@ -729,3 +729,110 @@ def test_taylor_leaves_the_backward_statistics_alone():
     dq0, dq1 = ref[0].double(), got[0].double()
     rel = ((dq0 - dq1).norm() / dq0.norm()).item()
     assert same >= 0.9 and rel <= 2e-3, (same, rel)
+
+
+# ---------------------------------------------------------------------------
+# Hilbert-order fixed-block plans (the DFSAttn-style baseline)
+# ---------------------------------------------------------------------------
+def oracle_hilbert_plan(w, inp, bsize, b=0, heads=None):
+    Qb, Kb, Vb = (bf16_bits(x[b]) for x in (inp.Q, inp.K, inp.V))
+    sel = heads is None
+    pl = oracle.plan_hilbert(Qb, Kb, Vb, w.T, w.H, w.W, w.heads, w.head_dim, bsize, w.top_k, _f32(w.top_p),
+                             _f32(w.max_frac), with_select=sel)
+    if not sel:
+        cnt, cols, diag = oracle.select(pl.Qbar[heads], pl.Kbar[heads], w.top_k, _f32(w.top_p), _f32(w.max_frac))
+        pl.cnt, pl.cols, pl.diag = cnt, cols, diag
+    return pl, (Qb, Kb, Vb)
+
+
+def compare_hilbert_plan(w, pl, view, b=0, heads=None):
+    """Order and block table exact; selection exact up to counted near-ties."""
+    assert np.all(view["zone_B"][b].cpu().numpy() == 0) and np.all(view["zone_shape"][b].cpu().numpy() == -1)
+    np.testing.assert_array_equal(view["perm"][b].cpu().numpy(), pl.perm)
+    assert view["n_blocks"][b] == pl.nb
+    np.testing.assert_array_equal(view["blk_off"][b, : pl.nb + 1].cpu().numpy(), pl.blk_off())
+    rp = view["row_ptr"].cpu().numpy()
+    col = view["col_idx"].cpu().numpy()
+    nbmax = view["nbmax"]
+    ties = 0
+    for hi, h in enumerate(range(w.heads) if heads is None else heads):
+        for i in range(pl.nb):
+            r = (b * w.heads + h) * nbmax + i
+            g_set = col[rp[r]:rp[r + 1]]
+            o_set = pl.cols[hi, i, : pl.cnt[hi, i]]
+            if len(g_set) != len(o_set) or np.any(g_set != o_set):
+                d = pl.diag[hi, i]
+                assert d[0] < TIE or d[1] < TIE, f"head {h} row {i}: selection differs without a near-tie"
+                ties += 1
+    return ties
+
+
+def run_gpu_hilbert(w, inp, bsize, backward=False, with_a=True):
+    P = _lib()
+    plan = P.PrismPlan(P.params_for(w, batch=inp.Q.shape[0], hilbert_block=bsize))
+    Q, K, V = (x.cuda() for x in (inp.Q, inp.K, inp.V))
+    plan.build(Q, K, V, inp.a.cuda() if with_a else None)
+    O, lse = plan.fwd()
+    out = dict(O=O, lse=lse, plan=plan)
+    if backward:
+        out["dQ"], out["dK"], out["dV"] = plan.bwd(O, inp.dO.cuda())
+    torch.cuda.synchronize()
+    plan.check()
+    out["view"] = plan.view()
+    return out
+
+
+@pytest.mark.parametrize("name,bsize", [("tiny_8x16x16", 64), ("dynamic_16x32x32", 128),
+                                        ("dynamic_small_d64", 256), ("batch2", 128)])
+def test_hilbert_plan_forward_backward_parity(name, bsize):
+    if name == "dynamic_small_d64":
+        w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=40, heads=3, head_dim=64, planted=2)
+    elif name == "batch2":
+        w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=24, W=32, heads=2, planted=2, batch=2)
+    else:
+        w = WORKLOADS[name]
+    w = scaled(w, backward=True)
+    inp = make_inputs(w, 17)
+    g = run_gpu_hilbert(w, inp, bsize, backward=True, with_a=(name != "tiny_8x16x16"))
+    for b in range(w.batch):
+        pl, bits = oracle_hilbert_plan(w, inp, bsize, b=b)
+        compare_hilbert_plan(w, pl, g["view"], b=b)
+        assert 0 < pl.cnt.min() and pl.cnt.max() < pl.nb
+        check_forward(w, inp, g, pl, bits, 1024, b=b)
+        dOb = bf16_bits(inp.dO[b])
+        rs = np.random.default_rng(8)
+        req_h, req_t = sample_rows(rs, w, 256)
+        dQ_ref = oracle.attn_bwd_dq_rows(pl, *bits, dOb, req_h, req_t)
+        assert_close("dQ", g["dQ"][b].float().cpu().numpy()[req_t, req_h], dQ_ref)
+        req_h, req_t = pick_dkv_rows(pl, 0, 2, 8, rs)
+        dK_ref, dV_ref = oracle.attn_bwd_dkv_rows(pl, *bits, dOb, req_h, req_t)
+        assert_close("dK", g["dK"][b].float().cpu().numpy()[req_t, req_h], dK_ref)
+        assert_close("dV", g["dV"][b].float().cpu().numpy()[req_t, req_h], dV_ref)
+        check_forward_taylor(w, g["plan"], pl, bits, 512, b=b)
+
+
+def test_hilbert_plan_rejections():
+    P = _lib()
+    w = WORKLOADS["tiny_8x16x16"]
+    with pytest.raises(P.PrismError):
+        P.PrismPlan(P.Params(1, 8, 16, 16, 2, 64, 2, 0.9, hilbert_block=96))
+    with pytest.raises(P.PrismError):
+        P.PrismPlan(P.Params(1, 8, 16, 16, 2, 64, 2, 0.9, fixed_shape=(4, 4, 4), hilbert_block=64))
+    plan = P.PrismPlan(P.params_for(w, hilbert_block=64))
+    inp = make_inputs(w, 2)
+    with pytest.raises(P.PrismError):  # no zone statistics in a Hilbert-order plan
+        plan.build_stats(inp.V.cuda(), inp.a.cuda())
+
+
+@pytest.mark.slow
+def test_hilbert_plan_2k_full_size():
+    """The 2K grid with 128-token Hilbert blocks: order exact, selection of one
+    head exact up to near-ties, forward on sampled rows of that head."""
+    w = WORKLOADS["latent2k_24x96x160"]
+    inp = make_inputs(w, 0, device="cuda")
+    g = run_gpu_hilbert(w, inp, 128)
+    heads = [3]
+    pl, bits = oracle_hilbert_plan(w, inp, 128, heads=heads)
+    ties = compare_hilbert_plan(w, pl, g["view"], heads=heads)
+    check_forward(w, inp, g, pl, bits, 128, heads=heads)
+    print("2K Hilbert near-ties", ties, "blocks", pl.nb)
