@@ -7,9 +7,12 @@
 //   P = exp(S*scale - LSE), dP = dO V^T, dS = P (dP - Delta),
 //   dV = P^T dO, dK = scale dS^T Q, dQ = scale dS K.
 //
-// Work unit: one 128-key tile of one head (a 64-token key block fills the
-// upper half with rows it ignores).  The CTA walks the query blocks of the
-// key block's CSC column as 64-row chunks.
+// Work unit: one 128-key tile of one head (a 256-token key block gives two,
+// a 128-token block one, and two consecutive 64-token blocks j, j+1 share
+// one).  The CTA walks the query blocks of the key block's CSC column as
+// 64-row chunks; a shared tile walks the union of its two columns, and the
+// key rows of a block whose column lacks the chunk's query block (a whole
+// warp's rows) take P = dS = 0 for that chunk.
 //
 // Per chunk c:
 //   S^T  = K Q_c^T         M=128 keys, N=64 queries   -> TMEM ST[c%3]
@@ -69,7 +72,9 @@ struct Layout {
     static constexpr uint32_t kBars = kDQ + 64 * D * 4;
     // kv, q_full[3], q_empty[3], s_full[2], p_full[2], dq_full[3], dq_empty[3], done
     static constexpr uint32_t kNumBars = 18;
-    static constexpr uint32_t kBytes = kBars + kNumBars * 8 + 16;
+    // then per stage the column mask of its query chunk in a shared tile
+    static constexpr uint32_t kMaskS = kBars + kNumBars * 8 + 16;
+    static constexpr uint32_t kBytes = kMaskS + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;
     static_assert(kAlloc <= 232448, "shared memory per block");
     static_assert(kDQ % 128 == 0, "TMA source alignment");
@@ -108,18 +113,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int *bo = blk_off + (size_t)b * (g.nbmax + 1);
     const int k0 = qt_row[(size_t)b * g.nbmax + tile];
-    const int jblk = qt_blk[(size_t)b * g.nbmax + tile];
-    const int kvalid = min(128, bo[jblk + 1] - k0);
+    int jblk, jblk2;
+    tile_blocks(qt_blk[(size_t)b * g.nbmax + tile], jblk, jblk2);
+    const bool shared_tile = jblk2 >= 0;
+    const int kvalid = min(128, bo[(shared_tile ? jblk2 : jblk) + 1] - k0);
     const size_t colid = (size_t)bh * g.nbmax + jblk;
     const int u_begin = colT_ptr[colid], u_end = colT_ptr[colid + 1];
+    // the second key block's column (empty unless the tile is shared)
+    const int u2_begin = shared_tile ? colT_ptr[colid + 1] : 0, u2_end = shared_tile ? colT_ptr[colid + 2] : 0;
 
-    int nchunk = 0;  // 64-row query chunks of the column
-    for (int u = u_begin + lane; u < u_end; u += 32) {
-        const int i = rowT[u];
-        nchunk += (bo[i + 1] - bo[i]) >> 6;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) nchunk += __shfl_xor_sync(0xffffffffu, nchunk, o);
+    // 64-row query chunks of the column(s)
+    const int nchunk = union_segments(rowT + u_begin, u_end - u_begin, rowT + u2_begin, u2_end - u2_begin, bo, lane);
 
     const uint32_t bar_kv = sbase + L::kBars;
     const uint32_t bar_qf = bar_kv + 8, bar_qe = bar_qf + 8 * kStages, bar_sf = bar_qe + 8 * kStages;
@@ -127,6 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_done = bar_de + 8 * kStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBars + L::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kBars + L::kNumBars * 8 + 8);
+    volatile uint32_t *mask_s = reinterpret_cast<volatile uint32_t *>(smem + L::kMaskS);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -171,11 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(sbase + L::kV + hf * L::kKVHalf + rh * 8192, &tmV, bar_kv, hf * 64,
                                 rowbase + k0 + rh * 64);
                 }
-            int u = u_begin, r = 0, r_end = 0;
-            if (u < u_end) {
-                r = bo[rowT[u]];
-                r_end = bo[rowT[u] + 1];
-            }
+            SegWalk wk;
+            wk.init(u_begin, u_end, u2_begin, u2_end, rowT, bo);
             int issued = 0;
             for (int c = 0; c < nchunk; ++c) {
                 const int st = c % kStages;
@@ -185,6 +187,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + L::kHalves * L::kQHalf;
                 const uint32_t sVec = sbase + L::kVec + st * 512;
                 const uint32_t bar = bar_qf + 8 * st;
+                const int r = wk.r;
+                mask_s[st] = (uint32_t)wk.mask;  // published by the arrive below
                 mbar_expect_tx(bar, 2 * 64 * D * 2 + 512);
                 for (int hf = 0; hf < L::kHalves; ++hf) {
                     tma_load_2d(sQ + hf * L::kQHalf, &tmQ, bar, hf * 64, rowbase + r);
@@ -193,11 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bulk_load(sVec, nlse_p + (size_t)rowbase + r, 256, bar);
                 bulk_load(sVec + 256, delta + (size_t)rowbase + r, 256, bar);
                 issued = c + 1;
-                r += 64;
-                if (r >= r_end && ++u < u_end) {
-                    r = bo[rowT[u]];
-                    r_end = bo[rowT[u] + 1];
-                }
+                wk.advance(rowT, bo);
             }
             for (int c = max(0, issued - kStages); c < issued; ++c)
                 mbar_wait(bar_qf + 8 * (c % kStages), (c / kStages) & 1, status, kSiteQFull, abort_flag);
@@ -263,6 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int rowid = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const bool live = rowid < kvalid;
+        const int half = shared_tile ? (quad >> 1) : 0;  // which key block's rows (warp-uniform)
         bool ok = true;
         for (int c = 0; c < nchunk; ++c) {
             const int st = c % kStages;
@@ -285,9 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tmem_wait_ld();
             uint32_t pd[16];  // P^T pairs then dS^T pairs
-            // key rows past the block (a 64-token key block fills half the tile) are
-            // a whole warp's rows, so the branch is warp-uniform
-            if (live) {
+            // key rows past the block, or of a block whose column lacks this query
+            // chunk, are whole warps' rows, so the branch is warp-uniform
+            if (live && ((mask_s[st] >> half) & 1u)) {
                 const uint64_t s2 = splat2(scale_log2);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -355,11 +356,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int d = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const bool leader = (warp == 2 + kSoftmaxWarps && lane == 0);
-        int u = u_begin, r = 0, r_end = 0;
-        if (u < u_end) {
-            r = bo[rowT[u]];
-            r_end = bo[rowT[u] + 1];
-        }
+        SegWalk wk;
+        wk.init(u_begin, u_end, u2_begin, u2_end, rowT, bo);
         for (int c = 0; c < nchunk; ++c) {
             const int st = c % kStages;
             if (!__all_sync(0xffffffffu,
@@ -385,14 +383,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_async_smem();
             named_bar_sync(1, 128);
             if (leader) {
-                tma_reduce_add_2d(&tmdQ, sbase + L::kDQ, 0, rowbase + r);
+                tma_reduce_add_2d(&tmdQ, sbase + L::kDQ, 0, rowbase + wk.r);
                 bulk_commit();
             }
-            r += 64;
-            if (r >= r_end && ++u < u_end) {
-                r = bo[rowT[u]];
-                r_end = bo[rowT[u] + 1];
-            }
+            wk.advance(rowT, bo);
         }
         if (leader) bulk_wait_all();  // every reduce has landed before the CTA exits
     }

@@ -5,9 +5,12 @@
 // under one online softmax, to the tokens of the key blocks in S_i.
 //
 // Work unit: one 128-row query tile of one head (a 256-token block gives two
-// tiles, a 128-token block one, a 64-token block one tile whose upper 64 rows
-// are computed and discarded).  The selected key blocks are streamed as
-// 64-row segments; two segments form a 128-key chunk.
+// tiles, a 128-token block one, and two consecutive 64-token blocks i, i+1
+// share one).  The selected key blocks are streamed as 64-row segments; two
+// segments form a 128-key chunk.  A shared tile streams S_i U S_{i+1}: the
+// producer writes, per chunk, which of the two sets each segment belongs to,
+// and each row half (whole softmax warps) gives the segments outside its own
+// set P = 0.
 //
 // Two CTAs share an SM (96 KB of shared memory and 256 TMEM columns each), so
 // while one CTA's softmax works the tensor cores run the other CTA's MMAs;
@@ -59,19 +62,23 @@ struct Layout {
     static constexpr uint32_t kK = kQ + kHalves * kTileBytes;
     static constexpr uint32_t kV = kK + kHalves * kTileBytes;
     static constexpr uint32_t kBars = kV + kHalves * kTileBytes;
-    // barriers: q, k_full, k_empty, v_full, v_empty, s, p, o  (8 B each) + tmem slot + abort
-    static constexpr uint32_t kNumBars = 9;
-    static constexpr uint32_t kBytes = kBars + kNumBars * 8 + 16;
+    // barriers: q, k_full, k_empty, v_full, v_empty, s, p, o, p2, mask[2]  (8 B each)
+    // + tmem slot + abort, then the two segment-mask words of a shared tile
+    static constexpr uint32_t kNumBars = 11;
+    static constexpr uint32_t kMaskW = kBars + kNumBars * 8 + 16;
+    static constexpr uint32_t kBytes = kMaskW + 8;
     static constexpr uint32_t kAlloc = kBytes + 1024;  // slack to align the base to 1024
-    // Taylor variant: per-softmax-warp bias of a chunk, then the log2 |B_j|
-    // table (int8, -1 for the blocks of S_i)
+    // Taylor variant: per-softmax-warp bias of a chunk, then two log2 |B_j|
+    // tables (int8, -1 for the blocks of S_i; the second for the second block
+    // of a shared tile)
     static constexpr uint32_t kBias = (kBytes + 15) & ~15u;
     static constexpr uint32_t kLg = kBias + 4 * 128 * 4;
-    static uint32_t taylor_alloc(int nbmax) { return kLg + ((nbmax + 15) & ~15u) + 1024; }
+    __host__ __device__ static uint32_t lg_stride(int nbmax) { return (nbmax + 15) & ~15u; }
+    static uint32_t taylor_alloc(int nbmax) { return kLg + 2 * lg_stride(nbmax) + 1024; }
 };
 
 // Site codes recorded with a timeout.
-enum { kSiteQ = 1, kSiteK, kSiteV, kSiteKEmpty, kSiteVEmpty, kSiteS, kSiteP, kSiteO };
+enum { kSiteQ = 1, kSiteK, kSiteV, kSiteKEmpty, kSiteVEmpty, kSiteS, kSiteP, kSiteO, kSiteMask };
 
 template <int D, bool kTaylor>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -94,19 +101,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int *bo = blk_off + (size_t)b * (g.nbmax + 1);
     const int q0 = qt_row[(size_t)b * g.nbmax + tile];
-    const int iblk = qt_blk[(size_t)b * g.nbmax + tile];
-    const int qvalid = min(128, bo[iblk + 1] - q0);
+    int iblk, iblk2;
+    tile_blocks(qt_blk[(size_t)b * g.nbmax + tile], iblk, iblk2);
+    const bool shared_tile = iblk2 >= 0;
+    const int qvalid = min(128, bo[(shared_tile ? iblk2 : iblk) + 1] - q0);
     const size_t crow = (size_t)bh * g.nbmax + iblk;
     const int c_begin = row_ptr[crow], c_end = row_ptr[crow + 1];
+    // the second query block's selection (empty unless the tile is shared)
+    const int c2_begin = shared_tile ? row_ptr[crow + 1] : 0, c2_end = shared_tile ? row_ptr[crow + 2] : 0;
 
     // number of 64-row key segments of the selection (every warp computes it)
-    int nseg = 0;
-    for (int u = c_begin + lane; u < c_end; u += 32) {
-        const int j = col[u];
-        nseg += (bo[j + 1] - bo[j]) >> 6;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) nseg += __shfl_xor_sync(0xffffffffu, nseg, o);
+    const int nseg = union_segments(col + c_begin, c_end - c_begin, col + c2_begin, c2_end - c2_begin, bo, lane);
     const int nchunk = (nseg + 1) >> 1;
     // Taylor variant: pooled chunks follow the selected ones
     const int nbb = kTaylor ? nbv[b] : 0;
@@ -114,15 +119,22 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int nchunk_all = nchunk + ((nseg_t + 1) >> 1);
     auto chunk_full = [&](int c) { return c < nchunk ? (2 * c + 1) < nseg : (2 * (c - nchunk) + 1) < nseg_t; };
     int8_t *lg = reinterpret_cast<int8_t *>(smem + L::kLg);
+    const uint32_t lgs = L::lg_stride(g.nbmax);
     if constexpr (kTaylor)  // block volumes are powers of two: log2 |B_j| is exact
-        for (int j = threadIdx.x; j < nbb; j += kThreads) lg[j] = (int8_t)(31 - __clz(bo[j + 1] - bo[j]));
+        for (int j = threadIdx.x; j < nbb; j += kThreads) {
+            const int8_t v = (int8_t)(31 - __clz(bo[j + 1] - bo[j]));
+            lg[j] = v;
+            lg[lgs + j] = v;
+        }
 
     const uint32_t bar_q = sbase + L::kBars;
     const uint32_t bar_kf = bar_q + 8, bar_ke = bar_q + 16, bar_vf = bar_q + 24, bar_ve = bar_q + 32;
     const uint32_t bar_s = bar_q + 40, bar_p = bar_q + 48, bar_o = bar_q + 56;
     const uint32_t bar_p2 = bar_q + 64;  // P of keys 64..127 (bar_p: keys 0..63)
+    const uint32_t bar_mk = bar_q + 72;  // [2]: the mask word of chunk c is in slot c & 1
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBars + L::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kBars + L::kNumBars * 8 + 8);
+    volatile uint32_t *mask_w = reinterpret_cast<volatile uint32_t *>(smem + L::kMaskW);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -135,6 +147,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_init(bar_p, 128);
             mbar_init(bar_p2, 128);
             mbar_init(bar_o, 1);
+            mbar_init(bar_mk, 1);
+            mbar_init(bar_mk + 8, 1);
             *abort_flag = 0;
             mbar_fence_init();
             prefetch_map(&tmQ);
@@ -150,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
     if constexpr (kTaylor) {  // the blocks of S_i are exact: no pooled term
         for (int u = c_begin + threadIdx.x; u < c_end; u += kThreads) lg[col[u]] = -1;
+        for (int u = c2_begin + threadIdx.x; u < c2_end; u += kThreads) lg[lgs + col[u]] = -1;
         __syncthreads();
     }
     const uint32_t tmem = *tmem_slot;
@@ -164,11 +179,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int rh = 0; rh < 2; ++rh)
                     tma_load_2d(sbase + L::kQ + hf * L::kTileBytes + rh * 8192, &tmQ, bar_q, hf * 64,
                                 rowbase + q0 + rh * 64);
-            int u = c_begin, r = 0, r_end = 0;
-            if (u < c_end) {
-                r = bo[col[u]];
-                r_end = bo[col[u] + 1];
-            }
+            SegWalk wk;
+            wk.init(c_begin, c_end, c2_begin, c2_end, col, bo);
             int kissued = 0, vissued = 0;
             for (int c = 0; c < nchunk_all; ++c) {
                 const bool pooled = kTaylor && c >= nchunk;
@@ -176,20 +188,22 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const uint32_t bytes = nsg * 64 * D * 2;
                 const CUtensorMap *mK = pooled ? &tmKb : &tmK, *mV = pooled ? &tmVb : &tmV;
                 int rows[2];
+                uint32_t segmask = 0;  // bits 2s, 2s+1: segment s in S_i, in S_{i+1}
                 if (pooled) {  // rows of the pooled [batch*heads][nbmax][D] copies
                     for (int gsg = 0; gsg < nsg; ++gsg) rows[gsg] = bh * g.nbmax + 128 * (c - nchunk) + 64 * gsg;
                 } else {
                     for (int gsg = 0; gsg < nsg; ++gsg) {
-                        rows[gsg] = rowbase + r;
-                        r += 64;
-                        if (r >= r_end && ++u < c_end) {
-                            r = bo[col[u]];
-                            r_end = bo[col[u] + 1];
-                        }
+                        rows[gsg] = rowbase + wk.r;
+                        segmask |= (uint32_t)wk.mask << (2 * gsg);
+                        wk.advance(col, bo);
                     }
                 }
                 // K_c once S_{c-1} has consumed the K buffer
                 if (c > 0 && !mbar_wait(bar_ke, (c - 1) & 1, status, kSiteKEmpty, abort_flag)) break;
+                if (shared_tile && !pooled) {  // the softmax has read this slot for chunk c - 2
+                    mask_w[c & 1] = segmask;
+                    mbar_arrive(bar_mk + 8 * (c & 1));
+                }
                 mbar_expect_tx(bar_kf, bytes);
                 for (int gsg = 0; gsg < nsg; ++gsg)
                     for (int hf = 0; hf < L::kHalves; ++hf)
@@ -252,15 +266,26 @@ __global__ void __launch_bounds__(kThreads, 2)
         float m = -INFINITY, l = 0.f;
         bool ok = true;
         const uint32_t bias_s = sbase + L::kBias + quad * 512;  // this warp's 128 column biases
+        const int half = shared_tile ? (quad >> 1) : 0;        // which query block's rows (warp-uniform)
+        const int8_t *lgh = lg + half * lgs;
         for (int c = 0; c < nchunk_all; ++c) {
             const bool pooled = kTaylor && c >= nchunk;
+            // segments of this chunk outside this half's selection get P = 0
+            bool live0 = true, live1 = true;
+            if (shared_tile && !pooled) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_mk + 8 * (c & 1), (c >> 1) & 1, status, kSiteMask, abort_flag));
+                if (!ok) break;
+                const uint32_t mw = mask_w[c & 1];
+                live0 = (mw >> half) & 1u;
+                live1 = (mw >> (2 + half)) & 1u;
+            }
             if (pooled) {  // biases of this chunk's pooled keys, before S lands
                 float *bias = reinterpret_cast<float *>(smem + L::kBias + quad * 512);
                 __syncwarp();  // the warp has read the previous chunk's biases
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int j = 128 * (c - nchunk) + 32 * e + lane;
-                    const int v = j < nbb ? lg[j] : -1;
+                    const int v = j < nbb ? lgh[j] : -1;
                     bias[32 * e + lane] = v < 0 ? -INFINITY : (float)v;
                 }
                 __syncwarp();
@@ -308,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             } else {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    if (q < nq) {
+                    if (q < nq && (q < 2 ? live0 : live1)) {
 #pragma unroll
                         for (int e = 0; e < 32; e += 8) {
                             const float *v = reinterpret_cast<const float *>(&sr[32 * q + e]);
@@ -351,14 +376,19 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int q = 0; q < 4; ++q)
                 if (q < nq) {
                     uint32_t pk[16];
+                    if (q < 2 ? live0 : live1) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        float x0, x1;
-                        fma2(__uint_as_float(sr[32 * q + 2 * e]), __uint_as_float(sr[32 * q + 2 * e + 1]), s2, c2, x0,
-                             x1);
-                        const float p0 = ex2(x0), p1 = ex2(x1);
-                        add2(acc2, p0, p1);
-                        pk[e] = pack_bf16x2(p0, p1);
+                        for (int e = 0; e < 16; ++e) {
+                            float x0, x1;
+                            fma2(__uint_as_float(sr[32 * q + 2 * e]), __uint_as_float(sr[32 * q + 2 * e + 1]), s2, c2,
+                                 x0, x1);
+                            const float p0 = ex2(x0), p1 = ex2(x1);
+                            add2(acc2, p0, p1);
+                            pk[e] = pack_bf16x2(p0, p1);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
                     }
                     tmem_st16(tSr + q * 16, pk);
                     if (q == 1) {  // P of keys 0..63 is in TMEM: the first half of P V may start

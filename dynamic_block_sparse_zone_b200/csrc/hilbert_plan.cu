@@ -67,8 +67,8 @@ __global__ void k_hilbert_perm(Geo g, int k, const int *__restrict__ rank, int *
     }
 }
 
-// Fixed blocks of B tokens: block table, 64-row tile map and 128-row query
-// tiles (a 64-token block is one tile whose upper rows are discarded).
+// Fixed blocks of B tokens: block table, 64-row tile map and 128-row tiles
+// (two 64-token blocks share a tile, marked by the complement of the first).
 __global__ void k_hilbert_tables(Geo g, int B, int *__restrict__ nb, int *__restrict__ blk_off,
                                  int *__restrict__ tile_blk, int *__restrict__ nqt, int *__restrict__ qt_row,
                                  int *__restrict__ qt_blk) {
@@ -78,10 +78,17 @@ __global__ void k_hilbert_tables(Geo g, int B, int *__restrict__ nb, int *__rest
         blk_off[(size_t)b * (g.nbmax + 1) + j] = j * B;
         if (j == nbk) {
             nb[b] = nbk;
-            nqt[b] = nbk * tpb;
+            nqt[b] = B == 64 ? nbk / 2 : nbk * tpb;
             continue;
         }
         for (int u = 0; u < B / kTile; ++u) tile_blk[(size_t)b * g.nbmax + j * (B / kTile) + u] = j;
+        if (B == 64) {
+            if ((j & 1) == 0) {
+                qt_row[(size_t)b * g.nbmax + j / 2] = j * B;
+                qt_blk[(size_t)b * g.nbmax + j / 2] = ~j;
+            }
+            continue;
+        }
         for (int r = 0; r < tpb; ++r) {
             qt_row[(size_t)b * g.nbmax + j * tpb + r] = j * B + r * 128;
             qt_blk[(size_t)b * g.nbmax + j * tpb + r] = j;

@@ -373,7 +373,7 @@ __global__ void __launch_bounds__(1024) k_zone_decide(Geo g, const double *__res
             zone_B[zm] = B;
             zone_shape[zm] = idx;
             nblk = kZoneVol / B;
-            ntile = nblk * ((B + 127) / 128);  // 128-row query tiles of the zone
+            ntile = kZoneVol / 128;  // 128-row tiles of the zone (two 64-token blocks share one)
         }
         int total, total_t;
         const int excl = block_scan_excl_1024(nblk, sbuf, &total);
@@ -403,6 +403,14 @@ __global__ void __launch_bounds__(1024) k_zone_decide(Geo g, const double *__res
             const int off = m * kZoneVol + l * B;
             blk_off[(size_t)b * (g.nbmax + 1) + j0 + l] = off;
             for (int u = 0; u < B / kTile; ++u) tile_blk[(size_t)b * g.nbmax + off / kTile + u] = j0 + l;
+            if (B == 64) {  // blocks l, l+1 share a tile, marked by the complement of the first
+                if ((l & 1) == 0) {
+                    qt_row[(size_t)b * g.nbmax + t] = off;
+                    qt_blk[(size_t)b * g.nbmax + t] = ~(j0 + l);
+                    ++t;
+                }
+                continue;
+            }
             for (int r = 0; r < B; r += 128, ++t) {
                 qt_row[(size_t)b * g.nbmax + t] = off + r;
                 qt_blk[(size_t)b * g.nbmax + t] = j0 + l;

@@ -57,9 +57,11 @@ struct Plan {
     int *blk_off;           // [batch][nbmax+1]
     int *tile_blk;          // [batch][nbmax]  64-row tile -> block
     int *zone_qt0;          // [batch][M+1]  first 128-row query tile of each zone
-    int *nqt;               // [batch]       number of 128-row query tiles
-    int *qt_row;            // [batch][nbmax] first block-contiguous row of each query tile
-    int *qt_blk;            // [batch][nbmax] block of each query tile
+    int *nqt;               // [batch]       number of 128-row tiles (query tiles of the
+                            //               forward, key tiles of the backward)
+    int *qt_row;            // [batch][nbmax] first block-contiguous row of each tile
+    int *qt_blk;            // [batch][nbmax] block of each tile; ~j for a tile holding the
+                            //               two 64-token blocks j and j+1
     int *perm;              // [batch][N]  block-contiguous position -> raster token
     // permuted head-major inputs and pooled blocks
     __nv_bfloat16 *Qp, *Kp, *Vp;   // [batch*heads][N][D]

@@ -59,6 +59,71 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *st
     return false;
 }
 
+// ---- the block lists a 128-row tile streams ----
+// A tile holds one block (qt_blk = j) or the two 64-token blocks j, j+1
+// (qt_blk = ~j); j2 = -1 when there is no second block.
+__device__ __forceinline__ void tile_blocks(int code, int &j1, int &j2) {
+    j1 = code < 0 ? ~code : code;
+    j2 = code < 0 ? j1 + 1 : -1;
+}
+// Is j in the ascending list L[0..n)?
+__device__ __forceinline__ bool sorted_has(const int *L, int n, int j) {
+    int lo = 0, hi = n - 1;
+    while (lo <= hi) {
+        const int mid = (lo + hi) >> 1;
+        const int v = L[mid];
+        if (v == j) return true;
+        if (v < j) lo = mid + 1;
+        else hi = mid - 1;
+    }
+    return false;
+}
+// 64-row segments of the union of two ascending block lists (every lane of
+// the warp gets the total).
+__device__ __forceinline__ int union_segments(const int *A, int na, const int *B, int nb, const int *bo, int lane) {
+    int n = 0;
+    for (int u = lane; u < na; u += 32) n += (bo[A[u] + 1] - bo[A[u]]) >> 6;
+    for (int u = lane; u < nb; u += 32)
+        if (!sorted_has(A, na, B[u])) n += (bo[B[u] + 1] - bo[B[u]]) >> 6;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+    return n;
+}
+// Walk over those segments in ascending block order, the two lists being the
+// index ranges [ua, a_end) and [ub, b_end) of one array L: r is the
+// segment's first block-contiguous row, mask bit 0 / bit 1 say whether its
+// block is in the first / second list.  L and the block offsets bo are passed
+// to each step rather than kept (the kernels are short of registers).
+struct SegWalk {
+    int ua, a_end, ub, b_end;
+    int r, r_end, mask;
+    __device__ __forceinline__ void pick(const int *L, const int *bo) {
+        const int ja = ua < a_end ? L[ua] : 0x7fffffff, jb = ub < b_end ? L[ub] : 0x7fffffff;
+        const int j = min(ja, jb);
+        mask = (ja == j ? 1 : 0) | (jb == j ? 2 : 0);
+        ua += ja == j;
+        ub += jb == j;
+        if (j != 0x7fffffff) {
+            r = bo[j];
+            r_end = bo[j + 1];
+        } else {
+            r = r_end = 0;
+            mask = 0;
+        }
+    }
+    __device__ __forceinline__ void init(int a0, int a1, int b0, int b1, const int *L, const int *bo) {
+        ua = a0;
+        a_end = a1;
+        ub = b0;
+        b_end = b1;
+        pick(L, bo);
+    }
+    __device__ __forceinline__ void advance(const int *L, const int *bo) {
+        r += 64;
+        if (r >= r_end) pick(L, bo);
+    }
+};
+
 // ---- TMA (2D tiled, this GPU's own memory, no multicast) ----
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
     asm volatile(
