@@ -292,7 +292,7 @@ def run_ours(args, rank, world, dev):
     # plan and the attention kernels, and copies its outputs back; the plan
     # overlaps one step's copies with its neighbours' kernels on three streams.
     e2e = None
-    if not args.no_e2e and not args.taylor:
+    if not args.no_e2e:
         host_in = [x.cpu().pin_memory() for x in (inp.Q, inp.K, inp.V, inp.a)]
         host_dO = None if args.fwd_only else inp.dO.cpu().pin_memory()
         host_out = [torch.empty(shp, dtype=torch.bfloat16).pin_memory() for _ in range(1 if args.fwd_only else 4)]
@@ -302,7 +302,7 @@ def run_ours(args, rank, world, dev):
 
         def e2e_step():
             if args.fwd_only:
-                return plan.step_host(*host_in, host_out[0])
+                return plan.step_host(*host_in, host_out[0], taylor=args.taylor)
             return plan.step_host(*host_in, host_out[0], dO=host_dO, dQ=host_out[1], dK=host_out[2], dV=host_out[3])
 
         for _ in range(max(1, args.warmup // 2)):

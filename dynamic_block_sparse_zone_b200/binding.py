@@ -54,7 +54,8 @@ _lib = None
 
 
 class prism_host_io(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("Q", "K", "V", "a_norm", "dO", "O", "lse", "dQ", "dK", "dV")]
+    _fields_ = [(n, ctypes.c_void_p) for n in ("Q", "K", "V", "a_norm", "dO", "O", "lse", "dQ", "dK", "dV")] + [
+        ("taylor", ctypes.c_int)]
 
 
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
@@ -288,7 +289,7 @@ class PrismPlan:
         return dQ, dK, dV
 
     # -- steps from host memory (pipelined across calls) ---------------------
-    def step_host(self, Q, K, V, a_norm, O, lse=None, dO=None, dQ=None, dK=None, dV=None) -> int:
+    def step_host(self, Q, K, V, a_norm, O, lse=None, dO=None, dQ=None, dK=None, dV=None, taylor=False) -> int:
         """Enqueues one layer step on host tensors (page-locked for overlap) and
         returns its ticket; the tensors are kept alive until step_wait covers it."""
         p = self.params
@@ -306,7 +307,8 @@ class PrismPlan:
         for t, n, dt, sh in host:
             if t.is_cuda or t.dtype != dt or tuple(t.shape) != tuple(sh) or not t.is_contiguous():
                 raise ValueError(f"{n}: expected a contiguous host tensor {dt} {tuple(sh)}")
-        io = prism_host_io(*(None if t is None else t.data_ptr() for t in (Q, K, V, a_norm, dO, O, lse, dQ, dK, dV)))
+        io = prism_host_io(*(None if t is None else t.data_ptr() for t in (Q, K, V, a_norm, dO, O, lse, dQ, dK, dV)),
+                           int(bool(taylor)))
         tk = ctypes.c_ulonglong()
         _check(load_library().prism_step_host(self._h, ctypes.byref(io), _stream(), ctypes.byref(tk)))
         self._held[tk.value] = [t for t, *_ in host]

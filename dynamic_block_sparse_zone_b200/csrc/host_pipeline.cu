@@ -146,7 +146,9 @@ prism_status host_step(Plan &pl, const prism_host_io &io, cudaStream_t user, uns
     st = launch_plan(pl, hp.in[s][kQ], hp.in[s][kK], hp.in[s][kV], static_cast<const float *>(hp.in[s][kA]), hp.comp);
     if (st != PRISM_OK) return st;
     pl.built = true;
-    st = launch_attn_fwd_tc(pl, hp.out[s][kO], io.lse ? static_cast<float *>(hp.out[s][kLse]) : nullptr, hp.comp);
+    float *lse_dev = io.lse ? static_cast<float *>(hp.out[s][kLse]) : nullptr;
+    st = io.taylor ? launch_attn_fwd_taylor(pl, hp.out[s][kO], lse_dev, hp.comp)
+                   : launch_attn_fwd_tc(pl, hp.out[s][kO], lse_dev, hp.comp);
     if (st != PRISM_OK) return st;
     pl.have_fwd = true;
     PRISM_CUDA_OK(cudaEventRecord(hp.fwd_done[s], hp.comp));

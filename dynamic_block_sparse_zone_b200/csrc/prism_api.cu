@@ -454,6 +454,10 @@ prism_status prism_step_host(prism_plan *plan, const prism_host_io *io, void *st
         return fail(PRISM_ERR_INVALID_ARG, "prism_step_host needs Q, K, V, a_norm and O");
     if (io->dO && (!io->dQ || !io->dK || !io->dV))
         return fail(PRISM_ERR_INVALID_ARG, "prism_step_host with dO needs dQ, dK and dV");
+    if (io->taylor && io->dO)
+        return fail(PRISM_ERR_INVALID_ARG, "a Taylor forward has no backward: taylor steps are forward-only");
+    if (io->taylor && !taylor_fits(plan->pl.g))
+        return fail(PRISM_ERR_UNSUPPORTED, "too many key blocks for the Taylor forward's shared-memory table");
     if (plan->pl.g.Ctot != plan->pl.g.C && !plan->pl.p.hilbert_block)
         return fail(PRISM_ERR_STATE, "prism_step_host runs unsharded zone plans only");
     prism_status s = device_guard(plan->pl);

@@ -249,8 +249,8 @@ PRISM_API prism_status prism_audio_norms(const void *h, float *a, int batch, int
  * outputs used (2 x 9 bf16 tensors of batch*N*heads*head_dim at most) and
  * freed with the plan.  Do not interleave host steps with the device-pointer
  * calls on one plan without prism_step_wait in between: both use the plan's
- * internal buffers.  PRISM_ERR_INVALID_ARG for a NULL required field or a
- * ticket that was never issued.                                            */
+ * internal buffers.  PRISM_ERR_INVALID_ARG for a NULL required field, for
+ * taylor with dO, or a ticket that was never issued.                        */
 typedef struct prism_host_io {
     const void *Q, *K, *V;  /* bf16, host                                     */
     const float *a_norm;    /* fp32, host                                     */
@@ -258,6 +258,8 @@ typedef struct prism_host_io {
     void *O;                /* bf16, host, written                            */
     float *lse;             /* fp32, host, written; may be NULL               */
     void *dQ, *dK, *dV;     /* bf16, host, written when dO != NULL            */
+    int taylor;             /* nonzero: the forward of prism_attn_fwd_taylor  */
+                            /* (forward-only steps: dO must be NULL)          */
 } prism_host_io;
 PRISM_API prism_status prism_step_host(prism_plan *plan, const prism_host_io *io, void *stream,
                                        unsigned long long *ticket);

@@ -500,6 +500,18 @@ def test_host_steps_match_the_device_path():
     with pytest.raises(P.PrismError):
         plan.step_wait(0)
     plan.step_wait(1)  # long completed: fine
+    # a forward-only step with the Taylor term equals prism_attn_fwd_taylor
+    Q, K, V, a, dO = pin[1]
+    O = torch.empty(shp, dtype=torch.bfloat16).pin_memory()
+    lse = torch.empty(lshp, dtype=torch.float32).pin_memory()
+    plan.step_wait(plan.step_host(Q, K, V, a, O, lse=lse, taylor=True))
+    plan.build(*(x.cuda() for x in (inputs[1].Q, inputs[1].K, inputs[1].V, inputs[1].a)))
+    rO, rl = plan.fwd(taylor=True)
+    torch.cuda.synchronize()
+    assert torch.equal(O, rO.cpu()) and torch.equal(lse, rl.cpu())
+    with pytest.raises(P.PrismError):  # the Taylor forward has no backward
+        g = [torch.empty(shp, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+        plan.step_host(Q, K, V, a, O, dO=dO, dQ=g[0], dK=g[1], dV=g[2], taylor=True)
     plan.close()
 
 
@@ -836,3 +848,39 @@ def test_hilbert_plan_2k_full_size():
     ties = compare_hilbert_plan(w, pl, g["view"], heads=heads)
     check_forward(w, inp, g, pl, bits, 128, heads=heads)
     print("2K Hilbert near-ties", ties, "blocks", pl.nb)
+
+
+def test_head_sharded_hilbert_plan_builds_alone():
+    """A Hilbert-order plan needs no zone statistics, so a shard of the heads
+    is built with prism_plan_build alone; its order, blocks, selections and
+    forward equal the whole layer's for those heads."""
+    P = _lib()
+    w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=4, planted=2)
+    inp = make_inputs(w, 19)
+    full = P.PrismPlan(P.params_for(w, hilbert_block=128))
+    Q, K, V = (x.cuda() for x in (inp.Q, inp.K, inp.V))
+    full.build(Q, K, V, None)
+    O_full, _ = full.fwd()
+    torch.cuda.synchronize()
+    vf = full.view()
+    hs = [2, 3]
+    p = P.params_for(scaled(w, heads=2), hilbert_block=128)
+    p.heads_total, p.head_offset = 4, 2
+    shard = P.PrismPlan(p)
+    Qs, Ks, Vs = (x[:, :, hs, :].contiguous().cuda() for x in (inp.Q, inp.K, inp.V))
+    shard.build(Qs, Ks, Vs, None)
+    O_sh, _ = shard.fwd()
+    torch.cuda.synchronize()
+    shard.check()
+    vs = shard.view()
+    assert vs["n_blocks"][0] == vf["n_blocks"][0]
+    assert torch.equal(vs["perm"], vf["perm"])
+    nbm = vf["nbmax"]
+    rpf, cf = vf["row_ptr"].cpu().numpy(), vf["col_idx"].cpu().numpy()
+    rps, cs = vs["row_ptr"].cpu().numpy(), vs["col_idx"].cpu().numpy()
+    for hi, h in enumerate(hs):
+        for i in range(vf["n_blocks"][0]):
+            a = cf[rpf[h * nbm + i]:rpf[h * nbm + i + 1]]
+            b = cs[rps[hi * nbm + i]:rps[hi * nbm + i + 1]]
+            assert np.array_equal(a, b)
+    assert torch.equal(O_sh.view(torch.int16), O_full[:, :, hs, :].contiguous().view(torch.int16))
