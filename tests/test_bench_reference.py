@@ -27,3 +27,30 @@ def test_reference_arm_prints_the_contract_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
     e2e = line["e2e"]
     assert e2e["value"] == line["value"] and e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+import pytest  # noqa: E402
+
+
+@pytest.mark.gpu
+def test_bench_line_of_our_arm_has_the_contract_keys():
+    """bench.py on the Tiny workload (seconds): the JSON line carries the
+    contract's keys, the roofline, end-to-end and clock records, and a
+    positive count of our kernel launches."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--workload", "tiny_8x16x16", "--fwd-only",
+           "--steps", "3", "--warmup", "3", "--no-cpu-baseline"]
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=900, cwd=ROOT)
+    assert res.returncode == 0, res.stderr[-2000:]
+    line = json.loads(res.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "gpu_launches", "e2e", "clocks"):
+        assert key in line, key
+    assert line["n_gpus"] == 1 and line["steps"] == 3 and line["warmup"] == 3 and line["scaling"] == "weak"
+    assert line["value"] > 0 and line["gpu_launches"] > 0
+    r = line["roofline"]
+    for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert key in r, key
+    assert r["peak"] > 0 and 0 < r["frac"] < 2
+    e = line["e2e"]
+    assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
+    assert "workload" in line["config"] and "l2" in line["config"]
