@@ -919,3 +919,54 @@ def test_large_logits_forward_backward_and_taylor():
     assert_close_scaled("dK", g["dK"][0].float().cpu().numpy()[req_t, req_h], dK_ref)
     assert_close_scaled("dV", g["dV"][0].float().cpu().numpy()[req_t, req_h], dV_ref)
     check_forward_taylor(w, g["plan"], pl, bits, 512)
+
+
+# grids of odd aspect (one zone wide, long and thin), batch 3, head_dim 64,
+# extreme k / p / cap, fixed shapes, Hilbert blocks: plan exactness, forward,
+# Taylor forward and (some) gradients against the oracle
+_ODD = [
+    dict(T=8, H=8, W=64, heads=2, head_dim=64, top_k=1, top_p=0.5, max_frac=0.0, planted=1),
+    dict(T=64, H=8, W=8, heads=1, head_dim=128, top_k=3, top_p=0.99, max_frac=0.25, planted=2, backward=True),
+    dict(T=8, H=24, W=8, heads=3, head_dim=64, top_k=2, top_p=0.8, max_frac=0.5, batch=3, planted=1),
+    dict(T=16, H=16, W=8, heads=2, head_dim=128, top_k=4, top_p=0.9, fixed_shape=(2, 4, 8), planted=1, backward=True),
+    dict(T=8, H=8, W=8, heads=2, head_dim=64, top_k=1, top_p=1.0, planted=0),
+    dict(T=16, H=8, W=24, heads=2, head_dim=128, top_k=2, top_p=0.95, max_frac=0.1, planted=2, hilbert=64),
+]
+
+
+@pytest.mark.parametrize("case", range(len(_ODD)))
+def test_odd_grids_and_parameters(case):
+    cfg = dict(_ODD[case])
+    hb = cfg.pop("hilbert", 0)
+    w = scaled(WORKLOADS["dynamic_16x32x32"], **cfg)
+    inp = make_inputs(w, 100 + case, with_grad_output=True)
+    P = _lib()
+    plan = P.PrismPlan(P.params_for(w, hilbert_block=hb))
+    Q, K, V, a = (x.cuda() for x in (inp.Q, inp.K, inp.V, inp.a))
+    plan.build(Q, K, V, a)
+    O, lse = plan.fwd()
+    out = dict(O=O, lse=lse, plan=plan)
+    if w.backward:
+        out["dQ"], out["dK"], out["dV"] = plan.bwd(O, inp.dO.cuda())
+    torch.cuda.synchronize()
+    plan.check()
+    out["view"] = plan.view()
+    taylor = plan.fwd(taylor=True)
+    for b in range(w.batch):
+        if hb:
+            pl, bits = oracle_hilbert_plan(w, inp, hb, b=b)
+            compare_hilbert_plan(w, pl, out["view"], b=b)
+        else:
+            pl, bits = oracle_plan(w, inp, b=b)
+            compare_plan(w, pl, out["view"], b=b)
+        check_forward(w, inp, out, pl, bits, min(w.N, 1024), b=b)
+        check_forward_taylor(w, plan, pl, bits, 256, b=b, out=taylor)
+        if w.backward:
+            rs = np.random.default_rng(case)
+            req_h, req_t = sample_rows(rs, w, 256)
+            dQ_ref = oracle.attn_bwd_dq_rows(pl, *bits, bf16_bits(inp.dO[b]), req_h, req_t)
+            assert_close("dQ", out["dQ"][b].float().cpu().numpy()[req_t, req_h], dQ_ref)
+            req_h, req_t = pick_dkv_rows(pl, 0, 2, 8, rs)
+            dK_ref, dV_ref = oracle.attn_bwd_dkv_rows(pl, *bits, bf16_bits(inp.dO[b]), req_h, req_t)
+            assert_close("dK", out["dK"][b].float().cpu().numpy()[req_t, req_h], dK_ref)
+            assert_close("dV", out["dV"][b].float().cpu().numpy()[req_t, req_h], dV_ref)
