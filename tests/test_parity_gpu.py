@@ -970,3 +970,34 @@ def test_odd_grids_and_parameters(case):
             dK_ref, dV_ref = oracle.attn_bwd_dkv_rows(pl, *bits, bf16_bits(inp.dO[b]), req_h, req_t)
             assert_close("dK", out["dK"][b].float().cpu().numpy()[req_t, req_h], dK_ref)
             assert_close("dV", out["dV"][b].float().cpu().numpy()[req_t, req_h], dV_ref)
+
+
+def test_hilbert_plan_update_and_host_step_without_audio():
+    """A Hilbert-order plan reused for new Q, K, V (the gather reads the plan's
+    permutation) attends like the oracle's plan of the first inputs applied to
+    the second; a host-buffer step of that plan runs without a_norm and equals
+    the device path bit for bit."""
+    P = _lib()
+    w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=2, planted=1)
+    first, second = make_inputs(w, 31), make_inputs(w, 32)
+    plan = P.PrismPlan(P.params_for(w, hilbert_block=128))
+    plan.build(*(x.cuda() for x in (first.Q, first.K, first.V)), None)
+    plan.update_qkv(*(x.cuda() for x in (second.Q, second.K, second.V)))
+    O, lse = plan.fwd()
+    torch.cuda.synchronize()
+    plan.check()
+    pl, _ = oracle_hilbert_plan(w, first, 128)
+    compare_hilbert_plan(w, pl, plan.view())
+    bits2 = tuple(bf16_bits(x[0]) for x in (second.Q, second.K, second.V))
+    rs = np.random.default_rng(2)
+    req_h, req_t = sample_rows(rs, w, 512)
+    O_ref, _ = oracle.attn_fwd_rows(pl, *bits2, req_h, req_t)
+    assert_close("O", O[0].float().cpu().numpy()[req_t, req_h], O_ref)
+    # host-buffer step, no audio norms
+    plan.build(*(x.cuda() for x in (second.Q, second.K, second.V)), None)
+    O_dev, _ = plan.fwd()
+    torch.cuda.synchronize()
+    pin = [x.pin_memory() for x in (second.Q, second.K, second.V)]
+    Oh = torch.empty(second.Q.shape, dtype=torch.bfloat16).pin_memory()
+    plan.step_wait(plan.step_host(*pin, None, Oh))
+    assert torch.equal(Oh, O_dev.cpu())
