@@ -109,3 +109,11 @@ def test_host_step_arguments_are_checked_on_the_host(lib):
     assert lib.prism_step_join(None, 1, None) == 1
     assert lib.prism_step_wait(None, 1) == 1
     assert b"NULL" in lib.prism_last_error()
+
+
+def test_timer_names_cover_every_id(lib):
+    from dynamic_block_sparse_zone_b200.binding import NUM_TIMERS
+    names = [lib.prism_timer_name(k).decode() for k in range(NUM_TIMERS)]
+    assert len(set(names)) == NUM_TIMERS and all(names)
+    assert {"zone_stats_v", "permute_pool", "select", "attn_fwd", "attn_bwd", "attn_fwd_taylor"} <= set(names)
+    assert lib.prism_timer_name(NUM_TIMERS) == b"" and lib.prism_timer_name(-1) == b""

@@ -1001,3 +1001,30 @@ def test_hilbert_plan_update_and_host_step_without_audio():
     Oh = torch.empty(second.Q.shape, dtype=torch.bfloat16).pin_memory()
     plan.step_wait(plan.step_host(*pin, None, Oh))
     assert torch.equal(Oh, O_dev.cpu())
+
+
+def test_per_kernel_timers_count_launches_and_reset():
+    """prism_plan_set_timing / prism_plan_read_timing: one record per launch of
+    each timed kernel (the score / select pair once per head group), positive
+    times, cleared by the read; nothing is recorded with timing off."""
+    P = _lib()
+    w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=16, heads=2, planted=1, backward=True)
+    inp = make_inputs(w, 41, with_grad_output=True)
+    plan = P.PrismPlan(P.params_for(w))
+    Q, K, V, a, dO = (x.cuda() for x in (inp.Q, inp.K, inp.V, inp.a, inp.dO))
+    plan.set_timing(True)
+    plan.read_timing()
+    plan.build(Q, K, V, a)
+    O, _ = plan.fwd()
+    plan.bwd(O, dO)
+    plan.fwd(taylor=True)
+    t = plan.read_timing()
+    for name in ("zone_stats_v", "zone_stats_a", "zone_decide", "permute_pool", "csr_csc", "attn_fwd",
+                 "attn_bwd_pre", "attn_bwd", "dq_finalize", "taylor_pool", "attn_fwd_taylor"):
+        assert t[name][1] == 1 and t[name][0] > 0, (name, t[name])
+    assert t["select"][1] >= 2 and t["select"][1] % 2 == 0  # scores + select per head group
+    assert all(n == 0 for _, n in plan.read_timing().values())
+    plan.set_timing(False)
+    plan.fwd()
+    torch.cuda.synchronize()
+    assert all(n == 0 for _, n in plan.read_timing().values())
