@@ -391,6 +391,55 @@ def exchange_zone_stats(whole: torch.Tensor, mine: torch.Tensor, group=None):
     return whole
 
 
+def sequence_to_heads(x: torch.Tensor, group=None) -> torch.Tensor:
+    """Sequence-sharded activations to head-sharded ones for a head-sharded plan:
+    x [B, N/R, heads, D] on rank r (tokens [r N/R, (r+1) N/R) of every head)
+    becomes [B, N, heads/R, D] (heads [r heads/R, (r+1) heads/R) of every token),
+    with one all-to-all (NCCL over NVLink on GPUs).  R = 1: x unchanged."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+        return x
+    R = dist.get_world_size(group)
+    B, n, Hn, D = x.shape
+    if Hn % R:
+        raise ValueError("heads must divide evenly among the ranks")
+    h = Hn // R
+    send = x.reshape(B, n, R, h, D).permute(2, 0, 1, 3, 4).contiguous()  # [dest rank][B][n][h][D]
+    recv = torch.empty_like(send)                                         # [source rank][B][n][h][D]
+    dist.all_to_all_single(recv, send, group=group)
+    return recv.permute(1, 0, 2, 3, 4).reshape(B, R * n, h, D)
+
+
+def heads_to_sequence(y: torch.Tensor, group=None) -> torch.Tensor:
+    """The inverse of sequence_to_heads (for O and the gradients): y [B, N,
+    heads/R, D] on rank r becomes [B, N/R, heads, D]."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+        return y
+    R = dist.get_world_size(group)
+    B, N, h, D = y.shape
+    if N % R:
+        raise ValueError("tokens must divide evenly among the ranks")
+    n = N // R
+    send = y.reshape(B, R, n, h, D).permute(1, 0, 2, 3, 4).contiguous()  # [dest rank][B][n][h][D]
+    recv = torch.empty_like(send)                                         # [source rank][B][n][h][D]
+    dist.all_to_all_single(recv, send, group=group)
+    return recv.permute(1, 2, 0, 3, 4).reshape(B, n, R * h, D)
+
+
+def gather_sequence(t: torch.Tensor, group=None) -> torch.Tensor:
+    """All-gather of token shards along axis 1 ([B, N/R, ...] -> [B, N, ...]),
+    e.g. the audio norms a plan needs for every token."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+        return t
+    R = dist.get_world_size(group)
+    parts = torch.empty((R * t.shape[0],) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
+    dist.all_gather_into_tensor(parts, t.contiguous(), group=group)  # rank-major concatenation
+    parts = parts.view((R,) + tuple(t.shape))
+    return parts.movedim(0, 1).reshape((t.shape[0], R * t.shape[1]) + tuple(t.shape[2:]))
+
+
 def prism_audio_norms(h: torch.Tensor, T: int, H: int, W: int, a: Optional[torch.Tensor] = None) -> torch.Tensor:
     """a_{t,h,w} = ||h^_{t,h,w}||_2 for h [batch, T*H*W, channels] bf16 on the current device."""
     if h.dtype != torch.bfloat16 or not h.is_cuda or h.dim() != 3 or not h.is_contiguous():

@@ -1,13 +1,15 @@
 """Head sharding of the plan (one rank per GPU holding some heads of a layer).
 
-The one exchange is an all-gather of per-chunk zone statistics; these tests
-check its host side (parameter validation, the all-gather helper over gloo
-with world size 2) without a GPU.  The GPU test that shards a layer across
+The plan's one exchange is an all-gather of per-chunk zone statistics; with
+sequence-sharded activations an all-to-all each way moves them to head
+shards and back.  These tests check the host side (parameter validation, the
+helpers over gloo with 2 and 3 ranks) without a GPU.  The GPU test that shards a layer across
 ranks emulated in one process is in test_parity_gpu.py.
 """
 import os
 import socket
 
+import pytest
 import torch
 import torch.multiprocessing as mp
 
@@ -68,3 +70,44 @@ def test_zone_stat_slices_all_gather_in_rank_order_gloo_world2():
         assert p.exitcode == 0
     expect = [100.0 + i for i in range(6)] + [200.0 + i for i in range(6)]
     assert out[0] == expect and out[1] == expect
+
+
+def _layout_worker(rank, world, port, out):
+    import torch
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    from dynamic_block_sparse_zone_b200.binding import gather_sequence, heads_to_sequence, sequence_to_heads
+    g = torch.Generator().manual_seed(7)
+    B, N, H, D = 2, 24, 6, 4
+    full = torch.randn(B, N, H, D, generator=g)
+    a_full = torch.randn(B, N, generator=g)
+    n, h = N // world, H // world
+    mine = full[:, rank * n:(rank + 1) * n].contiguous()
+    heads = sequence_to_heads(mine)
+    ok = torch.equal(heads, full[:, :, rank * h:(rank + 1) * h])
+    back = heads_to_sequence(heads)
+    ok = ok and torch.equal(back, mine)
+    a = gather_sequence(a_full[:, rank * n:(rank + 1) * n].contiguous())
+    ok = ok and torch.equal(a, a_full)
+    out[rank] = bool(ok)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sequence_head_layout_exchange_gloo(world):
+    """Sequence-sharded activations to a head shard and back (one all-to-all
+    each way) and the token all-gather of the audio norms, against slicing the
+    whole tensors."""
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    out = ctx.Manager().dict()
+    procs = [ctx.Process(target=_layout_worker, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    assert all(out[r] for r in range(world))
