@@ -12,6 +12,7 @@ import os
 from dataclasses import dataclass
 from typing import Optional, Tuple
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -26,7 +27,7 @@ EXPORTED = ("prism_plan_create", "prism_plan_bytes", "prism_plan_build", "prism_
             "prism_plan_set_timing", "prism_plan_read_timing", "prism_timer_name", "prism_zone_shapes_noalloc",
             "prism_plan_selftest_timeout", "prism_plan_update_qkv", "prism_step_host", "prism_step_join",
             "prism_step_wait", "prism_audio_norms", "prism_plan_build_stats", "prism_plan_stats_slice",
-            "prism_plan_build_finish", "prism_attn_fwd_taylor")
+            "prism_plan_build_finish", "prism_attn_fwd_taylor", "prism_plan_build_with_zones")
 NUM_TIMERS = 12
 
 
@@ -94,6 +95,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.prism_plan_stats_slice.restype = ctypes.c_int
     lib.prism_plan_build_finish.argtypes = [V, P, P, P, P]
     lib.prism_plan_build_finish.restype = ctypes.c_int
+    lib.prism_plan_build_with_zones.argtypes = [V, P, P, P, P, P, P]
+    lib.prism_plan_build_with_zones.restype = ctypes.c_int
     lib.prism_audio_norms.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
     lib.prism_audio_norms.restype = ctypes.c_int
     lib.prism_plan_destroy.argtypes = [V]
@@ -252,6 +255,19 @@ class PrismPlan:
         whole, mine = self.stats_slice()
         exchange_zone_stats(whole, mine, group)
         return self.build_finish(Q, K, V)
+
+    def build_with_zones(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, zone_B, zone_shape):
+        """The plan from given zone decisions (int arrays [batch, N/512]: volumes
+        64/128/256 and candidate-table indices) instead of the zone statistics."""
+        p = self.params
+        for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+            _need(t, n, torch.bfloat16, self._qkv_shape())
+        zB = np.ascontiguousarray(np.asarray(zone_B, dtype=np.int32).reshape(p.batch, p.N // 512))
+        zs = np.ascontiguousarray(np.asarray(zone_shape, dtype=np.int32).reshape(p.batch, p.N // 512))
+        _check(load_library().prism_plan_build_with_zones(self._h, _ptr(Q), _ptr(K), _ptr(V),
+                                                         zB.ctypes.data_as(ctypes.c_void_p),
+                                                         zs.ctypes.data_as(ctypes.c_void_p), _stream()))
+        return self
 
     def update_qkv(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor):
         """Reuse the plan (zones, shapes, permutation, selection) for new Q, K, V."""

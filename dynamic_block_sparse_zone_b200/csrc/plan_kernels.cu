@@ -10,6 +10,8 @@
 //                                    density rho, volume B(m) from tau_128 /
 //                                    tau_256, l*_d, nearest candidate shape;
 //                                    block table of the block-contiguous order
+//                                    (or the table alone, for decisions the
+//                                    caller gives)
 //   k_permute_pool                   block-contiguous head-major copies of Q,K,V
 //                                    and the mean-pooled blocks (Method section 3)
 //   k_select                         Method section 3: pooled block scores, block
@@ -274,9 +276,11 @@ __device__ __forceinline__ double zone_sig(const double *zone_part, const Geo &g
     return s / (double)g.Ctot;
 }
 
+// given: zone_B / zone_shape already hold the decisions (checked on the
+// host); only the block table is built.
 __global__ void __launch_bounds__(1024) k_zone_decide(Geo g, const double *__restrict__ zone_part,
                                                       const double *__restrict__ zone_a, double eps,
-                                                      int fixed_idx, int *__restrict__ zone_B,
+                                                      int fixed_idx, bool given, int *__restrict__ zone_B,
                                                       int *__restrict__ zone_shape, int *__restrict__ zone_blk0,
                                                       int *__restrict__ nb_out, int *__restrict__ blk_off,
                                                       int *__restrict__ tile_blk, int *__restrict__ zone_qt0,
@@ -289,7 +293,7 @@ __global__ void __launch_bounds__(1024) k_zone_decide(Geo g, const double *__res
     const int M = g.M;
     // pass 1: maxima of s(m) and of a over the grid
     double smax = 0.0, amax = -DBL_MAX;
-    for (int m = tid; m < M; m += blockDim.x) {
+    for (int m = given ? M : tid; m < M; m += blockDim.x) {
         size_t zm = (size_t)b * M + m;
         double s = __dadd_rn(__dadd_rn(zone_sig(zone_part, g, zm, 0), zone_sig(zone_part, g, zm, 1)),
                              zone_sig(zone_part, g, zm, 2));
@@ -323,7 +327,10 @@ __global__ void __launch_bounds__(1024) k_zone_decide(Geo g, const double *__res
     for (int base = 0; base < M; base += blockDim.x) {
         const int m = base + tid;
         int nblk = 0, ntile = 0;
-        if (m < M) {
+        if (m < M && given) {
+            nblk = kZoneVol / zone_B[(size_t)b * M + m];
+            ntile = kZoneVol / 128;
+        } else if (m < M) {
             size_t zm = (size_t)b * M + m;
             double sg[3], sa[3];
             for (int d = 0; d < 3; ++d) {
@@ -1013,10 +1020,23 @@ prism_status launch_plan_finish(Plan &pl, const void *Qv, const void *Kv, const 
     const auto *K = static_cast<const __nv_bfloat16 *>(Kv);
     const auto *V = static_cast<const __nv_bfloat16 *>(Vv);
     { TimerScope ts(pl, kTDecide, st);
-    k_zone_decide<<<g.batch, 1024, 0, st>>>(g, pl.zone_part, pl.zone_a, pl.p.eps, pl.fixed_idx,
+    k_zone_decide<<<g.batch, 1024, 0, st>>>(g, pl.zone_part, pl.zone_a, pl.p.eps, pl.fixed_idx, false,
                                             pl.zone_B, pl.zone_shape, pl.zone_blk0, pl.nb, pl.blk_off,
                                             pl.tile_blk, pl.zone_qt0, pl.nqt, pl.qt_row, pl.qt_blk); }
     return launch_gather_select(pl, Q, K, V, st);
+}
+
+// The plan from decisions already in zone_B / zone_shape: block table, then
+// as launch_plan_finish.
+prism_status launch_plan_given(Plan &pl, const void *Qv, const void *Kv, const void *Vv, cudaStream_t st) {
+    const Geo &g = pl.g;
+    { TimerScope ts(pl, kTDecide, st);
+    k_zone_decide<<<g.batch, 1024, 0, st>>>(g, pl.zone_part, pl.zone_a, pl.p.eps, pl.fixed_idx, true,
+                                            pl.zone_B, pl.zone_shape, pl.zone_blk0, pl.nb, pl.blk_off,
+                                            pl.tile_blk, pl.zone_qt0, pl.nqt, pl.qt_row, pl.qt_blk); }
+    PRISM_CUDA_OK(cudaGetLastError());
+    return launch_gather_select(pl, static_cast<const __nv_bfloat16 *>(Qv), static_cast<const __nv_bfloat16 *>(Kv),
+                                static_cast<const __nv_bfloat16 *>(Vv), st);
 }
 
 static int permute_pool_threads(const Geo &g) { return g.C / 8 >= 384 ? 384 : ((g.C / 8 + 31) / 32) * 32; }
@@ -1109,7 +1129,7 @@ prism_status launch_zone_decisions(const Geo &g, double eps, int fixed_idx, cons
     const size_t smem_v = 2 * 8 * 8 * kStatChunk * sizeof(float);
     k_zone_stats_v<<<dim3(nchunk, g.M, g.batch), 128, smem_v, st>>>(V, g, zone_part);
     k_zone_stats_a<<<dim3(g.M, g.batch), 512, 0, st>>>(a, g, zone_a);
-    k_zone_decide<<<g.batch, 1024, 0, st>>>(g, zone_part, zone_a, eps, fixed_idx, zone_B, zone_shape,
+    k_zone_decide<<<g.batch, 1024, 0, st>>>(g, zone_part, zone_a, eps, fixed_idx, false, zone_B, zone_shape,
                                             zone_blk0, nb, blk_off, tile_blk, zone_qt0, nqt, qt_row, qt_blk);
     PRISM_CUDA_OK(cudaGetLastError());
     return PRISM_OK;

@@ -390,6 +390,40 @@ prism_status prism_plan_build_finish(prism_plan *plan, const void *Q, const void
     return s;
 }
 
+prism_status prism_plan_build_with_zones(prism_plan *plan, const void *Q, const void *K, const void *V,
+                                        const int *zone_B, const int *zone_shape, void *stream) {
+    g_last_error.clear();
+    if (!plan || !Q || !K || !V || !zone_B || !zone_shape)
+        return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_plan_build_with_zones");
+    prism_status s = device_guard(plan->pl);
+    if (s != PRISM_OK) return s;
+    Plan &pl = plan->pl;
+    if (pl.p.hilbert_block) return fail(PRISM_ERR_STATE, "a Hilbert-order plan has no zones");
+    const uintptr_t al = (uintptr_t)Q | (uintptr_t)K | (uintptr_t)V;
+    if (al & 15) return fail(PRISM_ERR_INVALID_ARG, "Q, K, V must be 16-byte aligned");
+    int table[kNumShapes][3];
+    host_shape_table(table);
+    const size_t nz = (size_t)pl.g.batch * pl.g.M;
+    for (size_t z = 0; z < nz; ++z) {
+        const int B = zone_B[z], c = zone_shape[z];
+        if (B != 64 && B != 128 && B != 256)
+            return fail(PRISM_ERR_INVALID_ARG, "zone %zu (sample %zu): volume %d is not 64, 128 or 256", z % pl.g.M,
+                        z / pl.g.M, B);
+        if (c < 0 || c >= kNumShapes || (1 << (table[c][0] + table[c][1] + table[c][2])) != B)
+            return fail(PRISM_ERR_INVALID_ARG, "zone %zu (sample %zu): shape %d is not a candidate of volume %d",
+                        z % pl.g.M, z / pl.g.M, c, B);
+    }
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    pl.have_fwd = false;
+    pl.built = false;
+    pl.have_stats = false;
+    PRISM_CUDA_OK(cudaMemcpyAsync(pl.zone_B, zone_B, nz * sizeof(int), cudaMemcpyHostToDevice, st));
+    PRISM_CUDA_OK(cudaMemcpyAsync(pl.zone_shape, zone_shape, nz * sizeof(int), cudaMemcpyHostToDevice, st));
+    s = launch_plan_given(pl, Q, K, V, st);
+    if (s == PRISM_OK) pl.built = true;
+    return s;
+}
+
 prism_status prism_plan_update_qkv(prism_plan *plan, const void *Q, const void *K, const void *V, void *stream) {
     g_last_error.clear();
     if (!plan || !Q || !K || !V) return fail(PRISM_ERR_INVALID_ARG, "NULL argument to prism_plan_update_qkv");

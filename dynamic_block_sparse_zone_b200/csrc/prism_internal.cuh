@@ -117,6 +117,7 @@ prism_status launch_plan(Plan &pl, const void *Q, const void *K, const void *V, 
                          cudaStream_t st);
 prism_status launch_plan_stats(Plan &pl, const void *V, const float *a, cudaStream_t st);
 prism_status launch_plan_finish(Plan &pl, const void *Q, const void *K, const void *V, cudaStream_t st);
+prism_status launch_plan_given(Plan &pl, const void *Q, const void *K, const void *V, cudaStream_t st);
 prism_status launch_attn_fwd_tc(Plan &pl, void *O, float *lse, cudaStream_t st);
 prism_status launch_attn_fwd_taylor(Plan &pl, void *O, float *lse, cudaStream_t st);
 bool taylor_fits(const Geo &g);  // the Taylor forward's shared memory fits one CTA

@@ -164,6 +164,25 @@ PRISM_API prism_status prism_plan_stats_slice(prism_plan *plan, void **buf, size
 PRISM_API prism_status prism_plan_build_finish(prism_plan *plan, const void *Q, const void *K, const void *V,
                                                void *stream);
 
+/* Builds the plan from zone decisions the caller gives instead of the zone
+ * statistics [Prism guide, Method section 2: each zone's block volume B(m)
+ * and block shape; this call takes them as inputs and performs the rest of
+ * the plan]: the block table, the permutation and pooling, the selection and
+ * the CSR / CSC, exactly as prism_plan_build does after its own decisions.
+ *   zone_B      host int [batch][N/512]: 64, 128 or 256
+ *   zone_shape  host int [batch][N/512]: index into the 16-entry candidate
+ *               table (see prism_plan_view) whose volume is zone_B
+ *   Q, K, V     device, as prism_plan_build (16-byte aligned)
+ * Both host arrays are read before the call returns (the caller keeps them).
+ * fixed_shape is not applied; a head-sharded plan needs no statistics
+ * exchange on this path.  Errors: PRISM_ERR_INVALID_ARG for a NULL or
+ * misaligned pointer or an entry outside the table (message names the zone),
+ * PRISM_ERR_STATE for a Hilbert-order plan (it has no zones).  Use: stage-wise
+ * checks of the downstream steps, and decisions computed once for several
+ * layers.                                                                    */
+PRISM_API prism_status prism_plan_build_with_zones(prism_plan *plan, const void *Q, const void *K, const void *V,
+                                                   const int *zone_B, const int *zone_shape, void *stream);
+
 /* Plan reuse: gathers new Q, K, V (device, layouts above) into the plan's
  * block-contiguous copies using the plan's existing zone shapes, permutation
  * and selection, which are not recomputed.  Subsequent prism_attn_fwd /

@@ -237,8 +237,14 @@ class OraclePlan:
 
 
 def plan(Q_bits, K_bits, V_bits, a, T, H, W, heads, D, k, p, max_frac=0.0,
-         eps=1e-6, fixed_shape=None, with_select=True) -> OraclePlan:
-    """Full oracle plan for one sample.  *_bits: [N, heads, D] uint16 (bf16)."""
+         eps=1e-6, fixed_shape=None, with_select=True, zone_decisions=None) -> OraclePlan:
+    """Full oracle plan for one sample.  *_bits: [N, heads, D] uint16 (bf16).
+
+    zone_decisions: optional (zone_B, zone_shape) per zone that replace the
+    volumes and shapes Method sections 1-2 derive from the statistics; the
+    block table, permutation, pooling and selection (Method sections 2-3)
+    then follow from them, so the later steps can be checked on their own.
+    The statistics are still computed and returned; the tie gaps are +inf."""
     N = T * H * W
     sv, sa, am, amax = zone_stats(V_bits.reshape(N, heads * D), a, T, H, W)
     fixed = -1
@@ -247,6 +253,18 @@ def plan(Q_bits, K_bits, V_bits, a, T, H, W, heads, D, k, p, max_frac=0.0,
         table = [tuple(r) for r in shape_table()]
         fixed = table.index(ex)
     dec = zone_decide(sv, sa, am, amax, eps, fixed)
+    if zone_decisions is not None:
+        zB = np.asarray(zone_decisions[0], np.int32).reshape(-1)
+        zs = np.asarray(zone_decisions[1], np.int32).reshape(-1)
+        table = shape_table()
+        if zB.shape != dec["zone_B"].shape or zs.shape != zB.shape:
+            raise ValueError("zone_decisions: one volume and one shape per zone")
+        if np.any((zs < 0) | (zs >= len(table))):
+            raise ValueError("zone_decisions: shape index outside the candidate table")
+        if np.any(zB != (1 << table[zs].sum(axis=1))):
+            raise ValueError("zone_decisions: a volume differs from its shape's")
+        dec = dict(dec, zone_B=zB.copy(), zone_shape=zs.copy(),
+                   gap_shape=np.full(zB.shape, np.inf), gap_rho=np.full(zB.shape, np.inf))
     box = blocks(T, H, W, dec["zone_shape"])
     pm = perm(T, H, W, box)
     Qb = pool(Q_bits.reshape(N, heads, D), T, H, W, heads, D, box)

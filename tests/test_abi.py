@@ -88,6 +88,7 @@ def test_null_arguments_are_rejected(lib):
     assert lib.prism_plan_build_stats(None, None, None, None) == 1
     assert lib.prism_plan_build_finish(None, None, None, None, None) == 1
     assert lib.prism_plan_stats_slice(None, None, None, None, None) == 1
+    assert lib.prism_plan_build_with_zones(None, None, None, None, None, None, None) == 1
     assert b"NULL" in lib.prism_last_error()
     lib.prism_plan_destroy(None)  # no-op
 

@@ -246,6 +246,42 @@ def test_blocks_tile_each_zone_and_perm_is_block_contiguous():
     assert zone_of_block == sorted(zone_of_block)
 
 
+def test_plan_with_given_zone_decisions_uses_them():
+    """oracle.plan(zone_decisions=...) builds its blocks from the given shapes
+    (checked against the hand-written candidate table), pools and selects on
+    them, refuses a volume that differs from its shape's, and leaves the
+    statistics it computes unchanged."""
+    w = scaled(WORKLOADS["dynamic_16x32x32"], heads=2, head_dim=64)
+    inp = make_inputs(w, 5)
+    Qb, Kb, Vb = (bf16_bits(x[0]) for x in (inp.Q, inp.K, inp.V))
+    a = inp.a[0].numpy()
+    rs = np.random.default_rng(21)
+    shapes = golden_shapes()
+    M = w.N // 512
+    zs = rs.integers(0, 16, size=M).astype(np.int32)
+    zB = np.array([int(np.prod(shapes[c])) for c in zs], np.int32)
+    args = (Qb, Kb, Vb, a, w.T, w.H, w.W, w.heads, w.head_dim, w.top_k, np.float32(w.top_p))
+    ref = oracle.plan(*args)
+    pl = oracle.plan(*args, zone_decisions=(zB, zs))
+    assert np.array_equal(pl.zone_B, zB) and np.array_equal(pl.zone_shape, zs)
+    assert np.array_equal(pl.box, oracle.blocks(w.T, w.H, w.W, zs))
+    assert [tuple(b[3:]) for b in pl.box] == [shapes[c] for c in zs for _ in range(512 // int(np.prod(shapes[c])))]
+    assert pl.nb == sum(512 // v for v in zB)
+    np.testing.assert_array_equal(pl.sig_v, ref.sig_v)
+    # the pooled means are block means of the given blocks
+    j = pl.nb // 2
+    t0, h0, w0, bt, bh, bw = pl.box[j]
+    toks = [(t * w.H + h) * w.W + x for t in range(t0, t0 + bt) for h in range(h0, h0 + bh) for x in range(w0, w0 + bw)]
+    q = (Qb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    np.testing.assert_allclose(pl.Qbar[:, j, :], q[toks].mean(axis=0), rtol=0, atol=1e-12)
+    # selection on the given blocks: every row holds at least top_k blocks and its own mass >= p
+    assert np.all(pl.cnt >= min(w.top_k, pl.nb))
+    bad = zB.copy()
+    bad[0] = 128 if zB[0] != 128 else 64
+    with pytest.raises(ValueError):
+        oracle.plan(*args, zone_decisions=(bad, zs))
+
+
 def test_pool_closed_form_on_linear_field():
     T, H, W, heads, D = 8, 16, 16, 2, 4
     t, h, w = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")

@@ -50,10 +50,11 @@ def run_gpu(w, inp, backward=False):
     return out
 
 
-def oracle_plan(w, inp, b=0, heads=None):
+def oracle_plan(w, inp, b=0, heads=None, zone_decisions=None):
     Qb, Kb, Vb = (bf16_bits(x[b]) for x in (inp.Q, inp.K, inp.V))
     pl = oracle.plan(Qb, Kb, Vb, inp.a[b].cpu().numpy(), w.T, w.H, w.W, w.heads, w.head_dim, w.top_k,
-                     _f32(w.top_p), _f32(w.max_frac), fixed_shape=w.fixed_shape, with_select=heads is None)
+                     _f32(w.top_p), _f32(w.max_frac), fixed_shape=w.fixed_shape, with_select=heads is None,
+                     zone_decisions=zone_decisions)
     if heads is not None:  # selection of a few heads only (heads are independent)
         cnt, cols, diag = oracle.select(pl.Qbar[heads], pl.Kbar[heads], w.top_k, _f32(w.top_p), _f32(w.max_frac))
         pl.cnt, pl.cols, pl.diag = cnt, cols, diag
@@ -237,6 +238,99 @@ def test_backward_parity(name):
     assert_close("dK", g["dK"][0].float().cpu().numpy()[req_t, req_h], dK_ref)
     assert_close("dV", g["dV"][0].float().cpu().numpy()[req_t, req_h], dV_ref)
     check_gradient_sums(g, inp)
+
+
+# ---------------------------------------------------------------------------
+# Stage-wise parity: the steps after the zone decisions, fed given decisions
+# (prism_plan_build_with_zones), so that a decision flipped at a near-tie
+# upstream cannot hide a fault downstream, and every candidate shape is used.
+# ---------------------------------------------------------------------------
+def _small_d64():
+    return scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=3, head_dim=64, planted=2)
+
+
+def _random_zone_decisions(w, seed):
+    """Seeded shapes drawn uniformly over the 16 candidates, one per zone, and
+    their volumes."""
+    rs = np.random.default_rng(seed)
+    table = oracle.shape_table()
+    zs = rs.integers(0, len(table), size=w.N // 512).astype(np.int32)
+    return (1 << table[zs].sum(axis=1)).astype(np.int32), zs
+
+
+def run_gpu_given(w, inp, zB, zs, backward=False):
+    P = _lib()
+    plan = P.PrismPlan(P.params_for(w, batch=1))
+    Q, K, V = (x.cuda() for x in (inp.Q, inp.K, inp.V))
+    plan.build_with_zones(Q, K, V, zB[None], zs[None])
+    O, lse = plan.fwd()
+    out = dict(O=O, lse=lse)
+    if backward:
+        out["dQ"], out["dK"], out["dV"] = plan.bwd(O, inp.dO.cuda())
+    torch.cuda.synchronize()
+    plan.check()
+    out["view"] = plan.view()
+    return out
+
+
+@pytest.mark.parametrize("name", ["dynamic_16x32x32", "dynamic_small_d64"])
+def test_stagewise_plan_from_the_oracle_decisions(name):
+    w = WORKLOADS[name] if name in WORKLOADS else _small_d64()
+    inp = make_inputs(w, 4)
+    pl, bits = oracle_plan(w, inp)
+    g = run_gpu_given(w, inp, pl.zone_B, pl.zone_shape)
+    compare_plan(w, pl, g["view"])
+    check_forward(w, inp, g, pl, bits, 1536)
+
+
+@pytest.mark.parametrize("name,seed", [("dynamic_16x32x32", 31), ("dynamic_small_d64", 32), ("tiny_8x16x16", 33)])
+def test_plan_from_random_zone_decisions_forward_backward(name, seed):
+    w = scaled(WORKLOADS[name] if name in WORKLOADS else _small_d64(), backward=True)
+    inp = make_inputs(w, seed)
+    zB, zs = _random_zone_decisions(w, seed)
+    pl, bits = oracle_plan(w, inp, zone_decisions=(zB, zs))
+    g = run_gpu_given(w, inp, zB, zs, backward=True)
+    assert np.array_equal(g["view"]["zone_shape"][0].cpu().numpy(), zs)
+    compare_plan(w, pl, g["view"])
+    check_forward(w, inp, g, pl, bits, 1536)
+    dOb = bf16_bits(inp.dO[0])
+    rs = np.random.default_rng(seed)
+    req_h, req_t = sample_rows(rs, w, 512)
+    dQ_ref = oracle.attn_bwd_dq_rows(pl, *bits, dOb, req_h, req_t)
+    assert_close("dQ", g["dQ"][0].float().cpu().numpy()[req_t, req_h], dQ_ref)
+    req_h, req_t = sample_rows(rs, w, 256)
+    dK_ref, dV_ref = oracle.attn_bwd_dkv_rows(pl, *bits, dOb, req_h, req_t)
+    assert_close("dK", g["dK"][0].float().cpu().numpy()[req_t, req_h], dK_ref)
+    assert_close("dV", g["dV"][0].float().cpu().numpy()[req_t, req_h], dV_ref)
+
+
+def test_build_with_zones_rejections():
+    P = _lib()
+    w = WORKLOADS["dynamic_16x32x32"]
+    inp = make_inputs(w, 2)
+    Q, K, V = (x.cuda() for x in (inp.Q, inp.K, inp.V))
+    zB, zs = _random_zone_decisions(w, 3)
+    plan = P.PrismPlan(P.params_for(w))
+    for mutate in (lambda b, s: b.__setitem__(3, 96),                      # not a volume
+                   lambda b, s: b.__setitem__(5, 64 if b[5] != 64 else 128),  # volume differs from the shape's
+                   lambda b, s: s.__setitem__(7, 16),                      # outside the table
+                   lambda b, s: s.__setitem__(0, -1)):
+        b2, s2 = zB.copy(), zs.copy()
+        mutate(b2, s2)
+        with pytest.raises(P.PrismError) as e:
+            plan.build_with_zones(Q, K, V, b2[None], s2[None])
+        assert e.value.status == 1 and "zone" in str(e.value)
+    with pytest.raises(P.PrismError) as e:  # refused entries build nothing: still no plan
+        plan.fwd()
+    assert e.value.status == 6
+    plan.build_with_zones(Q, K, V, zB[None], zs[None])  # the plan stays usable
+    plan.fwd()
+    torch.cuda.synchronize()
+    plan.check()
+    hp = P.PrismPlan(P.params_for(w, hilbert_block=128))
+    with pytest.raises(P.PrismError) as e:
+        hp.build_with_zones(Q, K, V, zB[None], zs[None])
+    assert e.value.status == 6
 
 
 def check_gradient_sums(g, inp, b=0):
