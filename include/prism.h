@@ -173,7 +173,9 @@ PRISM_API prism_status prism_plan_build_finish(prism_plan *plan, const void *Q, 
  *   zone_shape  host int [batch][N/512]: index into the 16-entry candidate
  *               table (see prism_plan_view) whose volume is zone_B
  *   Q, K, V     device, as prism_plan_build (16-byte aligned)
- * Both host arrays are read before the call returns (the caller keeps them).
+ * Both host arrays are read before the call returns (the caller keeps them;
+ * being pageable host memory, their copy may wait for work already queued on
+ * the stream).
  * fixed_shape is not applied; a head-sharded plan needs no statistics
  * exchange on this path.  Errors: PRISM_ERR_INVALID_ARG for a NULL or
  * misaligned pointer or an entry outside the table (message names the zone),
