@@ -333,6 +333,50 @@ def test_build_with_zones_rejections():
     assert e.value.status == 6
 
 
+def test_head_shards_built_from_given_zone_decisions():
+    """Head shards built from the same given decisions (no statistics, no
+    exchange) hold the whole layer's plan: identical permutation and block
+    table, their heads' selections, and bit-identical forward outputs."""
+    P = _lib()
+    w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=4, planted=2)
+    inp = make_inputs(w, 6)
+    Q, K, V = (x.cuda() for x in (inp.Q, inp.K, inp.V))
+    zB, zs = _random_zone_decisions(w, 41)
+    whole = P.PrismPlan(P.params_for(w))
+    whole.build_with_zones(Q, K, V, zB[None], zs[None])
+    O_all, lse_all = whole.fwd()
+    v_all = whole.view()
+    torch.cuda.synchronize()
+    hs = 2
+    for r in range(2):
+        prm = P.params_for(w)
+        prm.heads, prm.heads_total, prm.head_offset = hs, w.heads, r * hs
+        plan = P.PrismPlan(prm)
+        sl = slice(r * hs, (r + 1) * hs)
+        Qr, Kr, Vr = (x[:, :, sl].contiguous() for x in (Q, K, V))
+        plan.build_with_zones(Qr, Kr, Vr, zB[None], zs[None])
+        O_r, lse_r = plan.fwd()
+        torch.cuda.synchronize()
+        plan.check()
+        v = plan.view()
+        for key in ("zone_B", "zone_shape", "perm"):
+            assert torch.equal(v[key], v_all[key]), key
+        nb = int(v["n_blocks"][0])
+        assert nb == int(v_all["n_blocks"][0])
+        assert torch.equal(v["blk_off"][:, :nb + 1], v_all["blk_off"][:, :nb + 1])
+        rp, rp_all = v["row_ptr"].cpu().numpy(), v_all["row_ptr"].cpu().numpy()
+        col, col_all = v["col_idx"].cpu().numpy(), v_all["col_idx"].cpu().numpy()
+        nbmax = v["nbmax"]
+        for hh in range(hs):
+            for i in range(nb):
+                ra, rb = hh * nbmax + i, (r * hs + hh) * nbmax + i
+                assert np.array_equal(col[rp[ra]:rp[ra + 1]], col_all[rp_all[rb]:rp_all[rb + 1]])
+        assert torch.equal(O_r, O_all[:, :, sl])
+        assert torch.equal(lse_r, lse_all[:, sl])
+        plan.close()
+    whole.close()
+
+
 def check_gradient_sums(g, inp, b=0):
     """Properties of softmax attention at any size: for every query the dS row
     sums to zero, so sum_t dK_t = 0; the P row sums to one, so
