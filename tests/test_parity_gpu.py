@@ -304,6 +304,30 @@ def test_plan_from_random_zone_decisions_forward_backward(name, seed):
     assert_close("dV", g["dV"][0].float().cpu().numpy()[req_t, req_h], dV_ref)
 
 
+def test_batch_two_from_given_zone_decisions():
+    """Two samples with their own given decisions (so their own block counts):
+    each sample's plan and forward match the oracle fed that sample's
+    decisions."""
+    P = _lib()
+    w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=2, planted=2, batch=2)
+    inp = make_inputs(w, 8)
+    dec = [_random_zone_decisions(w, 51 + b) for b in range(2)]
+    plan = P.PrismPlan(P.params_for(w))
+    Q, K, V = (x.cuda() for x in (inp.Q, inp.K, inp.V))
+    plan.build_with_zones(Q, K, V, np.stack([d[0] for d in dec]), np.stack([d[1] for d in dec]))
+    O, lse = plan.fwd()
+    torch.cuda.synchronize()
+    plan.check()
+    g = dict(O=O, lse=lse, view=plan.view())
+    nbs = []
+    for b in range(2):
+        pl, bits = oracle_plan(w, inp, b=b, zone_decisions=dec[b])
+        compare_plan(w, pl, g["view"], b=b)
+        check_forward(w, inp, g, pl, bits, 512, b=b)
+        nbs.append(pl.nb)
+    assert nbs[0] != nbs[1]  # the samples' block tables differ
+
+
 def test_build_with_zones_rejections():
     P = _lib()
     w = WORKLOADS["dynamic_16x32x32"]
