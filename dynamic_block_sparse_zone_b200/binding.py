@@ -390,21 +390,50 @@ def prism_zone_shapes_noalloc(params: Params, V: torch.Tensor, a_norm: torch.Ten
     _need(a_norm, "a_norm", torch.float32, (params.batch, params.T, params.H, params.W))
     _need(zone_B, "zone_B", torch.int32, (params.batch, M))
     _need(zone_shape, "zone_shape", torch.int32, (params.batch, M))
+    if not (V.device == a_norm.device == zone_B.device == zone_shape.device):
+        raise ValueError("V, a_norm, zone_B and zone_shape must be on one GPU")
     c = params.to_c()
-    _check(load_library().prism_zone_shapes_noalloc(ctypes.byref(c), _ptr(V), _ptr(a_norm), _ptr(zone_B),
-                                                    _ptr(zone_shape), _stream()))
+    # the library launches on the current device with that device's copy of
+    # its scratch array: make the tensors' GPU current for the call
+    with torch.cuda.device(V.device):
+        _check(load_library().prism_zone_shapes_noalloc(ctypes.byref(c), _ptr(V), _ptr(a_norm), _ptr(zone_B),
+                                                        _ptr(zone_shape), _stream()))
     return zone_B, zone_shape
 
 
 # Module-level names that mirror the C ABI.
+def _through_host(t: torch.Tensor, group) -> bool:
+    """gloo moves host tensors only: device tensors then go through host copies
+    (NCCL takes them as they are)."""
+    import torch.distributed as dist
+    return t.is_cuda and dist.get_backend(group) == "gloo"
+
+
 def exchange_zone_stats(whole: torch.Tensor, mine: torch.Tensor, group=None):
     """All-gather of the ranks' zone-statistics slices into `whole` (rank order =
     slice order).  Single process: nothing to exchange."""
     import torch.distributed as dist
     if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
         return whole
+    if _through_host(whole, group):
+        host = torch.empty(whole.shape, dtype=whole.dtype)
+        dist.all_gather_into_tensor(host, mine.cpu(), group=group)
+        whole.copy_(host)
+        return whole
     dist.all_gather_into_tensor(whole, mine.clone(), group=group)
     return whole
+
+
+def _all_to_all(send: torch.Tensor, group) -> torch.Tensor:
+    import torch.distributed as dist
+    if _through_host(send, group):
+        host = send.cpu()
+        recv = torch.empty_like(host)
+        dist.all_to_all_single(recv, host, group=group)
+        return recv.to(send.device)
+    recv = torch.empty_like(send)
+    dist.all_to_all_single(recv, send, group=group)
+    return recv
 
 
 def sequence_to_heads(x: torch.Tensor, group=None) -> torch.Tensor:
@@ -421,8 +450,7 @@ def sequence_to_heads(x: torch.Tensor, group=None) -> torch.Tensor:
         raise ValueError("heads must divide evenly among the ranks")
     h = Hn // R
     send = x.reshape(B, n, R, h, D).permute(2, 0, 1, 3, 4).contiguous()  # [dest rank][B][n][h][D]
-    recv = torch.empty_like(send)                                         # [source rank][B][n][h][D]
-    dist.all_to_all_single(recv, send, group=group)
+    recv = _all_to_all(send, group)                                       # [source rank][B][n][h][D]
     return recv.permute(1, 0, 2, 3, 4).reshape(B, R * n, h, D)
 
 
@@ -438,8 +466,7 @@ def heads_to_sequence(y: torch.Tensor, group=None) -> torch.Tensor:
         raise ValueError("tokens must divide evenly among the ranks")
     n = N // R
     send = y.reshape(B, R, n, h, D).permute(1, 0, 2, 3, 4).contiguous()  # [dest rank][B][n][h][D]
-    recv = torch.empty_like(send)                                         # [source rank][B][n][h][D]
-    dist.all_to_all_single(recv, send, group=group)
+    recv = _all_to_all(send, group)                                       # [source rank][B][n][h][D]
     return recv.permute(1, 2, 0, 3, 4).reshape(B, n, R * h, D)
 
 
@@ -450,8 +477,12 @@ def gather_sequence(t: torch.Tensor, group=None) -> torch.Tensor:
     if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
         return t
     R = dist.get_world_size(group)
-    parts = torch.empty((R * t.shape[0],) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
-    dist.all_gather_into_tensor(parts, t.contiguous(), group=group)  # rank-major concatenation
+    host = _through_host(t, group)
+    src = t.contiguous().cpu() if host else t.contiguous()
+    parts = torch.empty((R * t.shape[0],) + tuple(t.shape[1:]), dtype=t.dtype, device=src.device)
+    dist.all_gather_into_tensor(parts, src, group=group)  # rank-major concatenation
+    if host:
+        parts = parts.to(t.device)
     parts = parts.view((R,) + tuple(t.shape))
     return parts.movedim(0, 1).reshape((t.shape[0], R * t.shape[1]) + tuple(t.shape[2:]))
 

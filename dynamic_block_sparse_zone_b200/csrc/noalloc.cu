@@ -29,19 +29,60 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[PRISM_NOALLOC_S
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mu;
+// Per device: the scratch address and the id of the CUDA context it was
+// looked up in.  A device address belongs to one context; after
+// cudaDeviceReset the device's next primary context has a new id, so the
+// address, the kernel attributes and the constant table are set up again.
 unsigned char *g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// The id of the calling thread's current context (unique for the life of the
+// process; ids are never reused, unlike CUcontext handles).
+prism_status current_context_id(unsigned long long *id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    if (!get_current || !get_id) {
+        void *p1 = nullptr, *p2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p1, cudaEnableDefault, &q1) != cudaSuccess ||
+            q1 != cudaDriverEntryPointSuccess ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &p2, cudaEnableDefault, &q2) != cudaSuccess ||
+            q2 != cudaDriverEntryPointSuccess)
+            return fail(PRISM_ERR_CUDA, "cuCtxGetCurrent / cuCtxGetId unavailable");
+        get_current = reinterpret_cast<CtxGetCurrentFn>(p1);
+        get_id = reinterpret_cast<CtxGetIdFn>(p2);
+    }
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS) return fail(PRISM_ERR_CUDA, "cuCtxGetCurrent failed");
+    if (!ctx) {  // the runtime has not made its primary context current on this thread yet
+        int dev = 0;
+        PRISM_CUDA_OK(cudaGetDevice(&dev));
+        PRISM_CUDA_OK(cudaSetDevice(dev));
+        if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return fail(PRISM_ERR_CUDA, "no current CUDA context");
+    }
+    if (get_id(ctx, id) != CUDA_SUCCESS) return fail(PRISM_ERR_CUDA, "cuCtxGetId failed");
+    return PRISM_OK;
+}
 }  // namespace
 
-// Once per device, with that device current: the device address of the
-// scratch array, kernel attributes and the candidate-shape table.
+// Once per CUDA context of a device, with that device current: the device
+// address of the scratch array, kernel attributes and the candidate-shape
+// table.
 static prism_status noalloc_setup(int dev, unsigned char **out) {
     std::lock_guard<std::mutex> lock(g_setup_mu);
-    if (!g_scratch_ptr[dev]) {
+    unsigned long long ctx = 0;
+    prism_status s = current_context_id(&ctx);
+    if (s != PRISM_OK) return s;
+    if (!g_scratch_ptr[dev] || g_scratch_ctx[dev] != ctx) {
         unsigned char *p = nullptr;
         PRISM_CUDA_OK(cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_noalloc_scratch));
-        prism_status s = configure_zone_kernels();
+        s = configure_zone_kernels();
         if (s != PRISM_OK) return s;
         g_scratch_ptr[dev] = p;
+        g_scratch_ctx[dev] = ctx;
     }
     *out = g_scratch_ptr[dev];
     return PRISM_OK;
@@ -79,8 +120,9 @@ extern "C" PRISM_API prism_status prism_zone_shapes_noalloc(const prism_params *
     g.M = g.MT * g.MH * g.MW;
     g.nbmax = g.N / 64;
     g.C = p->heads * p->head_dim;
-    if (p->heads_total != 0 && p->heads_total != p->heads)
-        return fail(PRISM_ERR_UNSUPPORTED, "prism_zone_shapes_noalloc takes every head of the layer (no sharding)");
+    if ((p->heads_total != 0 && p->heads_total != p->heads) || p->head_offset != 0)
+        return fail(PRISM_ERR_UNSUPPORTED,
+                    "prism_zone_shapes_noalloc takes every head of the layer (heads_total 0 or heads, head_offset 0)");
     g.Ctot = g.C;
     g.chunk0 = 0;
     g.nchunk_tot = (g.C + kStatChunk - 1) / kStatChunk;

@@ -224,10 +224,16 @@ PRISM_API prism_status prism_attn_fwd(prism_plan *plan, void *O, float *lse, voi
 PRISM_API prism_status prism_attn_fwd_taylor(prism_plan *plan, void *O, float *lse, void *stream);
 
 /* Gradient of sum(O * dO) with respect to Q, K, V through the same sparse
- * attention (the plan and the forward's statistics are reused).  O is the
- * forward's output and dO the incoming gradient (device, bf16, user layout);
- * dQ, dK, dV are written (device, bf16, user layout).  Returns
- * PRISM_ERR_STATE if no forward ran since the last build.                  */
+ * attention (the plan and the forward's statistics are reused).  The pages
+ * define no such call: it is the standard softmax-attention gradient taken
+ * over the selected blocks S_i only [Prism guide, Method section 3 restricts
+ * the attention to S_i; the model is trained through it]:
+ *   P = exp(S/sqrt(D) - LSE), dV = P^T dO, dP = dO V^T,
+ *   dS = P (dP - rowsum(dO * O)), dQ = dS K / sqrt(D), dK = dS^T Q / sqrt(D).
+ * O is the forward's output and dO the incoming gradient (device, bf16, user
+ * layout); dQ, dK, dV are written (device, bf16, user layout).  dQ is summed
+ * in fp32 before its bf16 rounding.  Returns PRISM_ERR_STATE if no forward
+ * ran since the last build.                                                */
 PRISM_API prism_status prism_attn_bwd(prism_plan *plan, const void *O, const void *dO, void *dQ, void *dK,
                             void *dV, void *stream);
 
@@ -328,8 +334,11 @@ PRISM_API const char *prism_timer_name(int id);
  * until the process exits; a problem needing more (about
  * 24 * batch * N/512 * ceil(heads*head_dim/128) bytes plus 20 bytes per 64
  * tokens) returns PRISM_ERR_UNSUPPORTED before anything is launched.  The
- * first call on a device looks up the array's device address and sets kernel
- * attributes; make that first call before any stream capture.  All calls
+ * first call in a CUDA context (per device; again after cudaDeviceReset has
+ * replaced the device's primary context) looks up the array's device address,
+ * sets kernel attributes and uploads a small constant table; make that first
+ * call before any stream capture.  params' heads_total must be 0 or heads and
+ * head_offset 0 (the whole layer; no head shards).  All calls
  * share the array (nothing in it has to start at zero), so calls whose work
  * overlaps on the GPU (other streams or host threads) race: order them.
  * Only enqueues work on `stream`.                                          */

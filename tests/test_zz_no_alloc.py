@@ -63,3 +63,21 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
                                                     B._ptr(out), B._stream())
     assert st == 2
     assert b"scratch" in B.load_library().prism_last_error()
+
+
+def test_noalloc_rejects_a_head_shard():
+    """The entry point takes the whole layer: a head shard (head_offset > 0)
+    is refused, as prism_plan_create refuses heads outside heads_total."""
+    from dynamic_block_sparse_zone_b200.binding import Params, PrismError, prism_zone_shapes_noalloc
+    _lib()
+    w = WORKLOADS["tiny_8x16x16"]
+    inp = make_inputs(w, 5)
+    V, a = inp.V.cuda(), inp.a.cuda()
+    M = w.N // 512
+    zB = torch.zeros((1, M), dtype=torch.int32, device="cuda")
+    zS = torch.zeros((1, M), dtype=torch.int32, device="cuda")
+    p = Params(batch=1, T=w.T, H=w.H, W=w.W, heads=w.heads, head_dim=w.head_dim, top_k=w.top_k, top_p=w.top_p,
+               heads_total=0, head_offset=2)
+    with pytest.raises(PrismError) as e:
+        prism_zone_shapes_noalloc(p, V, a, zB, zS)
+    assert e.value.status == 2
