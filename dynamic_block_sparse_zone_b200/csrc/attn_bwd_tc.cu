@@ -14,28 +14,32 @@
 // key rows of a block whose column lacks the chunk's query block (a whole
 // warp's rows) take P = dS = 0 for that chunk.
 //
-// Per chunk c:
-//   S^T  = K Q_c^T         M=128 keys, N=64 queries   -> TMEM ST[c%3]
-//   dP^T = V dO_c^T        M=128 keys, N=64 queries   -> TMEM DP
-//   softmax warps: P^T, dS^T (bf16, packed over their own ST columns),
-//                  dS^T also to shared memory
+// Per chunk c (b = c & 1):
+//   S^T  = K Q_c^T         M=128 keys, N=64 queries   -> TMEM ST[b]
+//   dP^T = V dO_c^T        M=128 keys, N=64 queries   -> TMEM DP[b]
+//   softmax warps: P^T, dS^T (bf16, packed over their own ST[b] columns),
+//                  dS^T also to shared memory DS[b]
+//   dQ^T = K^T dS^T        both operands MN-major     -> TMEM DP[b] (dP^T is
+//                                                        consumed by then)
 //   dV  += P^T dO_c        A = P^T from TMEM          -> TMEM dV
 //   dK  += dS^T Q_c        A = dS^T from TMEM         -> TMEM dK
-//   dQ^T = K^T dS^T        both operands MN-major     -> TMEM ST[c%3]
 //   drain warps: dQ^T rows (lane = head-dim index) -> a [64 x D] fp32 tile in
 //                shared memory -> one TMA reduce-add into the dQ accumulator
-// Three ST buffers let S^T of chunk c+2 be issued while chunk c's dQ^T waits
-// to be drained; the single DP buffer is refilled (dP^T of chunk c+1) once the
-// softmax of chunk c has published its P^T / dS^T.
-// TMEM columns: dK [0,128), dV [128,256), ST[3] [256,448), DP [448,512).
+// Two ST and two DP buffers: S^T and dP^T of chunk c+2 are issued behind
+// chunk c's products, so the softmax of chunk c+1 (whose S^T and dP^T were
+// issued a chunk earlier) runs while the tensor cores work on chunk c.  dQ^T
+// is issued first among a chunk's products, so the drain reads it while dV,
+// dK and S^T of c+2 run; dP^T of c+2 then reuses the buffer.
+// TMEM columns: dK [0,128), dV [128,256), ST[2] [256,384), DP[2] [384,512).
 // In an ST buffer, after the softmax, columns [16g, 16g+8) hold P^T and
 // [16g+8, 16g+16) hold dS^T of queries [16g, 16g+16) (g = 0..3), packed as
 // bf16 pairs.
 //
-// dP^T of chunk c+1 waits for the softmax of chunk c, and the softmax of c+1
-// for that dP^T, so the softmax is spread over 16 warps, each owning one TMEM
-// lane quadrant (32 key rows) and 16 query columns, and does its arithmetic in
-// packed fp32 pairs.
+// The softmax runs in two groups of 8 warps that take alternate chunks (even
+// chunks, odd chunks), so one group's TMEM loads and stores overlap the other
+// group's exponentials.  In a group each warp owns one TMEM lane quadrant (32
+// key rows) and 32 query columns, taken as two 16-column halves, and does its
+// arithmetic in packed fp32 pairs.
 // Warp roles (704 threads): warp 0 TMA producer (K, V once; Q, dO, LSE,
 // Delta per chunk into a three-stage ring; LSE is kept negated, in log2 units), warp 1
 // MMA issuer, warps 2..17 softmax, warps 18..21 dQ drain (one head-dim row
@@ -54,7 +58,7 @@ constexpr int kSoftmaxWarps = 16;
 constexpr int kThreads = 32 * (2 + kSoftmaxWarps + 4);
 constexpr int kStages = 3;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColDK = 0, kColDV = 128, kColST = 256, kColDP = 448;
+constexpr uint32_t kColDK = 0, kColDV = 128, kColST = 256, kColDP = 384;  // ST[2], DP[2]: 64 columns each
 
 template <int D>
 struct Layout {
@@ -70,8 +74,8 @@ struct Layout {
     static constexpr uint32_t kVec = kDS + 2 * 16384;        // stage s: -LSE [64] f32 then Delta [64] f32
     static constexpr uint32_t kDQ = kVec + kStages * 512;    // dQ staging tile [64 queries][D] f32 (128-B aligned)
     static constexpr uint32_t kBars = kDQ + 64 * D * 4;
-    // kv, q_full[3], q_empty[3], s_full[2], p_full[2], dq_full[3], dq_empty[3], done
-    static constexpr uint32_t kNumBars = 18;
+    // kv, q_full[3], q_empty[3], s_full[2], p_full[2], dq_full[2], dq_empty[2], done
+    static constexpr uint32_t kNumBars = 16;
     // then per stage the column mask of its query chunk in a shared tile
     static constexpr uint32_t kMaskS = kBars + kNumBars * 8 + 16;
     static constexpr uint32_t kBytes = kMaskS + 16;
@@ -127,8 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const uint32_t bar_kv = sbase + L::kBars;
     const uint32_t bar_qf = bar_kv + 8, bar_qe = bar_qf + 8 * kStages, bar_sf = bar_qe + 8 * kStages;
-    const uint32_t bar_pf = bar_sf + 16, bar_df = bar_pf + 16, bar_de = bar_df + 8 * kStages;
-    const uint32_t bar_done = bar_de + 8 * kStages;
+    const uint32_t bar_pf = bar_sf + 16, bar_df = bar_pf + 16, bar_de = bar_df + 16;
+    const uint32_t bar_done = bar_de + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBars + L::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kBars + L::kNumBars * 8 + 8);
     volatile uint32_t *mask_s = reinterpret_cast<volatile uint32_t *>(smem + L::kMaskS);
@@ -139,12 +143,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int s = 0; s < kStages; ++s) {
                 mbar_init(bar_qf + 8 * s, 1);
                 mbar_init(bar_qe + 8 * s, 1);
-                mbar_init(bar_df + 8 * s, 1);
-                mbar_init(bar_de + 8 * s, 128);
             }
             for (int s = 0; s < 2; ++s) {
                 mbar_init(bar_sf + 8 * s, 1);
-                mbar_init(bar_pf + 8 * s, 32 * kSoftmaxWarps);
+                mbar_init(bar_pf + 8 * s, 32 * kSoftmaxWarps / 2);
+                mbar_init(bar_df + 8 * s, 1);
+                mbar_init(bar_de + 8 * s, 128);
             }
             mbar_init(bar_done, 1);
             *abort_flag = 0;
@@ -210,111 +214,107 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idAcc = idesc_bf16(128, D, true);           // A from TMEM, B MN-major
             constexpr uint32_t idDQ = idesc_bf16(128, 64, true, true);     // A and B MN-major
             bool ok = __all_sync(0xffffffffu, mbar_wait(bar_kv, 0, status, kSiteKV, abort_flag));
-            auto issue_st = [&](int c) -> bool {  // S^T of chunk c into ST[c % 3]
+            // S^T and dP^T of chunk c into ST[c & 1] and DP[c & 1]; dP^T waits
+            // for the drain of chunk c - 2 to have read its dQ^T out of DP[c & 1]
+            auto issue_sdp = [&](int c) -> bool {
                 const int st = c % kStages;
                 if (!__all_sync(0xffffffffu, mbar_wait(bar_qf + 8 * st, (c / kStages) & 1, status, kSiteQFull, abort_flag))) return false;
                 tc_fence_after();
-                const uint32_t sQ = sbase + L::kQ0 + st * L::kStage;
-                mma_over_d<D>(tmem + kColST + st * 64, sdesc(sbase + L::kK, 16, 1024), sdesc(sQ, 16, 1024), idST);
+                const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + L::kHalves * L::kQHalf;
+                mma_over_d<D>(tmem + kColST + (c & 1) * 64, sdesc(sbase + L::kK, 16, 1024), sdesc(sQ, 16, 1024), idST);
+                if (c >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar_de + 8 * (c & 1), ((c - 2) >> 1) & 1, status,
+                                                                 kSiteDQEmpty, abort_flag)))
+                    return false;
+                tc_fence_after();
+                mma_over_d<D>(tmem + kColDP + (c & 1) * 64, sdesc(sbase + L::kV, 16, 1024), sdesc(sO, 16, 1024), idST);
+                mma_commit(bar_sf + 8 * (c & 1));
                 return true;
             };
-            auto issue_dp = [&](int c) {  // dP^T of chunk c into DP (stage already waited by issue_st)
-                const uint32_t sO = sbase + L::kQ0 + (c % kStages) * L::kStage + L::kHalves * L::kQHalf;
-                mma_over_d<D>(tmem + kColDP, sdesc(sbase + L::kV, 16, 1024), sdesc(sO, 16, 1024), idST);
-                mma_commit(bar_sf + 8 * (c & 1));
-            };
-            if (ok) {
-                ok = issue_st(0);
-                if (ok) issue_dp(0);
-            }
-            if (ok && nchunk > 1) ok = issue_st(1);
+            if (ok) ok = issue_sdp(0);
+            if (ok && nchunk > 1) ok = issue_sdp(1);
             for (int c = 0; ok && c < nchunk; ++c) {
                 const int st = c % kStages;
                 if (!__all_sync(0xffffffffu, mbar_wait(bar_pf + 8 * (c & 1), (c >> 1) & 1, status, kSiteP, abort_flag))) break;
                 tc_fence_after();
-                if (c + 1 < nchunk) issue_dp(c + 1);
                 const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + L::kHalves * L::kQHalf;
-                const uint32_t tST = tmem + kColST + st * 64;
+                const uint32_t tST = tmem + kColST + (c & 1) * 64;
+                const uint32_t sDS = sbase + L::kDS + (c & 1) * 16384;
+                // dQ^T first, into the consumed dP^T buffer; K^T and dS^T
+                // MN-major: k-step kk (16 keys) 2048 B further in both
+                mma_ss8<128, 256, 384, 512, 640, 768, 896, 128, 256, 384, 512, 640, 768, 896>(
+                    tmem + kColDP + (c & 1) * 64, sdesc(sbase + L::kK, L::kKVHalf, 1024), sdesc(sDS, 8192, 1024), idDQ,
+                    0u);
+                mma_commit(bar_df + 8 * (c & 1));
                 const uint32_t acc = (c > 0) ? 1u : 0u;
                 // k-step kk of P^T / dS^T: columns 16 kk (+8 for dS^T);
                 // of dO / Q: 16 rows = 2048 B further
                 mma_ts4x2<16, 32, 48, 128, 256, 384>(tmem + kColDV, tST, sdesc(sO, L::kQHalf, 1024), tmem + kColDK,
                                                       tST + 8, sdesc(sQ, L::kQHalf, 1024), idAcc, acc);
                 mma_commit(bar_qe + 8 * st);
-                const uint32_t sDS = sbase + L::kDS + (c & 1) * 16384;
-                // K^T and dS^T MN-major: k-step kk (16 keys) 2048 B further in both
-                mma_ss8<128, 256, 384, 512, 640, 768, 896, 128, 256, 384, 512, 640, 768, 896>(
-                    tST, sdesc(sbase + L::kK, L::kKVHalf, 1024), sdesc(sDS, 8192, 1024), idDQ, 0u);
-                mma_commit(bar_df + 8 * st);
-                if (c + 2 < nchunk) {
-                    const int b2 = (c + 2) % kStages;  // = (c - 1) % 3: the buffer chunk c-1 used
-                    if (c >= 1 &&
-                        !__all_sync(0xffffffffu, mbar_wait(bar_de + 8 * b2, ((c - 1) / kStages) & 1, status, kSiteDQEmpty, abort_flag)))
-                        break;
-                    if (!issue_st(c + 2)) break;
-                }
+                if (c + 2 < nchunk && !issue_sdp(c + 2)) break;
             }
             mma_commit(bar_done);
         }
     } else if (warp < 2 + kSoftmaxWarps) {
         // ------------------------------------------------------------ softmax (key rows)
-        const int quad = warp & 3;          // TMEM lane quadrant this warp may access
-        const int cg = (warp - 2) >> 2;     // its 16 query columns [16 cg, 16 cg + 16)
+        const int quad = warp & 3;               // TMEM lane quadrant this warp may access
+        const int grp = (warp - 2) >> 3;         // the chunks of this parity
+        const int cg2 = ((warp - 2) >> 2) & 1;   // its 32 query columns [32 cg2, 32 cg2 + 32)
+        const int cg = (warp - 2) >> 2;          // epilogue column group
         const int rowid = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const bool live = rowid < kvalid;
         const int half = shared_tile ? (quad >> 1) : 0;  // which key block's rows (warp-uniform)
         bool ok = true;
-        for (int c = 0; c < nchunk; ++c) {
+        for (int c = grp; c < nchunk; c += 2) {
             const int st = c % kStages;
             ok = __all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * (c & 1), (c >> 1) & 1, status, kSiteS, abort_flag) &&
                                              mbar_wait(bar_qf + 8 * st, (c / kStages) & 1, status, kSiteQFull,
                                                        abort_flag));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t tST = tmem + kColST + st * 64 + 16 * cg + lane_off;
-            uint32_t sv[16], dv[16];
-            tmem_ld16(tST, sv);
-            tmem_ld16(tmem + kColDP + 16 * cg + lane_off, dv);
-            // -LSE (log2 units) and Delta of the 16 queries: the same for every lane
-            const uint32_t vec = sbase + L::kVec + st * 512 + cg * 64;
-            float4 N4[4], D4[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                N4[j] = lds_f4(vec + 16 * j);
-                D4[j] = lds_f4(vec + 256 + 16 * j);
-            }
-            tmem_wait_ld();
-            uint32_t pd[16];  // P^T pairs then dS^T pairs
-            // key rows past the block, or of a block whose column lacks this query
-            // chunk, are whole warps' rows, so the branch is warp-uniform
-            if (live && ((mask_s[st] >> half) & 1u)) {
-                const uint64_t s2 = splat2(scale_log2);
+            const bool act = live && ((mask_s[st] >> half) & 1u);
+            const uint32_t dsrow = sbase + L::kDS + (c & 1) * 16384 + rowid * 128;
+#pragma unroll 1
+            for (int sub = 0; sub < 2; ++sub) {
+                const int cq = 2 * cg2 + sub;  // 16 query columns [16 cq, 16 cq + 16)
+                const uint32_t tST = tmem + kColST + (c & 1) * 64 + 16 * cq + lane_off;
+                uint32_t sv[16], dv[16];
+                tmem_ld16(tST, sv);
+                tmem_ld16(tmem + kColDP + (c & 1) * 64 + 16 * cq + lane_off, dv);
+                const uint32_t vec = sbase + L::kVec + st * 512 + cq * 64;
+                float4 N4[4], D4[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const int q = 4 * j;
-                    float x0, x1, x2, x3, d0, d1, d2, d3;
-                    fma2(__uint_as_float(sv[q]), __uint_as_float(sv[q + 1]), s2, pair2(N4[j].x, N4[j].y), x0, x1);
-                    fma2(__uint_as_float(sv[q + 2]), __uint_as_float(sv[q + 3]), s2, pair2(N4[j].z, N4[j].w), x2, x3);
-                    const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
-                    // dS = P (dP - Delta), two lanes per instruction
-                    mul_sub2(p0, p1, __uint_as_float(dv[q]), __uint_as_float(dv[q + 1]), D4[j].x, D4[j].y, d0, d1);
-                    mul_sub2(p2, p3, __uint_as_float(dv[q + 2]), __uint_as_float(dv[q + 3]), D4[j].z, D4[j].w, d2, d3);
-                    pd[2 * j] = pack_bf16x2(p0, p1);
-                    pd[2 * j + 1] = pack_bf16x2(p2, p3);
-                    pd[8 + 2 * j] = pack_bf16x2(d0, d1);
-                    pd[8 + 2 * j + 1] = pack_bf16x2(d2, d3);
+                    N4[j] = lds_f4(vec + 16 * j);
+                    D4[j] = lds_f4(vec + 256 + 16 * j);
                 }
-            } else {
+                tmem_wait_ld();
+                uint32_t pd[16];
+                if (act) {
+                    const uint64_t s2 = splat2(scale_log2);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) pd[e] = 0u;
+                    for (int j = 0; j < 4; ++j) {
+                        const int q = 4 * j;
+                        float x0, x1, x2, x3, d0, d1, d2, d3;
+                        fma2(__uint_as_float(sv[q]), __uint_as_float(sv[q + 1]), s2, pair2(N4[j].x, N4[j].y), x0, x1);
+                        fma2(__uint_as_float(sv[q + 2]), __uint_as_float(sv[q + 3]), s2, pair2(N4[j].z, N4[j].w), x2, x3);
+                        const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+                        mul_sub2(p0, p1, __uint_as_float(dv[q]), __uint_as_float(dv[q + 1]), D4[j].x, D4[j].y, d0, d1);
+                        mul_sub2(p2, p3, __uint_as_float(dv[q + 2]), __uint_as_float(dv[q + 3]), D4[j].z, D4[j].w, d2, d3);
+                        pd[2 * j] = pack_bf16x2(p0, p1);
+                        pd[2 * j + 1] = pack_bf16x2(p2, p3);
+                        pd[8 + 2 * j] = pack_bf16x2(d0, d1);
+                        pd[8 + 2 * j + 1] = pack_bf16x2(d2, d3);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pd[e] = 0u;
+                }
+                tmem_st16(tST, pd);
+                sts_u4(dsrow + (((2 * cq) ^ (rowid & 7)) << 4), pd[8], pd[9], pd[10], pd[11]);
+                sts_u4(dsrow + (((2 * cq + 1) ^ (rowid & 7)) << 4), pd[12], pd[13], pd[14], pd[15]);
             }
-            // P^T over columns [16 cg, 16 cg + 8), dS^T over [16 cg + 8, 16 cg + 16): this warp's own S^T columns
-            tmem_st16(tST, pd);
-            // dS^T row to shared memory for dQ^T: 16-byte chunks 2 cg, 2 cg + 1 of the 128-byte row, swizzled
-            const uint32_t dsrow = sbase + L::kDS + (c & 1) * 16384 + rowid * 128;
-            sts_u4(dsrow + (((2 * cg) ^ (rowid & 7)) << 4), pd[8], pd[9], pd[10], pd[11]);
-            sts_u4(dsrow + (((2 * cg + 1) ^ (rowid & 7)) << 4), pd[12], pd[13], pd[14], pd[15]);
             tmem_wait_st();
             fence_async_smem();
             tc_fence_before();
@@ -359,17 +359,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         SegWalk wk;
         wk.init(u_begin, u_end, u2_begin, u2_end, rowT, bo);
         for (int c = 0; c < nchunk; ++c) {
-            const int st = c % kStages;
             if (!__all_sync(0xffffffffu,
-                            mbar_wait(bar_df + 8 * st, (c / kStages) & 1, status, kSiteDQFull, abort_flag)))
+                            mbar_wait(bar_df + 8 * (c & 1), (c >> 1) & 1, status, kSiteDQFull, abort_flag)))
                 break;
             tc_fence_after();
             uint32_t v[32], w[32];
-            tmem_ld32(tmem + kColST + st * 64 + lane_off, v);
-            tmem_ld32(tmem + kColST + st * 64 + lane_off + 32, w);
+            tmem_ld32(tmem + kColDP + (c & 1) * 64 + lane_off, v);
+            tmem_ld32(tmem + kColDP + (c & 1) * 64 + lane_off + 32, w);
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(bar_de + 8 * st);
+            mbar_arrive(bar_de + 8 * (c & 1));
             // the staging tile is free once the previous reduce has read it
             if (leader) bulk_wait_read_all();
             named_bar_sync(1, 128);

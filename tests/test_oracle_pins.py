@@ -712,3 +712,33 @@ def test_audio_norms_closed_forms_and_exact_sums():
         assert abs(Decimal(a[r]) - exact) / exact < Decimal("1e-14")
     # the batch and grid axes are kept
     assert oracle.audio_norms(hb.reshape(2, 3, 257)).shape == (2, 3)
+
+
+def test_selection_validity_check_accepts_oracle_rows_and_rejects_planted_mistakes():
+    """The check the GPU parity tests apply to a selection row that differs
+    from the oracle's at a near-tie: every oracle row passes it, and a row with
+    a planted mistake fails it (its best block dropped; one block too many)."""
+    import copy
+    from test_parity_gpu import valid_selection
+    w = scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=2, planted=2)
+    inp = make_inputs(w, 3)
+    Qb, Kb, Vb = (bf16_bits(x[0]) for x in (inp.Q, inp.K, inp.V))
+    pl = oracle.plan(Qb, Kb, Vb, inp.a[0].numpy(), w.T, w.H, w.W, w.heads, w.head_dim, w.top_k,
+                     float(np.float32(w.top_p)), 0.0)
+    dropped = extra = 0
+    for h in range(w.heads):
+        for i in range(pl.nb):
+            row = pl.cols[h, i, :pl.cnt[h, i]]
+            valid_selection(w, pl, h, i, row)
+            z = pl.Qbar[h, i] @ pl.Kbar[h, :pl.nb].T / np.sqrt(w.head_dim)
+            best = int(np.argmax(z))
+            with pytest.raises(AssertionError):
+                valid_selection(w, pl, h, i, np.sort(row[row != best]))
+            dropped += 1
+            if len(row) < pl.nb:
+                out = np.setdiff1d(np.arange(pl.nb), row)
+                nxt = out[np.argmax(z[out])]
+                with pytest.raises(AssertionError):
+                    valid_selection(w, pl, h, i, np.sort(np.append(row, nxt)))
+                extra += 1
+    assert dropped > 0 and extra > 0
