@@ -74,8 +74,8 @@ struct Layout {
     static constexpr uint32_t kVec = kDS + 2 * 16384;        // stage s: -LSE [64] f32 then Delta [64] f32
     static constexpr uint32_t kDQ = kVec + kStages * 512;    // dQ staging tile [64 queries][D] f32 (128-B aligned)
     static constexpr uint32_t kBars = kDQ + 64 * D * 4;
-    // kv, q_full[3], q_empty[3], s_full[2], p_full[2], dq_full[2], dq_empty[2], done
-    static constexpr uint32_t kNumBars = 16;
+    // kv, q_full[kStages], q_empty[kStages], s_full[2], p_full[2], dq_full[2], dq_empty[2], done
+    static constexpr uint32_t kNumBars = 10 + 2 * kStages;
     // then per stage the column mask of its query chunk in a shared tile
     static constexpr uint32_t kMaskS = kBars + kNumBars * 8 + 16;
     static constexpr uint32_t kBytes = kMaskS + 16;
