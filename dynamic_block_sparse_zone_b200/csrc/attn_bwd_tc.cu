@@ -39,11 +39,16 @@
 // chunks, odd chunks), so one group's TMEM loads and stores overlap the other
 // group's exponentials.  In a group each warp owns one TMEM lane quadrant (32
 // key rows) and 32 query columns, taken as two 16-column halves, and does its
-// arithmetic in packed fp32 pairs.
+// arithmetic in packed fp32 pairs.  The group issues its own products: a
+// named barrier closes the group's softmax of a chunk, and the group's first
+// warp issues dQ^T, dV, dK of that chunk and S^T, dP^T of the chunk two ahead
+// (no hand-off to a separate MMA warp).  The two groups' dV and dK products
+// accumulate into the same TMEM columns in whatever order they execute, so dK
+// and dV start from zero (written by the drain warps before the first chunk).
 // Warp roles (704 threads): warp 0 TMA producer (K, V once; Q, dO, LSE,
-// Delta per chunk into a three-stage ring; LSE is kept negated, in log2 units), warp 1
-// MMA issuer, warps 2..17 softmax, warps 18..21 dQ drain (one head-dim row
-// each).
+// Delta per chunk into a three-stage ring; LSE is kept negated, in log2
+// units), warp 1 idle, warps 2..17 softmax and MMA issue, warps 18..21 dQ
+// drain (one head-dim row each).
 #include <cuda.h>
 
 #include "tc_common.cuh"
@@ -74,8 +79,8 @@ struct Layout {
     static constexpr uint32_t kVec = kDS + 2 * 16384;        // stage s: -LSE [64] f32 then Delta [64] f32
     static constexpr uint32_t kDQ = kVec + kStages * 512;    // dQ staging tile [64 queries][D] f32 (128-B aligned)
     static constexpr uint32_t kBars = kDQ + 64 * D * 4;
-    // kv, q_full[kStages], q_empty[kStages], s_full[2], p_full[2], dq_full[2], dq_empty[2], done
-    static constexpr uint32_t kNumBars = 10 + 2 * kStages;
+    // kv, q_full[kStages], q_empty[kStages], s_full[2], dq_full[2], dq_empty[2], done
+    static constexpr uint32_t kNumBars = 8 + 2 * kStages;
     // then per stage the column mask of its query chunk in a shared tile
     static constexpr uint32_t kMaskS = kBars + kNumBars * 8 + 16;
     static constexpr uint32_t kBytes = kMaskS + 16;
@@ -94,7 +99,7 @@ __device__ __forceinline__ void mma_over_d(uint32_t d_tmem, uint64_t adesc, uint
         mma_ss4<2, 4, 6, 2, 4, 6>(d_tmem, adesc, bdesc, idesc, 0u);
 }
 
-enum { kSiteKV = 11, kSiteQFull, kSiteQEmpty, kSiteS, kSiteP, kSiteDQFull, kSiteDQEmpty, kSiteDone };
+enum { kSiteKV = 11, kSiteQFull, kSiteQEmpty, kSiteS, kSiteDQFull = 16, kSiteDQEmpty, kSiteDone };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -131,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const uint32_t bar_kv = sbase + L::kBars;
     const uint32_t bar_qf = bar_kv + 8, bar_qe = bar_qf + 8 * kStages, bar_sf = bar_qe + 8 * kStages;
-    const uint32_t bar_pf = bar_sf + 16, bar_df = bar_pf + 16, bar_de = bar_df + 16;
+    const uint32_t bar_df = bar_sf + 16, bar_de = bar_df + 16;
     const uint32_t bar_done = bar_de + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBars + L::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kBars + L::kNumBars * 8 + 8);
@@ -146,11 +151,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int s = 0; s < 2; ++s) {
                 mbar_init(bar_sf + 8 * s, 1);
-                mbar_init(bar_pf + 8 * s, 32 * kSoftmaxWarps / 2);
                 mbar_init(bar_df + 8 * s, 1);
                 mbar_init(bar_de + 8 * s, 128);
             }
-            mbar_init(bar_done, 1);
+            mbar_init(bar_done, 2);
             *abort_flag = 0;
             mbar_fence_init();
             prefetch_map(&tmQ);
@@ -168,6 +172,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int rowbase = bh * g.N;
+    if (warp >= 2 + kSoftmaxWarps) {  // dK, dV start from zero: both groups' products accumulate
+        const uint32_t lo = (uint32_t)((warp & 3) * 32) << 16;
+        uint32_t z[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) z[e] = 0u;
+#pragma unroll 1
+        for (int q = 0; q < 16; ++q) tmem_st16(tmem + kColDK + q * 16 + lo, z);
+        tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -208,53 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(bar_kv, 0, status, kSiteKV, abort_flag);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (nchunk > 0) {  // the whole warp runs the issue loop; elect.sync picks one lane
-            constexpr uint32_t idST = idesc_bf16(128, 64, false);          // K-major A and B
-            constexpr uint32_t idAcc = idesc_bf16(128, D, true);           // A from TMEM, B MN-major
-            constexpr uint32_t idDQ = idesc_bf16(128, 64, true, true);     // A and B MN-major
-            bool ok = __all_sync(0xffffffffu, mbar_wait(bar_kv, 0, status, kSiteKV, abort_flag));
-            // S^T and dP^T of chunk c into ST[c & 1] and DP[c & 1]; dP^T waits
-            // for the drain of chunk c - 2 to have read its dQ^T out of DP[c & 1]
-            auto issue_sdp = [&](int c) -> bool {
-                const int st = c % kStages;
-                if (!__all_sync(0xffffffffu, mbar_wait(bar_qf + 8 * st, (c / kStages) & 1, status, kSiteQFull, abort_flag))) return false;
-                tc_fence_after();
-                const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + L::kHalves * L::kQHalf;
-                mma_over_d<D>(tmem + kColST + (c & 1) * 64, sdesc(sbase + L::kK, 16, 1024), sdesc(sQ, 16, 1024), idST);
-                if (c >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar_de + 8 * (c & 1), ((c - 2) >> 1) & 1, status,
-                                                                 kSiteDQEmpty, abort_flag)))
-                    return false;
-                tc_fence_after();
-                mma_over_d<D>(tmem + kColDP + (c & 1) * 64, sdesc(sbase + L::kV, 16, 1024), sdesc(sO, 16, 1024), idST);
-                mma_commit(bar_sf + 8 * (c & 1));
-                return true;
-            };
-            if (ok) ok = issue_sdp(0);
-            if (ok && nchunk > 1) ok = issue_sdp(1);
-            for (int c = 0; ok && c < nchunk; ++c) {
-                const int st = c % kStages;
-                if (!__all_sync(0xffffffffu, mbar_wait(bar_pf + 8 * (c & 1), (c >> 1) & 1, status, kSiteP, abort_flag))) break;
-                tc_fence_after();
-                const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + L::kHalves * L::kQHalf;
-                const uint32_t tST = tmem + kColST + (c & 1) * 64;
-                const uint32_t sDS = sbase + L::kDS + (c & 1) * 16384;
-                // dQ^T first, into the consumed dP^T buffer; K^T and dS^T
-                // MN-major: k-step kk (16 keys) 2048 B further in both
-                mma_ss8<128, 256, 384, 512, 640, 768, 896, 128, 256, 384, 512, 640, 768, 896>(
-                    tmem + kColDP + (c & 1) * 64, sdesc(sbase + L::kK, L::kKVHalf, 1024), sdesc(sDS, 8192, 1024), idDQ,
-                    0u);
-                mma_commit(bar_df + 8 * (c & 1));
-                const uint32_t acc = (c > 0) ? 1u : 0u;
-                // k-step kk of P^T / dS^T: columns 16 kk (+8 for dS^T);
-                // of dO / Q: 16 rows = 2048 B further
-                mma_ts4x2<16, 32, 48, 128, 256, 384>(tmem + kColDV, tST, sdesc(sO, L::kQHalf, 1024), tmem + kColDK,
-                                                      tST + 8, sdesc(sQ, L::kQHalf, 1024), idAcc, acc);
-                mma_commit(bar_qe + 8 * st);
-                if (c + 2 < nchunk && !issue_sdp(c + 2)) break;
-            }
-            mma_commit(bar_done);
-        }
+        // no role: the softmax groups issue their own products
     } else if (warp < 2 + kSoftmaxWarps) {
         // ------------------------------------------------------------ softmax (key rows)
         const int quad = warp & 3;               // TMEM lane quadrant this warp may access
@@ -266,60 +236,103 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool live = rowid < kvalid;
         const int half = shared_tile ? (quad >> 1) : 0;  // which key block's rows (warp-uniform)
         bool ok = true;
+        const bool issuer = ((warp - 2) & 7) == 0;  // the group's first warp issues its products
+        constexpr uint32_t idST = idesc_bf16(128, 64, false);
+        constexpr uint32_t idAcc = idesc_bf16(128, D, true);
+        constexpr uint32_t idDQ = idesc_bf16(128, 64, true, true);
+        // S^T and dP^T of chunk c into ST[c & 1] and DP[c & 1]; dP^T waits for the
+        // drain of chunk c - 2 to have read its dQ^T out of DP[c & 1]
+        auto issue_sdp = [&](int c) -> bool {
+            const int st = c % kStages;
+            if (!__all_sync(0xffffffffu, mbar_wait(bar_qf + 8 * st, (c / kStages) & 1, status, kSiteQFull, abort_flag))) return false;
+            tc_fence_after();
+            const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + L::kHalves * L::kQHalf;
+            mma_over_d<D>(tmem + kColST + (c & 1) * 64, sdesc(sbase + L::kK, 16, 1024), sdesc(sQ, 16, 1024), idST);
+            if (c >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar_de + 8 * (c & 1), ((c - 2) >> 1) & 1, status,
+                                                             kSiteDQEmpty, abort_flag)))
+                return false;
+            tc_fence_after();
+            mma_over_d<D>(tmem + kColDP + (c & 1) * 64, sdesc(sbase + L::kV, 16, 1024), sdesc(sO, 16, 1024), idST);
+            mma_commit(bar_sf + 8 * (c & 1));
+            return true;
+        };
+        if (issuer && grp < nchunk) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_kv, 0, status, kSiteKV, abort_flag));
+            if (ok) ok = issue_sdp(grp);
+        }
+        // every warp of the group passes exactly one named barrier per chunk, on
+        // every path, so a failed wait cannot leave the others blocked
         for (int c = grp; c < nchunk; c += 2) {
             const int st = c % kStages;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * (c & 1), (c >> 1) & 1, status, kSiteS, abort_flag) &&
-                                             mbar_wait(bar_qf + 8 * st, (c / kStages) & 1, status, kSiteQFull,
-                                                       abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            const bool act = live && ((mask_s[st] >> half) & 1u);
-            const uint32_t dsrow = sbase + L::kDS + (c & 1) * 16384 + rowid * 128;
+            if (ok)
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * (c & 1), (c >> 1) & 1, status, kSiteS, abort_flag) &&
+                                                 mbar_wait(bar_qf + 8 * st, (c / kStages) & 1, status, kSiteQFull,
+                                                           abort_flag));
+            if (ok) {
+                tc_fence_after();
+                const bool act = live && ((mask_s[st] >> half) & 1u);
+                const uint32_t dsrow = sbase + L::kDS + (c & 1) * 16384 + rowid * 128;
 #pragma unroll 1
-            for (int sub = 0; sub < 2; ++sub) {
-                const int cq = 2 * cg2 + sub;  // 16 query columns [16 cq, 16 cq + 16)
-                const uint32_t tST = tmem + kColST + (c & 1) * 64 + 16 * cq + lane_off;
-                uint32_t sv[16], dv[16];
-                tmem_ld16(tST, sv);
-                tmem_ld16(tmem + kColDP + (c & 1) * 64 + 16 * cq + lane_off, dv);
-                const uint32_t vec = sbase + L::kVec + st * 512 + cq * 64;
-                float4 N4[4], D4[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    N4[j] = lds_f4(vec + 16 * j);
-                    D4[j] = lds_f4(vec + 256 + 16 * j);
-                }
-                tmem_wait_ld();
-                uint32_t pd[16];
-                if (act) {
-                    const uint64_t s2 = splat2(scale_log2);
+                for (int sub = 0; sub < 2; ++sub) {
+                    const int cq = 2 * cg2 + sub;  // 16 query columns [16 cq, 16 cq + 16)
+                    const uint32_t tST = tmem + kColST + (c & 1) * 64 + 16 * cq + lane_off;
+                    uint32_t sv[16], dv[16];
+                    tmem_ld16(tST, sv);
+                    tmem_ld16(tmem + kColDP + (c & 1) * 64 + 16 * cq + lane_off, dv);
+                    const uint32_t vec = sbase + L::kVec + st * 512 + cq * 64;
+                    float4 N4[4], D4[4];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        const int q = 4 * j;
-                        float x0, x1, x2, x3, d0, d1, d2, d3;
-                        fma2(__uint_as_float(sv[q]), __uint_as_float(sv[q + 1]), s2, pair2(N4[j].x, N4[j].y), x0, x1);
-                        fma2(__uint_as_float(sv[q + 2]), __uint_as_float(sv[q + 3]), s2, pair2(N4[j].z, N4[j].w), x2, x3);
-                        const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
-                        mul_sub2(p0, p1, __uint_as_float(dv[q]), __uint_as_float(dv[q + 1]), D4[j].x, D4[j].y, d0, d1);
-                        mul_sub2(p2, p3, __uint_as_float(dv[q + 2]), __uint_as_float(dv[q + 3]), D4[j].z, D4[j].w, d2, d3);
-                        pd[2 * j] = pack_bf16x2(p0, p1);
-                        pd[2 * j + 1] = pack_bf16x2(p2, p3);
-                        pd[8 + 2 * j] = pack_bf16x2(d0, d1);
-                        pd[8 + 2 * j + 1] = pack_bf16x2(d2, d3);
+                        N4[j] = lds_f4(vec + 16 * j);
+                        D4[j] = lds_f4(vec + 256 + 16 * j);
                     }
-                } else {
+                    tmem_wait_ld();
+                    uint32_t pd[16];
+                    if (act) {
+                        const uint64_t s2 = splat2(scale_log2);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pd[e] = 0u;
+                        for (int j = 0; j < 4; ++j) {
+                            const int q = 4 * j;
+                            float x0, x1, x2, x3, d0, d1, d2, d3;
+                            fma2(__uint_as_float(sv[q]), __uint_as_float(sv[q + 1]), s2, pair2(N4[j].x, N4[j].y), x0, x1);
+                            fma2(__uint_as_float(sv[q + 2]), __uint_as_float(sv[q + 3]), s2, pair2(N4[j].z, N4[j].w), x2, x3);
+                            const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+                            mul_sub2(p0, p1, __uint_as_float(dv[q]), __uint_as_float(dv[q + 1]), D4[j].x, D4[j].y, d0, d1);
+                            mul_sub2(p2, p3, __uint_as_float(dv[q + 2]), __uint_as_float(dv[q + 3]), D4[j].z, D4[j].w, d2, d3);
+                            pd[2 * j] = pack_bf16x2(p0, p1);
+                            pd[2 * j + 1] = pack_bf16x2(p2, p3);
+                            pd[8 + 2 * j] = pack_bf16x2(d0, d1);
+                            pd[8 + 2 * j + 1] = pack_bf16x2(d2, d3);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pd[e] = 0u;
+                    }
+                    tmem_st16(tST, pd);
+                    sts_u4(dsrow + (((2 * cq) ^ (rowid & 7)) << 4), pd[8], pd[9], pd[10], pd[11]);
+                    sts_u4(dsrow + (((2 * cq + 1) ^ (rowid & 7)) << 4), pd[12], pd[13], pd[14], pd[15]);
                 }
-                tmem_st16(tST, pd);
-                sts_u4(dsrow + (((2 * cq) ^ (rowid & 7)) << 4), pd[8], pd[9], pd[10], pd[11]);
-                sts_u4(dsrow + (((2 * cq + 1) ^ (rowid & 7)) << 4), pd[12], pd[13], pd[14], pd[15]);
+                tmem_wait_st();
+                fence_async_smem();
             }
-            tmem_wait_st();
-            fence_async_smem();
             tc_fence_before();
-            mbar_arrive(bar_pf + 8 * (c & 1));
+            named_bar_sync(2 + grp, 32 * kSoftmaxWarps / 2);
+            if (issuer && ok && !*abort_flag) {
+                tc_fence_after();
+                const uint32_t sQ = sbase + L::kQ0 + st * L::kStage, sO = sQ + L::kHalves * L::kQHalf;
+                const uint32_t tSTc = tmem + kColST + (c & 1) * 64;
+                const uint32_t sDS = sbase + L::kDS + (c & 1) * 16384;
+                mma_ss8<128, 256, 384, 512, 640, 768, 896, 128, 256, 384, 512, 640, 768, 896>(
+                    tmem + kColDP + (c & 1) * 64, sdesc(sbase + L::kK, L::kKVHalf, 1024), sdesc(sDS, 8192, 1024), idDQ,
+                    0u);
+                mma_commit(bar_df + 8 * (c & 1));
+                mma_ts4x2<16, 32, 48, 128, 256, 384>(tmem + kColDV, tSTc, sdesc(sO, L::kQHalf, 1024), tmem + kColDK,
+                                                      tSTc + 8, sdesc(sQ, L::kQHalf, 1024), idAcc, 1u);
+                mma_commit(bar_qe + 8 * st);
+                if (c + 2 < nchunk) ok = issue_sdp(c + 2);
+            }
         }
+        if (issuer) mma_commit(bar_done);  // both groups' products: done counts two commits
         // epilogue: column groups 0, 1 write halves of dK (scaled), 2, 3 halves of dV
         if (ok && nchunk > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, status, kSiteDone, abort_flag));
         if (ok) {
