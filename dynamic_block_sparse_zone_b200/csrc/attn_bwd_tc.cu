@@ -43,8 +43,10 @@
 // named barrier closes the group's softmax of a chunk, and the group's first
 // warp issues dQ^T, dV, dK of that chunk and S^T, dP^T of the chunk two ahead
 // (no hand-off to a separate MMA warp).  The two groups' dV and dK products
-// accumulate into the same TMEM columns in whatever order they execute, so dK
-// and dV start from zero (written by the drain warps before the first chunk).
+// accumulate into the same TMEM columns: a token passed between the groups
+// keeps them in chunk order (deterministic sums), and dK and dV start from zero
+// (written by the drain warps before the first chunk), so no product needs to
+// know whether it is the first.
 // Warp roles (704 threads): warp 0 TMA producer (K, V once; Q, dO, LSE,
 // Delta per chunk into a three-stage ring; LSE is kept negated, in log2
 // units), warp 1 idle, warps 2..17 softmax and MMA issue, warps 18..21 dQ
@@ -79,8 +81,8 @@ struct Layout {
     static constexpr uint32_t kVec = kDS + 2 * 16384;        // stage s: -LSE [64] f32 then Delta [64] f32
     static constexpr uint32_t kDQ = kVec + kStages * 512;    // dQ staging tile [64 queries][D] f32 (128-B aligned)
     static constexpr uint32_t kBars = kDQ + 64 * D * 4;
-    // kv, q_full[kStages], q_empty[kStages], s_full[2], dq_full[2], dq_empty[2], done
-    static constexpr uint32_t kNumBars = 8 + 2 * kStages;
+    // kv, q_full[kStages], q_empty[kStages], s_full[2], dq_full[2], dq_empty[2], done, token
+    static constexpr uint32_t kNumBars = 9 + 2 * kStages;
     // then per stage the column mask of its query chunk in a shared tile
     static constexpr uint32_t kMaskS = kBars + kNumBars * 8 + 16;
     static constexpr uint32_t kBytes = kMaskS + 16;
@@ -99,7 +101,7 @@ __device__ __forceinline__ void mma_over_d(uint32_t d_tmem, uint64_t adesc, uint
         mma_ss4<2, 4, 6, 2, 4, 6>(d_tmem, adesc, bdesc, idesc, 0u);
 }
 
-enum { kSiteKV = 11, kSiteQFull, kSiteQEmpty, kSiteS, kSiteDQFull = 16, kSiteDQEmpty, kSiteDone };
+enum { kSiteKV = 11, kSiteQFull, kSiteQEmpty, kSiteS, kSiteDQFull = 16, kSiteDQEmpty, kSiteDone, kSiteToken };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -138,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_qf = bar_kv + 8, bar_qe = bar_qf + 8 * kStages, bar_sf = bar_qe + 8 * kStages;
     const uint32_t bar_df = bar_sf + 16, bar_de = bar_df + 16;
     const uint32_t bar_done = bar_de + 16;
+    const uint32_t bar_tok = bar_done + 8;  // dV, dK of a chunk have been issued
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBars + L::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kBars + L::kNumBars * 8 + 8);
     volatile uint32_t *mask_s = reinterpret_cast<volatile uint32_t *>(smem + L::kMaskS);
@@ -155,6 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_init(bar_de + 8 * s, 128);
             }
             mbar_init(bar_done, 2);
+            mbar_init(bar_tok, 1);
             *abort_flag = 0;
             mbar_fence_init();
             prefetch_map(&tmQ);
@@ -326,10 +330,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem + kColDP + (c & 1) * 64, sdesc(sbase + L::kK, L::kKVHalf, 1024), sdesc(sDS, 8192, 1024), idDQ,
                     0u);
                 mma_commit(bar_df + 8 * (c & 1));
-                mma_ts4x2<16, 32, 48, 128, 256, 384>(tmem + kColDV, tSTc, sdesc(sO, L::kQHalf, 1024), tmem + kColDK,
-                                                      tSTc + 8, sdesc(sQ, L::kQHalf, 1024), idAcc, 1u);
-                mma_commit(bar_qe + 8 * st);
-                if (c + 2 < nchunk) ok = issue_sdp(c + 2);
+                // dV, dK in chunk order (the other group has issued those of chunk c - 1),
+                // so that their fp32 sums do not depend on the two groups' timing
+                if (c >= 1)
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_tok, (c - 1) & 1, status, kSiteToken, abort_flag));
+                if (ok) {
+                    tc_fence_after();
+                    mma_ts4x2<16, 32, 48, 128, 256, 384>(tmem + kColDV, tSTc, sdesc(sO, L::kQHalf, 1024),
+                                                          tmem + kColDK, tSTc + 8, sdesc(sQ, L::kQHalf, 1024), idAcc, 1u);
+                    tc_fence_before();
+                    if (lane == 0) mbar_arrive(bar_tok);
+                    __syncwarp();
+                    mma_commit(bar_qe + 8 * st);
+                    if (c + 2 < nchunk) ok = issue_sdp(c + 2);
+                }
             }
         }
         if (issuer) mma_commit(bar_done);  // both groups' products: done counts two commits
