@@ -1298,3 +1298,28 @@ def test_per_kernel_timers_count_launches_and_reset():
     plan.fwd()
     torch.cuda.synchronize()
     assert all(n == 0 for _, n in plan.read_timing().values())
+
+
+def test_backward_is_deterministic():
+    """dK and dV of repeated backward passes over the same plan and inputs are
+    bit-identical: the two softmax groups of the backward kernel issue their dV
+    and dK products in chunk order, so the fp32 sums are formed in one order.
+    dQ is summed by reduce-adds from many key tiles in whatever order they land,
+    so it agrees up to fp32 summation order (at most one bf16 ulp after
+    rounding)."""
+    P = _lib()
+    w = scaled(WORKLOADS["dynamic_16x32x32"], backward=True)
+    inp = make_inputs(w, 21)
+    Q, K, V, a, dO = (x.cuda() for x in (inp.Q, inp.K, inp.V, inp.a, inp.dO))
+    plan = P.PrismPlan(P.params_for(w))
+    plan.build(Q, K, V, a)
+    O, lse = plan.fwd()
+    runs = [[t.clone() for t in plan.bwd(O, dO)] for _ in range(3)]
+    torch.cuda.synchronize()
+    plan.check()
+    for r in runs[1:]:
+        assert torch.equal(r[1], runs[0][1]), "dK differs between runs"
+        assert torch.equal(r[2], runs[0][2]), "dV differs between runs"
+        diff = (r[0].float() - runs[0][0].float()).abs()
+        assert bool((diff <= 2.0 ** -7 * runs[0][0].float().abs() + 1e-6).all()), float(diff.max())
+    plan.close()
