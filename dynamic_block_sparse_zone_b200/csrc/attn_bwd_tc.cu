@@ -143,6 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_tok = bar_done + 8;  // dV, dK of a chunk have been issued
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBars + L::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kBars + L::kNumBars * 8 + 8);
+    volatile int *drain_fail = abort_flag + 1;  // a drain warp's wait failed
     volatile uint32_t *mask_s = reinterpret_cast<volatile uint32_t *>(smem + L::kMaskS);
 
     if (warp == 0) {
@@ -160,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar_done, 2);
             mbar_init(bar_tok, 1);
             *abort_flag = 0;
+            *drain_fail = 0;
             mbar_fence_init();
             prefetch_map(&tmQ);
             prefetch_map(&tmK);
@@ -387,8 +389,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         wk.init(u_begin, u_end, u2_begin, u2_end, rowT, bo);
         for (int c = 0; c < nchunk; ++c) {
             if (!__all_sync(0xffffffffu,
-                            mbar_wait(bar_df + 8 * (c & 1), (c >> 1) & 1, status, kSiteDQFull, abort_flag)))
+                            mbar_wait(bar_df + 8 * (c & 1), (c >> 1) & 1, status, kSiteDQFull, abort_flag))) {
+                // meet the other drain warps at this chunk's first barrier and leave with them
+                if (lane == 0) *drain_fail = 1;
+                named_bar_sync(1, 128);
                 break;
+            }
             tc_fence_after();
             uint32_t v[32], w[32];
             tmem_ld32(tmem + kColDP + (c & 1) * 64 + lane_off, v);
@@ -399,6 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the staging tile is free once the previous reduce has read it
             if (leader) bulk_wait_read_all();
             named_bar_sync(1, 128);
+            // the same answer in every drain warp: they write the flag only before this barrier
+            if (*drain_fail) break;
             const uint32_t stage = sbase + L::kDQ + d * 4;
             if (d < D) {  // head_dim 64: dQ^T rows 64..127 are padding
 #pragma unroll
