@@ -428,10 +428,12 @@ __global__ void __launch_bounds__(1024) k_zone_decide(Geo g, const double *__res
 
 // ---------------------------------------------------------------------------
 // K3: block-contiguous, head-major copies of Q, K, V and the fp64 block means
-// of Q and K.  One CTA per block; a thread owns 8 channels of one head.
+// of Q and K.  One CTA per (block, slice of kPPThreads x 8 channels); a thread
+// owns 8 channels of one head and walks the block's tokens.
 // ---------------------------------------------------------------------------
+constexpr int kPPThreads = 128;
 struct BlockGeom {
-    int off, B, t0, h0, w0, bT, bH, bW;
+    int off, B, t0, h0, w0, bT, bH, bW, eH, eW;  // edges bT x bH x bW; bH = 2^eH, bW = 2^eW
 };
 
 __device__ __forceinline__ BlockGeom block_geom(const Geo &g, const int *blk_off_b, const int *zone_shape_b, int j) {
@@ -440,9 +442,11 @@ __device__ __forceinline__ BlockGeom block_geom(const Geo &g, const int *blk_off
     r.B = blk_off_b[j + 1] - r.off;
     const int m = r.off / kZoneVol;
     const int s = zone_shape_b[m];
+    r.eH = c_shape_exp[s][1];
+    r.eW = c_shape_exp[s][2];
     r.bT = 1 << c_shape_exp[s][0];
-    r.bH = 1 << c_shape_exp[s][1];
-    r.bW = 1 << c_shape_exp[s][2];
+    r.bH = 1 << r.eH;
+    r.bW = 1 << r.eW;
     const int lidx = (r.off - m * kZoneVol) / r.B;
     const int nW = 8 / r.bW, nH = 8 / r.bH;
     const int iw = lidx % nW, ih = (lidx / nW) % nH, it = lidx / (nW * nH);
@@ -454,14 +458,14 @@ __device__ __forceinline__ BlockGeom block_geom(const Geo &g, const int *blk_off
 }
 
 __device__ __forceinline__ int block_token(const Geo &g, const BlockGeom &bg, int r) {
-    const int tt = r / (bg.bH * bg.bW), hh = (r / bg.bW) % bg.bH, ww = r % bg.bW;
+    const int tt = r >> (bg.eH + bg.eW), hh = (r >> bg.eW) & (bg.bH - 1), ww = r & (bg.bW - 1);
     return ((bg.t0 + tt) * g.H + (bg.h0 + hh)) * g.W + (bg.w0 + ww);
 }
 
 // kPerm: the blocks are runs of an existing permutation (Hilbert-order plans),
 // which is read instead of derived from the zone shapes and written.
 template <bool kPerm>
-__global__ void __launch_bounds__(384) k_permute_pool(const __nv_bfloat16 *__restrict__ Q,
+__global__ void __launch_bounds__(kPPThreads, 5) k_permute_pool(const __nv_bfloat16 *__restrict__ Q,
                                                       const __nv_bfloat16 *__restrict__ K,
                                                       const __nv_bfloat16 *__restrict__ V, Geo g,
                                                       const int *__restrict__ nb, const int *__restrict__ blk_off,
@@ -469,7 +473,8 @@ __global__ void __launch_bounds__(384) k_permute_pool(const __nv_bfloat16 *__res
                                                       __nv_bfloat16 *__restrict__ Qp, __nv_bfloat16 *__restrict__ Kp,
                                                       __nv_bfloat16 *__restrict__ Vp, double *__restrict__ Qbar,
                                                       double *__restrict__ Kbar) {
-    const int j = blockIdx.x, b = blockIdx.y;
+    const int nslice = (g.C / 8 + kPPThreads - 1) / kPPThreads;
+    const int j = blockIdx.x / nslice, slice = blockIdx.x % nslice, b = blockIdx.y;
     if (j >= nb[b]) return;
     BlockGeom bg;
     if constexpr (kPerm) {
@@ -478,13 +483,15 @@ __global__ void __launch_bounds__(384) k_permute_pool(const __nv_bfloat16 *__res
         bg.B = bo[j + 1] - bo[j];
     } else {
         bg = block_geom(g, blk_off + (size_t)b * (g.nbmax + 1), zone_shape + (size_t)b * g.M, j);
-        for (int r = threadIdx.x; r < bg.B; r += blockDim.x)
-            perm[(size_t)b * g.N + bg.off + r] = block_token(g, bg, r);
+        if (slice == 0)
+            for (int r = threadIdx.x; r < bg.B; r += blockDim.x)
+                perm[(size_t)b * g.N + bg.off + r] = block_token(g, bg, r);
     }
     const int *pb = perm + (size_t)b * g.N + bg.off;
     const int G = g.C / 8;
     const double inv = 1.0 / (double)bg.B;  // B is a power of two: exact
-    for (int grp = threadIdx.x; grp < G; grp += blockDim.x) {
+    const int grp = slice * kPPThreads + threadIdx.x;
+    if (grp < G) {
         const int hd = (grp * 8) / g.D, d0 = (grp * 8) % g.D;
         const size_t bh = (size_t)b * g.heads + hd;
         double sq[8], sk[8];
@@ -1039,17 +1046,15 @@ prism_status launch_plan_given(Plan &pl, const void *Qv, const void *Kv, const v
                                 static_cast<const __nv_bfloat16 *>(Vv), st);
 }
 
-static int permute_pool_threads(const Geo &g) { return g.C / 8 >= 384 ? 384 : ((g.C / 8 + 31) / 32) * 32; }
-
 static void launch_permute_pool(Plan &pl, const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
                                 cudaStream_t st) {
     const Geo &g = pl.g;
     TimerScope ts(pl, kTPermutePool, st);
     if (pl.p.hilbert_block)
-        k_permute_pool<true><<<dim3(g.nbmax, g.batch), permute_pool_threads(g), 0, st>>>(
+        k_permute_pool<true><<<dim3((g.C / 8 + kPPThreads - 1) / kPPThreads * g.nbmax, g.batch), kPPThreads, 0, st>>>(
             Q, K, V, g, pl.nb, pl.blk_off, pl.zone_shape, pl.perm, pl.Qp, pl.Kp, pl.Vp, pl.Qbar, pl.Kbar);
     else
-        k_permute_pool<false><<<dim3(g.nbmax, g.batch), permute_pool_threads(g), 0, st>>>(
+        k_permute_pool<false><<<dim3((g.C / 8 + kPPThreads - 1) / kPPThreads * g.nbmax, g.batch), kPPThreads, 0, st>>>(
             Q, K, V, g, pl.nb, pl.blk_off, pl.zone_shape, pl.perm, pl.Qp, pl.Kp, pl.Vp, pl.Qbar, pl.Kbar);
 }
 
