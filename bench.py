@@ -364,12 +364,12 @@ def run_ours(args, rank, world, dev):
         ach = kernels[dom]["tflops"]
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                 "frac": round(ach / peak, 4), "peak_kind": f"bf16 dense sustained ({peak_src})",
-                "traffic": traffic_for(dom)}
+                "traffic": traffic_for(dom, w)}
     else:
         peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         ach = kernels[dom].get("gbs", 0.0)
         roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
-                "frac": round(ach / peak, 4), "peak_kind": f"HBM copy ({peak_src})", "traffic": traffic_for(dom)}
+                "frac": round(ach / peak, 4), "peak_kind": f"HBM copy ({peak_src})", "traffic": traffic_for(dom, w)}
     # one timer record per kernel launch, except the CSR/CSC scope (9 kernels)
     launches_per_step = sum(n * (9 if k == "csr_csc" else 1) for k, (t, n) in timing.items()) // max(args.steps, 1)
     result = {
@@ -430,9 +430,10 @@ def measure_fp64_peak(dev):
     return round(2.0 * n ** 3 / (best * 1e-3) / 1e12, 2)
 
 
-def traffic_for(kernel):
+def traffic_for(kernel, w):
     """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
-    the current kernel source."""
+    the current kernel source and for this workload at this size (a record
+    lists the workloads whose launch of the kernel it covers)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -441,6 +442,8 @@ def traffic_for(kernel):
             d = json.load(f)
         rec = d.get(kernel)
         if not rec:
+            return None
+        if w.name not in rec["workloads"] or w.heads != rec["heads"] or w.batch != rec["batch"]:
             return None
         import hashlib
         src = os.path.join(ROOT, "dynamic_block_sparse_zone_b200", "csrc", rec["source"])

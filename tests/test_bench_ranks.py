@@ -50,3 +50,18 @@ def test_aggregate_value_is_weak_scaling():
     two = bench.aggregate_value(352e12, 5, 2, 2500.0)
     assert two == pytest.approx(2 * one)
     assert one == pytest.approx(352e12 * 5 / 2.5 / 1e12)
+
+
+def test_traffic_record_applies_only_to_its_workload():
+    """The per-launch DRAM bytes of the committed ncu capture are reported only
+    for the workload and size they were taken on, and only while the kernel
+    source is the one captured."""
+    import bench
+    from dynamic_block_sparse_zone_b200.synth import WORKLOADS, scaled
+    train = WORKLOADS["latent2k_train_24x96x160"]
+    rec = bench.traffic_for("attn_bwd", train)
+    assert rec is None or rec > 0
+    assert bench.traffic_for("attn_bwd", scaled(train, heads=2)) is None
+    assert bench.traffic_for("attn_bwd", WORKLOADS["latent720p_24x48x80"]) is None
+    assert bench.traffic_for("attn_fwd", WORKLOADS["tiny_8x16x16"]) is None
+    assert bench.traffic_for("no_such_kernel", train) is None
