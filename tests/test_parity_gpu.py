@@ -652,6 +652,8 @@ EDGE_CASES = {
     # cap binding at head_dim 64
     "cap_d64": scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=2, head_dim=64, planted=2, top_k=2,
                       top_p=0.95, max_frac=0.1),
+    # 1280 channels: the permute-and-pool kernel's second 1024-channel slice is a quarter full
+    "ragged_channel_slice": scaled(WORKLOADS["dynamic_16x32x32"], T=8, H=16, W=32, heads=10, planted=2),
 }
 
 
