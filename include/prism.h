@@ -232,8 +232,11 @@ PRISM_API prism_status prism_attn_fwd_taylor(prism_plan *plan, void *O, float *l
  *   dS = P (dP - rowsum(dO * O)), dQ = dS K / sqrt(D), dK = dS^T Q / sqrt(D).
  * O is the forward's output and dO the incoming gradient (device, bf16, user
  * layout); dQ, dK, dV are written (device, bf16, user layout).  dQ is summed
- * in fp32 before its bf16 rounding.  Returns PRISM_ERR_STATE if no forward
- * ran since the last build.                                                */
+ * in fp32 before its bf16 rounding.  Repeated calls on the same plan and
+ * inputs give bit-identical dK and dV (their fp32 sums are formed in one
+ * order); dQ's partial sums from different key tiles are added in the order
+ * they arrive, so dQ can differ in its last bit.  Returns PRISM_ERR_STATE if
+ * no forward ran since the last build.                                     */
 PRISM_API prism_status prism_attn_bwd(prism_plan *plan, const void *O, const void *dO, void *dQ, void *dK,
                             void *dV, void *stream);
 
