@@ -65,3 +65,15 @@ def test_traffic_record_applies_only_to_its_workload():
     assert bench.traffic_for("attn_bwd", WORKLOADS["latent720p_24x48x80"]) is None
     assert bench.traffic_for("attn_fwd", WORKLOADS["tiny_8x16x16"]) is None
     assert bench.traffic_for("no_such_kernel", train) is None
+
+
+def test_nvidia_smi_id_follows_cuda_visible_devices(monkeypatch):
+    """The clock sampler asks nvidia-smi about the GPU the process runs on:
+    torch's device i is the i-th entry of CUDA_VISIBLE_DEVICES."""
+    import bench
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "3,5")
+    assert bench.smi_device_id(0) == "3" and bench.smi_device_id(1) == "5"
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "GPU-1b2c, GPU-9f00")
+    assert bench.smi_device_id(1) == "GPU-9f00"
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES")
+    assert bench.smi_device_id(2) == "2"
